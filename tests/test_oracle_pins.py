@@ -1,0 +1,361 @@
+"""Pins of the CPU oracle to facts fixed outside itself: library routines
+(statistics.NormalDist, math.fsum, torch casts, numpy searchsorted), closed
+forms, the pages' worked example and storage figures, invariants the pages
+state, and brute force on tiny inputs.  CPU only."""
+import math
+import statistics
+import struct
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from qlora_block_absmax_b200 import synth
+from tests.conftest import read_golden
+
+PSTAR = 0.5 * ((1 - 1 / 30) + (1 - 1 / 32))
+
+
+def f32(x):
+    return struct.unpack("<f", struct.pack("<f", x))[0]
+
+
+# ---------------------------------------------------------------- code book
+
+def test_codebook_matches_independent_quantile_routine():
+    """Same definition evaluated with statistics.NormalDist.inv_cdf (a
+    different inverse-CDF algorithm) agrees bit for bit in fp32."""
+    _, c32 = oracle.codebook()
+    nd = statistics.NormalDist()
+    neg = [-nd.inv_cdf(0.5 + (PSTAR - 0.5) * (k / 7)) for k in range(7, 0, -1)]
+    pos = [nd.inv_cdf(0.5 + (PSTAR - 0.5) * (k / 8)) for k in range(1, 9)]
+    v = np.array(neg + [0.0] + pos)
+    v = v / np.abs(v).max()
+    assert np.array_equal(v.astype(np.float32), c32)
+
+
+def test_codebook_equal_share_of_bell_curve():
+    """'How NF4 works': each level covers an equal share of the normal curve --
+    mapping the levels back through the normal CDF gives equally spaced
+    probabilities (8 steps above zero, 7 below)."""
+    c64, _ = oracle.codebook()
+    zmax = statistics.NormalDist().inv_cdf(PSTAR)
+    cdf = [0.5 * (1 + math.erf(c * zmax / math.sqrt(2))) for c in c64]
+    pos = np.diff(cdf[7:])
+    neg = np.diff(cdf[:8])
+    assert np.allclose(pos, (PSTAR - 0.5) / 8, rtol=0, atol=1e-12)
+    assert np.allclose(neg, (PSTAR - 0.5) / 7, rtol=0, atol=1e-12)
+
+
+def test_codebook_shape():
+    c64, c32 = oracle.codebook()
+    assert c32[0] == -1.0 and c32[15] == 1.0
+    assert struct.pack("<f", c32[7]) == b"\x00\x00\x00\x00"  # exact +0
+    assert np.all(np.diff(c32) > 0)
+    assert (c32 < 0).sum() == 7 and (c32 > 0).sum() == 8
+    # finer marks near zero, coarser far out ('How NF4 works')
+    gaps_pos = np.diff(c64[7:])
+    gaps_neg = np.diff(c64[:8])[::-1]        # from zero outward
+    assert np.all(np.diff(gaps_pos) > 0) and np.all(np.diff(gaps_neg) > 0)
+
+
+# ---------------------------------------------------------------- bf16
+
+def test_bf16_rounding_matches_torch_cast():
+    r = synth.rng(7)
+    x = np.concatenate([
+        r.standard_normal(20000).astype(np.float32) * np.float32(3.0),
+        (r.standard_normal(2000) * 1e30).astype(np.float32),
+        np.array([0.0, -0.0, 1.0, 3.0e38, -3.0e38, 1e-40, -1e-40], np.float32),
+    ])
+    # exact ties: bf16 value plus half an ulp
+    ties = (synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(x[:500])).view(np.uint32) | 0x8000).view(np.float32)
+    x = np.concatenate([x, ties])
+    want = synth.f32_to_bf16_bits(x)
+    got = np.array([oracle.bf16_rn(float(v)) for v in x], np.uint16)
+    assert np.array_equal(got, want)
+
+
+# ---------------------------------------------------------------- nearest code
+
+def _midpoints():
+    _, c32 = oracle.codebook()
+    return np.array([(float(c32[i]) + float(c32[i + 1])) / 2 for i in range(15)])  # exact in fp64
+
+
+def test_nearest_code_equals_midpoint_count_near_every_midpoint():
+    """argmin-distance (the oracle) == number of exact midpoints strictly below
+    x (numpy searchsorted), exhaustively for the 2x64 fp32 values around every
+    midpoint and for random values in [-1, 1]."""
+    mids = _midpoints()
+    xs = []
+    for m in mids:
+        b = np.array([m], np.float32).view(np.int32)[0]
+        for d in range(-64, 65):
+            xs.append(np.array([b + d], np.int32).view(np.float32)[0])
+    xs = np.concatenate([np.array(xs, np.float32),
+                         synth.rng(11).uniform(-1, 1, 20000).astype(np.float32),
+                         np.array([-1, 1, 0, -0.0], np.float32)])
+    want = np.searchsorted(mids, xs.astype(np.float64), side="left")
+    got = np.array([oracle.nearest_code(float(x)) for x in xs])
+    assert np.array_equal(got, want)
+
+
+def test_nearest_code_special_values():
+    _, c32 = oracle.codebook()
+    for i, c in enumerate(c32):
+        assert oracle.nearest_code(float(c)) == i
+    assert oracle.nearest_code(0.0) == 7 and oracle.nearest_code(-0.0) == 7
+    assert oracle.nearest_code(1.0) == 15 and oracle.nearest_code(-1.0) == 0
+
+
+# ---------------------------------------------------------------- level-1 quantize
+
+def _brute_quantize(w, bs):
+    """numpy brute force: fp32 division by the block absmax, argmin |x - c|."""
+    _, c32 = oracle.codebook()
+    n = w.size
+    codes = np.zeros(n, np.uint8)
+    absmax = np.zeros((n + bs - 1) // bs, np.float32)
+    for b in range(absmax.size):
+        blk = w[b * bs:(b + 1) * bs]
+        a = np.abs(blk).max()
+        absmax[b] = a
+        if a == 0:
+            codes[b * bs:b * bs + blk.size] = 7
+            continue
+        x = (blk / a).astype(np.float32)
+        d = np.abs(x.astype(np.float64)[:, None] - c32.astype(np.float64)[None, :])
+        codes[b * bs:b * bs + blk.size] = np.argmin(d, axis=1)  # first minimum = lower index
+    if n % 2:
+        codes = np.append(codes, 7)
+    packed = (codes[0::2] << 4) | codes[1::2]
+    return packed.astype(np.uint8), absmax
+
+
+@pytest.mark.parametrize("n,bs", [(1, 64), (63, 64), (64, 64), (65, 64), (127, 64), (4097, 64), (1000, 32)])
+def test_quantize_brute_force_tiny(n, bs):
+    w = synth.normal_weights((n,), 100 + n)
+    w[::17] = 0.0
+    p, a = oracle.quantize(w, bs)
+    bp, ba = _brute_quantize(w, bs)
+    assert np.array_equal(a, ba)
+    assert np.array_equal(p, bp)
+
+
+def test_quantize_packing_order_hand_example():
+    """Step 4: two codes per byte; first element in the high nibble; odd tail
+    padded with the zero code."""
+    w = np.array([1.0, -1.0, 0.0, 0.5, 0.25], np.float32)
+    p, a = oracle.quantize(w, 64)
+    # 0.5 lies between c12 = 0.4407 and c13 = 0.5626, nearer c12; 0.25 nearest c10 = 0.2461
+    assert a.tolist() == [1.0]
+    assert p.tolist() == [0xF0, 0x7C, 0xA7]
+
+
+def test_quantize_invariants():
+    w = synth.normal_weights((64 * 500,), 5)
+    w[64 * 3:64 * 4] = 0.0              # all-zero block
+    w[64 * 7 + 5] = -0.0
+    p, a = oracle.quantize(w, 64)
+    codes = np.empty(w.size, np.uint8)
+    codes[0::2] = p >> 4
+    codes[1::2] = p & 15
+    blocks = w.reshape(-1, 64)
+    cb = codes.reshape(-1, 64)
+    assert np.array_equal(a, np.abs(blocks).max(axis=1))
+    for b in range(blocks.shape[0]):
+        if a[b] == 0:
+            assert np.all(cb[b] == 7)
+            continue
+        j = np.argmax(np.abs(blocks[b]))
+        assert cb[b, j] == (15 if blocks[b, j] > 0 else 0)   # max element -> +-1 code
+    assert np.all(codes[w == 0] == 7)                          # zeros -> zero code
+
+
+def test_quantize_dequantize_roundtrip_is_identity_on_codes():
+    w = synth.normal_weights((64 * 2000 + 31,), 9)
+    p, a = oracle.quantize(w, 64)
+    wh = oracle.dequantize(p, a, w.size, 64)
+    p2, a2 = oracle.quantize(wh, 64)
+    assert np.array_equal(p2, p) and np.array_equal(a2, a)
+
+
+def test_quantize_bf16_path_is_exact_widening():
+    wb = synth.normal_weights((64 * 100 + 3,), 21, dtype="bf16")
+    p1, a1 = oracle.quantize(wb, 64)
+    p2, a2 = oracle.quantize(synth.bf16_bits_to_f32(wb), 64)
+    assert np.array_equal(p1, p2) and np.array_equal(a1, a2)
+
+
+# ---------------------------------------------------------------- exact sum
+
+def test_exact_sum_matches_fsum():
+    r = synth.rng(3)
+    cases = [
+        np.abs(r.standard_normal(10000)).astype(np.float32) * np.float32(0.05),
+        (r.standard_normal(5000) * np.exp(r.uniform(-60, 60, 5000))).astype(np.float32),
+        np.array([1e30, 1.0, -1e30, 1e-30], np.float32),
+        np.array([3.0e38, 3.0e38, -3.0e38], np.float32),
+        np.array([1e-45, 2e-45, -1e-45, 1e-40], np.float32),
+        np.array([2.0 ** 60, 1.0, 2.0 ** -60], np.float32),
+        np.zeros(7, np.float32),
+    ]
+    for a in cases:
+        assert oracle.exact_sum(a) == math.fsum(a.astype(np.float64).tolist())
+
+
+# ---------------------------------------------------------------- E4M3
+
+def test_e4m3_decode_matches_torch_float8():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn)
+    ref = codes.to(torch.float32).numpy()
+    got = np.array([oracle.e4m3_decode(c) for c in range(256)], np.float32)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan) and nan.sum() == 2
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert got[0x7e] == 448.0 and len(set(got[~nan].tolist())) == 253
+
+
+def test_e4m3_encode_matches_torch_rne_inside_range():
+    vals = np.array(sorted(set(oracle.e4m3_decode(c) for c in range(0x7f))), np.float64)
+    mids = (vals[:-1] + vals[1:]) / 2                       # exact ties
+    r = synth.rng(4)
+    ys = np.concatenate([vals, -vals, mids, -mids,
+                         r.uniform(-448, 448, 5000), r.standard_normal(3000) * 0.01,
+                         np.nextafter(mids, 0), np.nextafter(mids, 1000)]).astype(np.float32)
+    ys = ys[np.abs(ys) <= 448]
+    ref = torch.from_numpy(ys).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_encode(float(y)) for y in ys], np.uint8)
+    assert np.array_equal(got, ref)
+
+
+def test_e4m3_encode_saturates():
+    for y in [448.0, 449.0, 464.0, 1e6, 3e38]:
+        assert oracle.e4m3_encode(y) == 0x7e and oracle.e4m3_encode(-y) == 0xfe
+
+
+# ---------------------------------------------------------------- second level / worked example
+
+def test_worked_example_int8():
+    g = read_golden("worked_example_int8.txt")
+    w = np.array(g["weights"], np.float32)
+    q, scale = oracle.blockwise_8bit(w, 256, oracle.DQ_INT8)
+    assert scale[0] == np.float32(g["absmax"][0])
+    assert np.array_equal(q.view(np.int8).astype(int), np.array(g["codes"], int))
+    assert np.allclose(w / scale[0], g["scaled"], atol=1e-7)
+    for code, approx in zip(g["dequant_of"], g["dequant_approx"]):
+        v = oracle.blockwise_8bit_value(int(np.int8(code).view(np.uint8)), float(scale[0]), oracle.DQ_INT8)
+        assert abs(v - approx) < 1e-4
+    errs = [abs(oracle.blockwise_8bit_value(int(qq), float(scale[0]), oracle.DQ_INT8) - float(ww))
+            for qq, ww in zip(q[:2], w[:2])]
+    assert np.allclose(errs, g["error_approx"], atol=5e-4)
+
+
+@pytest.mark.parametrize("code,top", [(oracle.DQ_E4M3, 0x7e), (oracle.DQ_INT8, 127)])
+def test_blockwise_8bit_block_max_maps_to_top_code(code, top):
+    v = synth.rng(8).standard_normal(256 * 9 + 77).astype(np.float32)
+    q, scale = oracle.blockwise_8bit(v, 256, code)
+    for g in range(scale.size):
+        blk = v[g * 256:(g + 1) * 256]
+        j = np.argmax(np.abs(blk))
+        assert scale[g] == np.abs(blk).max()
+        want = top if blk[j] > 0 else (top | 0x80 if code == oracle.DQ_E4M3 else (256 - top))
+        assert q[g * 256 + j] == want
+        assert oracle.blockwise_8bit_value(int(q[g * 256 + j]), float(scale[g]), code) == blk[j]
+
+
+def test_double_quant_mean_and_reconstruction_bound():
+    w = synth.add_outliers(synth.normal_weights((64 * 4096,), 31), 32)
+    _, a = oracle.quantize(w, 64)
+    for code, rel in [(oracle.DQ_E4M3, 2.0 ** -4), (oracle.DQ_INT8, 1.0 / 254)]:
+        q, scale, mean = oracle.double_quant(a, 256, code)
+        exact = sum(Fraction(float(x)) for x in a) / a.size          # exact mean
+        assert mean == f32(float(Fraction(math.fsum(a.astype(np.float64))) / a.size))
+        assert abs(Fraction(mean) - exact) <= abs(exact) * Fraction(2) ** -24
+        ah = oracle.absmax_reconstruct(q, scale, mean, 256, code)
+        for g in range(scale.size):
+            blk = slice(g * 256, (g + 1) * 256)
+            # 8-bit grid error: half a step of the code around the block absmax of residuals
+            assert np.all(np.abs(ah[blk] - a[blk]) <= scale[g] * rel * 1.0001 + 1e-7)
+
+
+def test_double_quant_degenerate_constant_absmax():
+    a = np.full(1000, 0.375, np.float32)
+    q, scale, mean = oracle.double_quant(a, 256, oracle.DQ_E4M3)
+    assert mean == 0.375 and np.all(scale == 0) and np.all(q == 0)
+    assert np.all(oracle.absmax_reconstruct(q, scale, mean) == a)
+
+
+# ---------------------------------------------------------------- storage arithmetic
+
+def storage_bytes(n, bs=64, dq=True, dq_bs=256):
+    nb = -(-n // bs)
+    if not dq:
+        return -(-n // 2) + 4 * nb
+    return -(-n // 2) + nb + 4 * (-(-nb // dq_bs)) + 4
+
+
+def test_storage_matches_pages_figures():
+    g = read_golden("storage_claims.txt")
+    n = 4096 * 4096
+    bits = 8 * storage_bytes(n) / n
+    assert abs(bits - (4 + 8 / 64 + 32 / (64 * 256) + 32 / n)) < 1e-9   # ~4.127 (+ one fp32 mean)
+    saving = 8 * (storage_bytes(n, dq=False) - storage_bytes(n)) / n
+    assert abs(saving - g["dq_saving_bits_per_param"][0]) < 0.05        # "about 0.4"
+    params = synth.LLAMA8B_LAYERS * sum(r * c for _, r, c in synth.LLAMA8B_LAYER)
+    total = synth.LLAMA8B_LAYERS * sum(storage_bytes(r * c) for _, r, c in synth.LLAMA8B_LAYER)
+    gb = total / 1e9
+    assert g["int4_7b_gb_before_scales"][0] < gb < g["nf4_7b_gb"][0]   # 3.5 GB + small overhead, < ~4 GB
+    assert abs(params * 2 / 1e9 - g["fp16_7b_gb"][0]) < 0.2 * g["fp16_7b_gb"][0]
+
+
+# ---------------------------------------------------------------- dequantize
+
+def test_dequantize_against_numpy_products():
+    w = synth.normal_weights((64 * 300 + 5,), 41)
+    p, a = oracle.quantize(w, 64)
+    _, c32 = oracle.codebook()
+    codes = np.empty(p.size * 2, np.uint8)
+    codes[0::2] = p >> 4
+    codes[1::2] = p & 15
+    codes = codes[:w.size]
+    want = (c32[codes] * np.repeat(a, 64)[:w.size]).astype(np.float32)
+    got = oracle.dequantize(p, a, w.size, 64)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+    got16 = oracle.dequantize(p, a, w.size, 64, "bf16")
+    assert np.array_equal(got16, synth.f32_to_bf16_bits(want))
+    # block max reconstructs to +-absmax exactly; zero codes give 0
+    blocks = w[:64 * 300].reshape(-1, 64)
+    j = np.argmax(np.abs(blocks), axis=1)
+    assert np.array_equal(np.abs(got[:64 * 300].reshape(-1, 64)[np.arange(300), j]), a[:300])
+    assert np.all(got[codes == 7] == 0)
+
+
+# ---------------------------------------------------------------- matmul
+
+def test_matmul_one_hot_columns_and_numpy_dot():
+    N, K = 48, 192
+    w = synth.normal_weights((N, K), 51)
+    p, a = oracle.quantize(w, 64)
+    wc = synth.bf16_bits_to_f32(oracle.dequantize(p, a, N * K, 64, "bf16")).reshape(N, K)
+    # one-hot activations pick columns of the 16-bit expanded weight exactly
+    eye = synth.f32_to_bf16_bits(np.eye(K, dtype=np.float32)[[0, 5, 63, 64, 191]])
+    y = oracle.matmul(p, a, N, K, eye)
+    assert np.array_equal(y, wc[:, [0, 5, 63, 64, 191]].T.astype(np.float64))
+    x = synth.activations((3, K), 52)
+    y = oracle.matmul(p, a, N, K, x)
+    ref = synth.bf16_bits_to_f32(x).astype(np.float64) @ wc.astype(np.float64).T
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-15)
+    ys = oracle.matmul_sampled(p, a, N, K, x, np.array([0, 2, 1]), np.array([0, 47, 13]))
+    assert np.array_equal(ys, y[[0, 2, 1], [0, 47, 13]])
+
+
+def test_matmul_zero_codes_give_zero():
+    N, K = 16, 128
+    p = np.full(N * K // 2, 0x77, np.uint8)
+    a = np.ones(N * K // 64, np.float32)
+    x = synth.activations((2, K), 3)
+    assert np.all(oracle.matmul(p, a, N, K, x) == 0)
