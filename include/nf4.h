@@ -1,0 +1,169 @@
+/*
+ * nf4.h -- C ABI of libnf4: blockwise NF4 4-bit weight quantization with double
+ * quantization of the absmax constants, dequantization, and the 4-bit-weight x
+ * bf16-activation matmul that dequantizes on the fly (GEMV for decode, GEMM for
+ * prefill), for NVIDIA B200 (sm_100a).
+ *
+ * Method sources (web pages on bitsandbytes / QLoRA):
+ *   [bnb-tools] "bitsandbytes" (ozercemkelahmet.com/tools/bitsandbytes):
+ *               "How it works" Steps 1-5, "How NF4 works", "Double quantization",
+ *               "A worked example".
+ *   [bnb-tut]   "bitsandbytes quantization tutorial: 4-bit and 8-bit models"
+ *               (mljourney.com): "4-bit Loading with NF4", "How NF4 Works".
+ *
+ * Conventions for every entry point:
+ *   - Memory: all buffers are allocated and owned by the caller; the library
+ *     allocates nothing.  "device" pointers must point to memory of the
+ *     current CUDA device; "host" pointers to host memory.
+ *   - Execution: work is enqueued asynchronously on `stream` (a cudaStream_t;
+ *     NULL = legacy default stream).  Arguments are validated on the host
+ *     first; on any error nothing is launched and no buffer is touched.
+ *   - Alignment: device pointers must be 16-byte aligned unless stated
+ *     otherwise (NF4_ERR_MISALIGNED).
+ *   - Sizes: element counts are int64; 0 is valid and launches nothing.
+ *   - Inputs must be finite; NaN or Inf inputs give unspecified codes.
+ *   - No in-place operation: outputs must not overlap inputs.
+ *   - Errors: functions return an nf4_status and never throw or abort.
+ *     NF4_ERR_CUDA carries a launch failure; device-side waits that exceed
+ *     their bound set an error word read by nf4_check_device_error().
+ *   - Thread safety: every function is reentrant; concurrent calls on
+ *     different streams are independent.
+ */
+#ifndef NF4_H
+#define NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NF4_API __attribute__((visibility("default")))
+#else
+#define NF4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *nf4_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  NF4_OK = 0,
+  NF4_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad enum, short workspace */
+  NF4_ERR_MISALIGNED = 2,  /* a pointer breaks the stated alignment */
+  NF4_ERR_UNSUPPORTED = 3, /* a valid but unimplemented configuration */
+  NF4_ERR_ARCH = 4,        /* current device is not sm_100 (B200 class) */
+  NF4_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
+  NF4_ERR_TIMEOUT = 6      /* a device-side wait gave up (see nf4_check_device_error) */
+} nf4_status;
+
+typedef enum { NF4_F32 = 0, NF4_BF16 = 1 } nf4_dtype;
+
+/* 8-bit code of the double-quantized absmax constants.
+ * NF4_DQ_E4M3: OCP FP8 E4M3 ("float8", [bnb-tut] "How NF4 Works"), top code 448.
+ * NF4_DQ_INT8: linear int8 -127..127, round half away from zero ([bnb-tools]
+ *              "A worked example"), top code 127. */
+typedef enum { NF4_DQ_E4M3 = 0, NF4_DQ_INT8 = 1 } nf4_dq_code;
+
+/* A quantized weight W of shape [rows, cols] (row-major, rows = output
+ * features N, cols = input features K), flattened for quantization so the
+ * level-1 blocks run along a row.  All pointers are device pointers.
+ *   packed        ceil(rows*cols/2) bytes, two codes per byte, element 2j in
+ *                 the high nibble of byte j ([bnb-tools] Step 4)
+ *   absmax        nb = ceil(rows*cols/blocksize) fp32 block scales, or NULL
+ *                 when the weight is double-quantized
+ *   absmax_q      nb 8-bit codes of the mean-removed scales (double quant)
+ *   absmax_scale  ceil(nb/dq_blocksize) fp32 second-level block absmax values
+ *   absmax_mean   1 fp32: the mean removed before second-level quantization
+ *   blocksize     64 (only value implemented); dq_blocksize 256; dq_code nf4_dq_code */
+typedef struct {
+  const uint8_t *packed;
+  const float *absmax;
+  const uint8_t *absmax_q;
+  const float *absmax_scale;
+  const float *absmax_mean;
+  int64_t rows, cols;
+  int32_t blocksize, dq_blocksize, dq_code;
+} nf4_weight;
+
+/* Blockwise NF4 quantization, [bnb-tools] "How it works" Steps 1-4.
+ * For each block of `blocksize` consecutive elements (the last may be short):
+ * a = max|w|; x = fp32(w / a); code = index of the nearest NF4 level (ties to
+ * the lower index; every code 7 when a == 0); two codes per byte.
+ *   src         device, n elements of src_dtype (NF4_F32 or NF4_BF16); 16-byte aligned
+ *   packed_out  device, ceil(n/2) bytes; an odd tail's low nibble is 7 (zero code)
+ *   absmax_out  device, ceil(n/blocksize) fp32 (the level-1 scales a)
+ * blocksize must be 64 (else NF4_ERR_UNSUPPORTED). */
+NF4_API nf4_status nf4_quantize(const void *src, int32_t src_dtype, int64_t n, int32_t blocksize,
+                        uint8_t *packed_out, float *absmax_out, nf4_stream_t stream);
+
+/* Double quantization of the fp32 absmax array, [bnb-tut] "How NF4 Works"
+ * (scale constants quantized from float32 to float8) and [bnb-tools] "Double
+ * quantization".  mu = fp32(fp64(exact sum of absmax) / nb) (one per tensor);
+ * r = fp32(absmax - mu); per block of dq_blocksize: m = max|r| (stored in
+ * scale_out), y = fp32(fp32(r / m) * Q), q = E4M3 round-to-nearest-even with
+ * saturation (Q = 448) or int8 round-half-away clamped to +-127 (Q = 127).
+ *   absmax      device, nb fp32 (finite, any sign)
+ *   q_out       device, nb bytes (E4M3 bits, or int8 two's complement)
+ *   scale_out   device, ceil(nb/dq_blocksize) fp32
+ *   mean_out    device, 1 fp32 (4-byte aligned)
+ *   workspace   device scratch of nf4_double_quant_workspace_bytes(nb) bytes,
+ *               16-byte aligned; its contents on entry are ignored
+ * dq_blocksize must be 256.  nb == 0 launches nothing and leaves mean_out unset. */
+NF4_API nf4_status nf4_double_quant(const float *absmax, int64_t nb, int32_t dq_blocksize, int32_t dq_code,
+                            uint8_t *q_out, float *scale_out, float *mean_out, void *workspace,
+                            size_t workspace_bytes, nf4_stream_t stream);
+NF4_API size_t nf4_double_quant_workspace_bytes(int64_t nb);
+
+/* Dequantization, [bnb-tools] Step 5 ("Dequantization": expand back to a higher
+ * precision with the scale and the code book).  With double quantization the
+ * scale is first reconstructed: a^ = fp32(fp32(fp32(dec(q)/Q) * m) + mu).
+ * w^ = fp32(code[idx] * a^); out = w^ (NF4_F32) or bf16_rn(w^) (NF4_BF16).
+ *   w    weight descriptor (rows*cols elements; rows/cols need no alignment)
+ *   out  device, rows*cols elements of out_dtype, 16-byte aligned */
+NF4_API nf4_status nf4_dequantize(const nf4_weight *w, void *out, int32_t out_dtype, nf4_stream_t stream);
+
+/* Decode GEMV, [bnb-tools] Step 5 (expand each block to 16-bit with its scale
+ * and the code book, then multiply) with bf16 compute ([bnb-tut] "4-bit
+ * Loading with NF4", bnb_4bit_compute_dtype=bfloat16):
+ *   y[b, n] = bf16_rn( sum_k Wc[n, k] * x[b, k] ),  Wc = bf16_rn(w^)
+ * accumulated in fp32 (order unspecified).
+ *   x  device bf16 [batch, cols] row-major;  y  device bf16 [batch, rows]
+ *   1 <= batch <= 8; cols % 64 == 0; rows % 16 == 0. */
+NF4_API nf4_status nf4_gemv(const nf4_weight *w, const void *x, int32_t batch, void *y, nf4_stream_t stream);
+
+/* Prefill GEMM, same arithmetic as nf4_gemv for m activation rows:
+ *   Y[m, n] = bf16_rn( sum_k Wc[n, k] * X[m, k] )
+ * on tcgen05 tensor cores (bf16 x bf16 -> fp32 in tensor memory).
+ *   x  device bf16 [m, cols];  y  device bf16 [m, rows];  m >= 1
+ *   cols % 64 == 0; rows % 128 == 0.
+ *   workspace  device scratch of nf4_gemm_workspace_bytes(w, m) bytes (may be
+ *              NULL when that size is 0), 16-byte aligned. */
+NF4_API nf4_status nf4_gemm(const nf4_weight *w, const void *x, int64_t m, void *y, void *workspace,
+                    size_t workspace_bytes, nf4_stream_t stream);
+NF4_API size_t nf4_gemm_workspace_bytes(const nf4_weight *w, int64_t m);
+
+/* Bytes of a quantized tensor of n elements: ceil(n/2) codes + either
+ * 4*ceil(n/blocksize) (fp32 absmax) or ceil(n/blocksize) 8-bit codes +
+ * 4*ceil(nb/dq_blocksize) + 4 (double quant).  Host only. */
+NF4_API size_t nf4_storage_bytes(int64_t n, int32_t blocksize, int32_t double_quant, int32_t dq_blocksize);
+
+/* Synchronizes `stream`, then reports and clears the device error word of the
+ * current device: NF4_OK, or NF4_ERR_TIMEOUT if a device-side bounded wait
+ * gave up since the last check; NF4_ERR_CUDA if the stream reports an error. */
+NF4_API nf4_status nf4_check_device_error(nf4_stream_t stream);
+
+/* Static string naming a status. Host only. */
+NF4_API const char *nf4_status_string(nf4_status s);
+
+/* The library's 16 NF4 levels (ascending, index 7 = 0.0f), copied to host
+ * memory `out`.  Host only. */
+NF4_API void nf4_code_table(float out[16]);
+
+/* 1 if the current CUDA device is sm_100 (B200 class), else 0. */
+NF4_API int32_t nf4_device_supported(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NF4_H */

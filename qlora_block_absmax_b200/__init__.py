@@ -1,0 +1,196 @@
+"""qlora_block_absmax_b200 -- blockwise NF4 quantization with double
+quantization, dequantization and the NF4-weight x bf16 matmul on B200.
+
+This module only marshals torch tensors (device memory, the current stream)
+into the C ABI of libnf4.so; every step of the computation runs in the
+library's sm_100a kernels.  There is no CPU path.
+
+Typical use:
+    qw = quantize_weight(W)            # W: [N, K] bf16/fp32 CUDA tensor
+    y = gemv(qw, x)                    # x: [B, K] bf16, B <= 8
+    Y = gemm(qw, X)                    # X: [M, K] bf16
+    W_hat = dequantize(qw, torch.bfloat16)
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import NF4_BF16, NF4_DQ_E4M3, NF4_DQ_INT8, NF4_F32, NF4Error
+
+__all__ = ["QuantizedWeight", "quantize", "double_quant", "quantize_weight", "dequantize", "gemv", "gemm",
+           "storage_bytes", "code_table", "check_device_error", "NF4Error", "library_path"]
+
+BLOCKSIZE = 64
+DQ_BLOCKSIZE = 256
+_DQ_CODES = {"e4m3": NF4_DQ_E4M3, "int8": NF4_DQ_INT8}
+
+
+def library_path() -> str:
+    _lib.load()
+    return _lib.LIB_PATH
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(stream: Optional[torch.cuda.Stream] = None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need_cuda(t: torch.Tensor, name: str) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+@dataclass
+class QuantizedWeight:
+    """A weight [rows, cols] in NF4: packed codes plus either fp32 block
+    scales (absmax) or the double-quantized record (absmax_q, absmax_scale,
+    absmax_mean)."""
+    packed: torch.Tensor
+    rows: int
+    cols: int
+    absmax: Optional[torch.Tensor] = None
+    absmax_q: Optional[torch.Tensor] = None
+    absmax_scale: Optional[torch.Tensor] = None
+    absmax_mean: Optional[torch.Tensor] = None
+    dq_code: int = NF4_DQ_E4M3
+    blocksize: int = BLOCKSIZE
+    dq_blocksize: int = DQ_BLOCKSIZE
+
+    @property
+    def double_quant(self) -> bool:
+        return self.absmax is None
+
+    def descriptor(self) -> _lib.NF4Weight:
+        return _lib.NF4Weight(_ptr(self.packed), _ptr(self.absmax), _ptr(self.absmax_q), _ptr(self.absmax_scale),
+                              _ptr(self.absmax_mean), self.rows, self.cols, self.blocksize, self.dq_blocksize,
+                              self.dq_code)
+
+    def storage_bytes(self) -> int:
+        return storage_bytes(self.rows * self.cols, self.double_quant)
+
+
+def quantize(w: torch.Tensor, blocksize: int = BLOCKSIZE, out=None, stream=None):
+    """Level-1 NF4 quantization of a flattened fp32/bf16 tensor.
+    Returns (packed uint8 [ceil(n/2)], absmax fp32 [ceil(n/64)])."""
+    _need_cuda(w, "w")
+    if w.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("quantize takes float32 or bfloat16")
+    n = w.numel()
+    if out is None:
+        packed = torch.empty((n + 1) // 2, dtype=torch.uint8, device=w.device)
+        absmax = torch.empty((n + blocksize - 1) // blocksize, dtype=torch.float32, device=w.device)
+    else:
+        packed, absmax = out
+    st = _lib.load().nf4_quantize(_ptr(w), NF4_BF16 if w.dtype == torch.bfloat16 else NF4_F32, n, blocksize,
+                                  _ptr(packed), _ptr(absmax), _stream(stream))
+    _lib.check(st, "nf4_quantize")
+    return packed, absmax
+
+
+def double_quant(absmax: torch.Tensor, code: str = "e4m3", dq_blocksize: int = DQ_BLOCKSIZE, out=None,
+                 workspace: Optional[torch.Tensor] = None, stream=None):
+    """Second-level quantization of the fp32 absmax array.
+    Returns (q uint8 [nb], scale fp32 [ceil(nb/256)], mean fp32 [1])."""
+    _need_cuda(absmax, "absmax")
+    lib = _lib.load()
+    nb = absmax.numel()
+    if out is None:
+        q = torch.empty(nb, dtype=torch.uint8, device=absmax.device)
+        scale = torch.empty((nb + dq_blocksize - 1) // dq_blocksize, dtype=torch.float32, device=absmax.device)
+        mean = torch.empty(1, dtype=torch.float32, device=absmax.device)
+    else:
+        q, scale, mean = out
+    ws_bytes = lib.nf4_double_quant_workspace_bytes(nb)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=absmax.device)
+    st = lib.nf4_double_quant(_ptr(absmax), nb, dq_blocksize, _DQ_CODES[code], _ptr(q), _ptr(scale), _ptr(mean),
+                              _ptr(workspace), workspace.numel(), _stream(stream))
+    _lib.check(st, "nf4_double_quant")
+    return q, scale, mean
+
+
+def quantize_weight(w: torch.Tensor, use_double_quant: bool = True, code: str = "e4m3",
+                    stream=None) -> QuantizedWeight:
+    """Quantize a 2-D weight [rows, cols] (nn.Linear layout: out x in)."""
+    if w.dim() != 2:
+        raise ValueError("quantize_weight takes a 2-D [rows, cols] tensor")
+    packed, absmax = quantize(w, stream=stream)
+    qw = QuantizedWeight(packed=packed, rows=w.shape[0], cols=w.shape[1], absmax=absmax)
+    if use_double_quant:
+        q, scale, mean = double_quant(absmax, code, stream=stream)
+        qw = QuantizedWeight(packed=packed, rows=w.shape[0], cols=w.shape[1], absmax_q=q, absmax_scale=scale,
+                             absmax_mean=mean, dq_code=_DQ_CODES[code])
+    return qw
+
+
+def dequantize(qw: QuantizedWeight, dtype: torch.dtype = torch.float32, out=None, stream=None) -> torch.Tensor:
+    """Expand to fp32 or bf16 [rows, cols]."""
+    if dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("dequantize produces float32 or bfloat16")
+    if out is None:
+        out = torch.empty(qw.rows, qw.cols, dtype=dtype, device=qw.packed.device)
+    d = qw.descriptor()
+    st = _lib.load().nf4_dequantize(ctypes.byref(d), _ptr(out), NF4_BF16 if dtype == torch.bfloat16 else NF4_F32,
+                                    _stream(stream))
+    _lib.check(st, "nf4_dequantize")
+    return out
+
+
+def gemv(qw: QuantizedWeight, x: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+    """y[b, n] = bf16(sum_k Wc[n, k] x[b, k]) for x bf16 [B, cols], 1 <= B <= 8."""
+    _need_cuda(x, "x")
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be bfloat16")
+    x2 = x.reshape(-1, qw.cols)
+    if out is None:
+        out = torch.empty(x2.shape[0], qw.rows, dtype=torch.bfloat16, device=x.device)
+    d = qw.descriptor()
+    st = _lib.load().nf4_gemv(ctypes.byref(d), _ptr(x2), x2.shape[0], _ptr(out), _stream(stream))
+    _lib.check(st, "nf4_gemv")
+    return out
+
+
+def gemm(qw: QuantizedWeight, x: torch.Tensor, out=None, workspace: Optional[torch.Tensor] = None,
+         stream=None) -> torch.Tensor:
+    """Y[m, n] = bf16(sum_k Wc[n, k] X[m, k]) for X bf16 [M, cols]."""
+    _need_cuda(x, "x")
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be bfloat16")
+    x2 = x.reshape(-1, qw.cols)
+    m = x2.shape[0]
+    lib = _lib.load()
+    d = qw.descriptor()
+    if out is None:
+        out = torch.empty(m, qw.rows, dtype=torch.bfloat16, device=x.device)
+    ws_bytes = lib.nf4_gemm_workspace_bytes(ctypes.byref(d), m)
+    if workspace is None and ws_bytes:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=x.device)
+    st = lib.nf4_gemm(ctypes.byref(d), _ptr(x2), m, _ptr(out), _ptr(workspace),
+                      workspace.numel() if workspace is not None else 0, _stream(stream))
+    _lib.check(st, "nf4_gemm")
+    return out
+
+
+def storage_bytes(n: int, use_double_quant: bool = True) -> int:
+    return int(_lib.load().nf4_storage_bytes(n, BLOCKSIZE, 1 if use_double_quant else 0, DQ_BLOCKSIZE))
+
+
+def code_table() -> list:
+    buf = (ctypes.c_float * 16)()
+    _lib.load().nf4_code_table(buf)
+    return list(buf)
+
+
+def check_device_error(stream=None) -> None:
+    _lib.check(_lib.load().nf4_check_device_error(_stream(stream)), "device error word")

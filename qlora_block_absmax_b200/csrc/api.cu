@@ -1,0 +1,211 @@
+// api.cu -- extern "C" entry points of libnf4 (declared in include/nf4.h).
+// Host-side validation happens before any launch; kernels live in the other
+// translation units (quantize.cu, double_quant.cu, dequantize.cu, gemv.cu,
+// gemm_sm100.cu).
+#include <mutex>
+
+#include "../../include/nf4.h"
+#include "internal.h"
+#include "nf4_codebook.h"
+
+namespace {
+
+__device__ unsigned g_error_word;  // device-side error flags (nf4::kErrTimeout)
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+  int cc_major = 0;
+  unsigned* error_word = nullptr;
+};
+
+std::mutex g_mutex;
+DeviceInfo g_info[kMaxDevices];
+
+// Info of the current device, filled on first use.
+nf4_status device_info(DeviceInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NF4_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo& d = g_info[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return NF4_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+      return NF4_ERR_CUDA;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return NF4_ERR_CUDA;
+    d.error_word = static_cast<unsigned*>(p);
+    d.ready = true;
+  }
+  *out = d;
+  return d.cc_major == 10 ? NF4_OK : NF4_ERR_ARCH;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+nf4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? NF4_OK : NF4_ERR_CUDA; }
+
+// Common checks of a weight descriptor; fills the kernel-side scale view.
+nf4_status check_weight(const nf4_weight* w, nf4::Scales* s) {
+  if (w == nullptr || w->packed == nullptr) return NF4_ERR_INVALID_ARG;
+  if (w->rows < 0 || w->cols < 0) return NF4_ERR_INVALID_ARG;
+  if (w->blocksize != nf4::kBlock) return NF4_ERR_UNSUPPORTED;
+  if (!aligned(w->packed, 16)) return NF4_ERR_MISALIGNED;
+  if (w->absmax != nullptr) {
+    if (!aligned(w->absmax, 4)) return NF4_ERR_MISALIGNED;
+    *s = nf4::Scales{w->absmax, nullptr, nullptr, nullptr, 0};
+    return NF4_OK;
+  }
+  if (w->absmax_q == nullptr || w->absmax_scale == nullptr || w->absmax_mean == nullptr) return NF4_ERR_INVALID_ARG;
+  if (w->dq_blocksize != nf4::kDqBlock) return NF4_ERR_UNSUPPORTED;
+  if (w->dq_code != NF4_DQ_E4M3 && w->dq_code != NF4_DQ_INT8) return NF4_ERR_INVALID_ARG;
+  if (!aligned(w->absmax_scale, 4) || !aligned(w->absmax_mean, 4)) return NF4_ERR_MISALIGNED;
+  *s = nf4::Scales{nullptr, w->absmax_q, w->absmax_scale, w->absmax_mean, w->dq_code};
+  return NF4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* nf4_status_string(nf4_status s) {
+  switch (s) {
+    case NF4_OK: return "NF4_OK";
+    case NF4_ERR_INVALID_ARG: return "NF4_ERR_INVALID_ARG";
+    case NF4_ERR_MISALIGNED: return "NF4_ERR_MISALIGNED";
+    case NF4_ERR_UNSUPPORTED: return "NF4_ERR_UNSUPPORTED";
+    case NF4_ERR_ARCH: return "NF4_ERR_ARCH";
+    case NF4_ERR_CUDA: return "NF4_ERR_CUDA";
+    case NF4_ERR_TIMEOUT: return "NF4_ERR_TIMEOUT";
+  }
+  return "NF4_ERR_UNKNOWN";
+}
+
+void nf4_code_table(float out[16]) {
+  static const float code[16] = NF4_CODE_INIT;
+  for (int i = 0; i < 16; ++i) out[i] = code[i];
+}
+
+size_t nf4_storage_bytes(int64_t n, int32_t blocksize, int32_t double_quant, int32_t dq_blocksize) {
+  if (n <= 0 || blocksize <= 0) return 0;
+  const size_t nb = (size_t)((n + blocksize - 1) / blocksize);
+  size_t bytes = (size_t)((n + 1) / 2);
+  if (!double_quant) return bytes + 4 * nb;
+  if (dq_blocksize <= 0) return 0;
+  return bytes + nb + 4 * ((nb + dq_blocksize - 1) / dq_blocksize) + 4;
+}
+
+size_t nf4_double_quant_workspace_bytes(int64_t /*nb*/) { return nf4::kDoubleQuantWorkspace; }
+
+size_t nf4_gemm_workspace_bytes(const nf4_weight* w, int64_t m) {
+  if (w == nullptr || w->rows <= 0 || w->cols <= 0 || m <= 0) return 0;
+  return nf4::gemm_workspace_bytes(w->rows, w->cols, m);
+}
+
+int32_t nf4_device_supported(void) {
+  DeviceInfo d;
+  return device_info(&d) == NF4_OK ? 1 : 0;
+}
+
+nf4_status nf4_quantize(const void* src, int32_t src_dtype, int64_t n, int32_t blocksize, uint8_t* packed_out,
+                        float* absmax_out, nf4_stream_t stream) {
+  if (n < 0) return NF4_ERR_INVALID_ARG;
+  if (src_dtype != NF4_F32 && src_dtype != NF4_BF16) return NF4_ERR_INVALID_ARG;
+  if (blocksize != nf4::kBlock) return NF4_ERR_UNSUPPORTED;
+  if (n == 0) return NF4_OK;
+  if (src == nullptr || packed_out == nullptr || absmax_out == nullptr) return NF4_ERR_INVALID_ARG;
+  if (!aligned(src, 16) || !aligned(packed_out, 16) || !aligned(absmax_out, 4)) return NF4_ERR_MISALIGNED;
+  DeviceInfo d;
+  nf4_status st = device_info(&d);
+  if (st != NF4_OK) return st;
+  return from_cuda(nf4::launch_quantize(src, src_dtype == NF4_BF16, n, packed_out, absmax_out,
+                                        reinterpret_cast<cudaStream_t>(stream), d.num_sms));
+}
+
+nf4_status nf4_double_quant(const float* absmax, int64_t nb, int32_t dq_blocksize, int32_t dq_code, uint8_t* q_out,
+                            float* scale_out, float* mean_out, void* workspace, size_t workspace_bytes,
+                            nf4_stream_t stream) {
+  if (nb < 0) return NF4_ERR_INVALID_ARG;
+  if (dq_code != NF4_DQ_E4M3 && dq_code != NF4_DQ_INT8) return NF4_ERR_INVALID_ARG;
+  if (dq_blocksize != nf4::kDqBlock) return NF4_ERR_UNSUPPORTED;
+  if (nb == 0) return NF4_OK;
+  if (absmax == nullptr || q_out == nullptr || scale_out == nullptr || mean_out == nullptr || workspace == nullptr)
+    return NF4_ERR_INVALID_ARG;
+  if (workspace_bytes < nf4::kDoubleQuantWorkspace) return NF4_ERR_INVALID_ARG;
+  if (!aligned(absmax, 16) || !aligned(q_out, 16) || !aligned(scale_out, 4) || !aligned(mean_out, 4) ||
+      !aligned(workspace, 16))
+    return NF4_ERR_MISALIGNED;
+  DeviceInfo d;
+  nf4_status st = device_info(&d);
+  if (st != NF4_OK) return st;
+  return from_cuda(nf4::launch_double_quant(absmax, nb, dq_code, q_out, scale_out, mean_out, workspace,
+                                            reinterpret_cast<cudaStream_t>(stream), d.num_sms));
+}
+
+nf4_status nf4_dequantize(const nf4_weight* w, void* out, int32_t out_dtype, nf4_stream_t stream) {
+  nf4::Scales s;
+  nf4_status st = check_weight(w, &s);
+  if (st != NF4_OK) return st;
+  if (out_dtype != NF4_F32 && out_dtype != NF4_BF16) return NF4_ERR_INVALID_ARG;
+  const int64_t n = w->rows * w->cols;
+  if (n == 0) return NF4_OK;
+  if (out == nullptr) return NF4_ERR_INVALID_ARG;
+  if (!aligned(out, 16)) return NF4_ERR_MISALIGNED;
+  DeviceInfo d;
+  if ((st = device_info(&d)) != NF4_OK) return st;
+  return from_cuda(nf4::launch_dequantize(w->packed, s, n, out, out_dtype == NF4_BF16,
+                                          reinterpret_cast<cudaStream_t>(stream), d.num_sms));
+}
+
+nf4_status nf4_gemv(const nf4_weight* w, const void* x, int32_t batch, void* y, nf4_stream_t stream) {
+  nf4::Scales s;
+  nf4_status st = check_weight(w, &s);
+  if (st != NF4_OK) return st;
+  if (batch < 1 || batch > 8) return NF4_ERR_INVALID_ARG;
+  if (w->cols % nf4::kBlock != 0 || w->rows % 16 != 0) return NF4_ERR_UNSUPPORTED;
+  if (w->rows == 0 || w->cols == 0) return NF4_OK;
+  if (x == nullptr || y == nullptr) return NF4_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(y, 4)) return NF4_ERR_MISALIGNED;
+  DeviceInfo d;
+  if ((st = device_info(&d)) != NF4_OK) return st;
+  return from_cuda(nf4::launch_gemv(w->packed, s, w->rows, w->cols, x, batch, y,
+                                    reinterpret_cast<cudaStream_t>(stream), d.num_sms));
+}
+
+nf4_status nf4_gemm(const nf4_weight* w, const void* x, int64_t m, void* y, void* workspace, size_t workspace_bytes,
+                    nf4_stream_t stream) {
+  nf4::Scales s;
+  nf4_status st = check_weight(w, &s);
+  if (st != NF4_OK) return st;
+  if (m < 0) return NF4_ERR_INVALID_ARG;
+  if (w->cols % nf4::kBlock != 0 || w->rows % 128 != 0) return NF4_ERR_UNSUPPORTED;
+  if (m == 0 || w->rows == 0 || w->cols == 0) return NF4_OK;
+  if (x == nullptr || y == nullptr) return NF4_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(y, 16)) return NF4_ERR_MISALIGNED;
+  const size_t need = nf4::gemm_workspace_bytes(w->rows, w->cols, m);
+  if (workspace_bytes < need || (need > 0 && workspace == nullptr)) return NF4_ERR_INVALID_ARG;
+  if (need > 0 && !aligned(workspace, 16)) return NF4_ERR_MISALIGNED;
+  DeviceInfo d;
+  if ((st = device_info(&d)) != NF4_OK) return st;
+  return from_cuda(nf4::launch_gemm(w->packed, s, w->rows, w->cols, x, m, y, workspace, d.error_word,
+                                    reinterpret_cast<cudaStream_t>(stream), d.num_sms));
+}
+
+nf4_status nf4_check_device_error(nf4_stream_t stream) {
+  DeviceInfo d;
+  nf4_status st = device_info(&d);
+  if (st != NF4_OK) return st;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return NF4_ERR_CUDA;
+  unsigned word = 0;
+  if (cudaMemcpy(&word, d.error_word, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess) return NF4_ERR_CUDA;
+  if (word != 0) {
+    const unsigned zero = 0;
+    if (cudaMemcpy(d.error_word, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return NF4_ERR_CUDA;
+    return NF4_ERR_TIMEOUT;
+  }
+  return NF4_OK;
+}
+
+}  // extern "C"

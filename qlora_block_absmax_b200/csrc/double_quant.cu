@@ -1,0 +1,221 @@
+// double_quant.cu -- double quantization of the level-1 absmax array.
+//
+// "bitsandbytes quantization tutorial" (mljourney.com), "How NF4 Works": the
+// per-block scale constants are themselves quantized from float32 to float8;
+// "bitsandbytes" (ozercemkelahmet.com/tools), "Double quantization".  The
+// second level reuses the level-1 recipe with an 8-bit code book, in the order
+// of that page's "A worked example": block absmax m, x = RN(r / m),
+// y = RN(x * Q), code = round(y) -- E4M3 (Q = 448, nearest-even, saturating)
+// or int8 (Q = 127, half away from zero, clamped).  The mean is removed first
+// (one fp32 per tensor): mu = fp32(fp64(exact sum) / nb).
+//
+// Kernel 1 (sum): every fp32 value is an integer multiple of 2^-149, so each
+// thread adds its values into ten signed 64-bit limbs holding 32 bits each of
+// a 320-bit fixed-point number; integer addition makes the total exact and
+// independent of order.  Warp shuffles and shared memory combine threads,
+// 64-bit atomics combine CTAs, and the last CTA to finish normalises the limbs,
+// rounds the sum once to fp64 and writes mu.
+// Kernel 2 (codes): one warp per 256-value block.
+#include "nf4_common.cuh"
+#include "internal.h"
+
+namespace nf4 {
+namespace {
+
+constexpr int kLimbs = 10;
+
+struct SumWorkspace {
+  unsigned long long limb[kLimbs];  // two's-complement running sums of 32-bit digits
+  unsigned int done;                // CTAs finished
+};
+static_assert(sizeof(SumWorkspace) <= kDoubleQuantWorkspace, "workspace");
+
+__device__ __forceinline__ void add_value(long long (&acc)[kLimbs], float x) {
+  const uint32_t u = __float_as_uint(x);
+  const uint32_t e = (u >> 23) & 0xffu, f = u & 0x7fffffu;
+  const uint32_t mant = e ? (f | 0x800000u) : f;  // value = mant * 2^(sh - 149)
+  const int sh = e ? (int)e - 1 : 0;
+  const int li = sh >> 5;
+  const uint64_t v = (uint64_t)mant << (sh & 31);
+  long long lo = (long long)(v & 0xffffffffull), hi = (long long)(v >> 32);
+  if (u >> 31) {
+    lo = -lo;
+    hi = -hi;
+  }
+#pragma unroll
+  for (int L = 0; L < kLimbs; ++L) acc[L] += (L == li) ? lo : ((L == li + 1) ? hi : 0);
+}
+
+// bits [pos, pos + cnt) of the normalised limbs (cnt <= 32), as an integer
+__device__ uint64_t limb_bits(const uint32_t* d, int pos, int cnt) {
+  uint64_t r = 0;
+  for (int i = 0; i < cnt; ++i) {
+    const int p = pos + i;
+    if (p < 0 || p >= 32 * kLimbs) continue;
+    r |= (uint64_t)((d[p >> 5] >> (p & 31)) & 1u) << i;
+  }
+  return r;
+}
+
+// Normalise the signed limbs, round the total to fp64 (nearest even) and
+// return mu = fp32(fp64 sum / nb).  Single thread.
+__device__ float finish_mean(const long long* limb_in, int64_t nb) {
+  long long l[kLimbs];
+  for (int L = 0; L < kLimbs; ++L) l[L] = limb_in[L];
+  for (int L = 0; L < kLimbs - 1; ++L) {  // carry: limbs 0..8 into [0, 2^32)
+    const long long carry = l[L] >> 32;   // arithmetic shift = floor division
+    l[L] -= carry * (1LL << 32);
+    l[L + 1] += carry;
+  }
+  const bool neg = l[kLimbs - 1] < 0;
+  uint32_t d[kLimbs];
+  if (neg) {  // magnitude of a negative total: subtract from zero
+    long long borrow = 0;
+    for (int L = 0; L < kLimbs - 1; ++L) {
+      long long t = -l[L] - borrow;
+      borrow = t < 0;
+      d[L] = (uint32_t)(t + (borrow ? (1LL << 32) : 0));
+    }
+    d[kLimbs - 1] = (uint32_t)(-l[kLimbs - 1] - borrow);
+  } else {
+    for (int L = 0; L < kLimbs; ++L) d[L] = (uint32_t)l[L];
+  }
+  int top = -1;
+  for (int p = 32 * kLimbs - 1; p >= 0; --p)
+    if ((d[p >> 5] >> (p & 31)) & 1u) {
+      top = p;
+      break;
+    }
+  double s = 0.0;
+  if (top >= 0) {
+    uint64_t m;
+    int exp2;  // s = m * 2^exp2
+    if (top < 53) {
+      m = limb_bits(d, 0, 32) | (limb_bits(d, 32, 21) << 32);
+      exp2 = -149;
+    } else {
+      const int low = top - 52;
+      m = limb_bits(d, low, 32) | (limb_bits(d, low + 32, 21) << 32);
+      const bool round = limb_bits(d, low - 1, 1) != 0;
+      bool sticky = false;
+      for (int p = 0; p < low - 1 && !sticky; ++p) sticky = (d[p >> 5] >> (p & 31)) & 1u;
+      if (round && (sticky || (m & 1u))) m += 1;  // may reach 2^53: still exact
+      exp2 = low - 149;
+    }
+    // m < 2^54 and -149 <= exp2 <= 118: both factors exact, product exact
+    s = __dmul_rn((double)m, __longlong_as_double((long long)(exp2 + 1023) << 52));
+  }
+  if (neg) s = -s;
+  return __double2float_rn(__ddiv_rn(s, (double)nb));
+}
+
+__global__ void __launch_bounds__(256) dq_sum_kernel(const float* __restrict__ a, int64_t nb,
+                                                     SumWorkspace* __restrict__ ws, float* __restrict__ mean_out) {
+  long long acc[kLimbs];
+#pragma unroll
+  for (int L = 0; L < kLimbs; ++L) acc[L] = 0;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nb; i += (int64_t)gridDim.x * blockDim.x)
+    add_value(acc, a[i]);
+#pragma unroll
+  for (int L = 0; L < kLimbs; ++L)
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc[L] += __shfl_xor_sync(0xffffffffu, acc[L], off);
+
+  __shared__ long long red[8][kLimbs];
+  __shared__ bool last;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0)
+#pragma unroll
+    for (int L = 0; L < kLimbs; ++L) red[warp][L] = acc[L];
+  __syncthreads();
+  if (threadIdx.x < kLimbs) {
+    long long t = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w][threadIdx.x];
+    atomicAdd(&ws->limb[threadIdx.x], (unsigned long long)t);  // wraps mod 2^64 = signed add
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(&ws->done, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (last && threadIdx.x == 0) {
+    __threadfence();
+    long long l[kLimbs];
+    for (int L = 0; L < kLimbs; ++L) l[L] = (long long)atomicAdd(&ws->limb[L], 0ull);
+    *mean_out = finish_mean(l, nb);
+  }
+}
+
+__global__ void __launch_bounds__(256) dq_code_kernel(const float* __restrict__ a, int64_t nb, int dq_code,
+                                                      const float* __restrict__ mean, uint8_t* __restrict__ q,
+                                                      float* __restrict__ scale) {
+  const int lane = threadIdx.x & 31;
+  const int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t ngroups = (nb + kDqBlock - 1) / kDqBlock;
+  if (g >= ngroups) return;  // whole warp leaves together
+  const float mu = *mean;
+  const int64_t first = g * kDqBlock + lane * 8;
+  const bool full = (g + 1) * kDqBlock <= nb;
+  float r[8];
+  if (full) {
+    const float4* p = reinterpret_cast<const float4*>(a + first);
+    float4 v0 = p[0], v1 = p[1];
+    r[0] = v0.x; r[1] = v0.y; r[2] = v0.z; r[3] = v0.w;
+    r[4] = v1.x; r[5] = v1.y; r[6] = v1.z; r[7] = v1.w;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) r[i] = (first + i < nb) ? a[first + i] : mu;  // mu -> residual 0
+  }
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    r[i] = __fsub_rn(r[i], mu);  // residual after removing the mean
+    m = fmaxf(m, fabsf(r[i]));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if (lane == 0) scale[g] = m;
+  const float Q = dq_code == 0 ? kE4M3Top : kInt8Top;
+  float y[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) y[i] = (m != 0.0f) ? __fmul_rn(__fdiv_rn(r[i], m), Q) : 0.0f;
+  uint32_t lo, hi;
+  if (dq_code == 0) {
+    lo = pack_e4m3x2(y[0], y[1]) | (pack_e4m3x2(y[2], y[3]) << 16);
+    hi = pack_e4m3x2(y[4], y[5]) | (pack_e4m3x2(y[6], y[7]) << 16);
+  } else {
+    uint32_t b[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float t = fminf(fmaxf(roundf(y[i]), -127.0f), 127.0f);  // half away from zero, clamp
+      b[i] = (uint32_t)(uint8_t)(int8_t)(int)t;
+    }
+    lo = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+    hi = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+  }
+  if (full) {
+    *reinterpret_cast<uint2*>(q + first) = make_uint2(lo, hi);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (first + i < nb) q[first + i] = (uint8_t)((i < 4 ? lo : hi) >> (8 * (i & 3)));
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_double_quant(const float* absmax, int64_t nb, int dq_code, uint8_t* q, float* scale,
+                                float* mean, void* workspace, cudaStream_t stream, int num_sms) {
+  cudaError_t err = cudaMemsetAsync(workspace, 0, sizeof(SumWorkspace), stream);
+  if (err != cudaSuccess) return err;
+  int64_t grid1 = (nb + 256 * 8 - 1) / (256 * 8);
+  if (grid1 > num_sms) grid1 = num_sms;
+  if (grid1 < 1) grid1 = 1;
+  dq_sum_kernel<<<(unsigned)grid1, 256, 0, stream>>>(absmax, nb, static_cast<SumWorkspace*>(workspace), mean);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  const int64_t ngroups = (nb + kDqBlock - 1) / kDqBlock;
+  const int64_t grid2 = (ngroups + 7) / 8;
+  dq_code_kernel<<<(unsigned)grid2, 256, 0, stream>>>(absmax, nb, dq_code, mean, q, scale);
+  return cudaGetLastError();
+}
+
+}  // namespace nf4

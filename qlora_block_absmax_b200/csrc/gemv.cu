@@ -1,0 +1,224 @@
+// gemv.cu -- decode GEMV (and skinny GEMM, m <= 64) with on-the-fly NF4 dequantization.
+//
+// "bitsandbytes" (ozercemkelahmet.com/tools), "How it works" Step 5: each block
+// is expanded back to 16-bit with its scale and the code book, then
+// multiplied; compute dtype bfloat16 ("bitsandbytes quantization tutorial",
+// mljourney.com, "4-bit Loading with NF4").  So the effective weight is
+// Wc = bf16_rn(RN(code[idx] * a)) and y[b, n] = bf16_rn(sum_k Wc[n, k] x[b, k])
+// with fp32 accumulation.
+//
+// Mapping (one CTA = one 16-row tile, 8 warps splitting K; one warp step =
+// 16 rows x 256 k):
+//   lane (g = lane/4, t = lane%4) owns rows g and g+8 of the tile and level-1
+//   block t of the step (64 codes = 32 bytes per row, two 16-byte loads).
+//   Per (row, block) the lane builds the 16 bf16 values bf16_rn(code[i] * a)
+//   and keeps their low and high bytes as four 8-byte byte-permute pools; a
+//   packed 32-bit word of 8 codes is then decoded with byte permutes: the
+//   code nibbles themselves are the permute selectors, bit 3 of each nibble
+//   picks the pool half.
+//   The decoded bf16 pairs are the A operand of mma.sync m16n8k16 (weights
+//   as the M side, activations as the N side: batch <= 8 per n-tile), so one
+//   decode feeds up to 8 activation rows per n-tile.  Lanes with the same t
+//   use the same four k positions per MMA, which keeps the B fragment a
+//   contiguous 8-byte slice of x.
+// Partial sums of the 8 warps are added in a fixed order through shared
+// memory, so results are deterministic.
+#include "nf4_common.cuh"
+#include "internal.h"
+
+namespace nf4 {
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kStepK = 256;  // k per warp step (4 level-1 blocks)
+
+struct Table {  // byte pools: low/high bytes of bf16(code[i] * a), i in 0..7 (A) and 8..15 (B)
+  uint32_t la0, la1, lb0, lb1, ha0, ha1, hb0, hb1;
+};
+
+__device__ __forceinline__ Table make_table(float a) {
+  constexpr float code[16] = NF4_CODE_INIT;
+  uint32_t r[8];
+#pragma unroll
+  for (int m = 0; m < 8; ++m) r[m] = pack_bf16x2(__fmul_rn(code[2 * m], a), __fmul_rn(code[2 * m + 1], a));
+  Table T;
+  T.la0 = prmt(r[0], r[1], 0x6420);
+  T.la1 = prmt(r[2], r[3], 0x6420);
+  T.lb0 = prmt(r[4], r[5], 0x6420);
+  T.lb1 = prmt(r[6], r[7], 0x6420);
+  T.ha0 = prmt(r[0], r[1], 0x7531);
+  T.ha1 = prmt(r[2], r[3], 0x7531);
+  T.hb0 = prmt(r[4], r[5], 0x7531);
+  T.hb1 = prmt(r[6], r[7], 0x7531);
+  return T;
+}
+
+// Decode 8 codes (one packed word) into 4 bf16x2 registers:
+// out[0] = (e0, e1), out[1] = (e2, e3), out[2] = (e4, e5), out[3] = (e6, e7),
+// element e_j being the j-th code in memory order (high nibble first).
+__device__ __forceinline__ void decode_word(uint32_t q, const Table& T, uint32_t (&out)[4]) {
+  const uint32_t qx = q ^ 0x88888888u;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t s = h ? (q >> 16) : q;    // 4 selector nibbles
+    const uint32_t sx = h ? (qx >> 16) : qx; // same, pool-B view (bit 3 flipped)
+    const uint32_t la = prmt(T.la0, T.la1, s), lb = prmt(T.lb0, T.lb1, sx);
+    const uint32_t ha = prmt(T.ha0, T.ha1, s), hb = prmt(T.hb0, T.hb1, sx);
+    const uint32_t m1 = prmt(0x7f7f7f7fu, 0x7f7f7f7fu, sx);  // 0x7f where code >= 8, else 0
+    const uint32_t M = m1 | (m1 + m1);                          // 0xff where code >= 8
+    const uint32_t L = (la & ~M) | (lb & M);
+    const uint32_t H = (ha & ~M) | (hb & M);
+    out[2 * h] = prmt(L, H, 0x4051);      // selector nibble k -> element: 1,0,3,2
+    out[2 * h + 1] = prmt(L, H, 0x6273);
+  }
+}
+
+__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+struct StepData {
+  uint4 w0[2], w1[2];  // 32 code bytes of row g and of row g+8
+  float s0, s1;        // plain scales, or second-level block absmax (double quant)
+  uint32_t q0, q1;     // 8-bit scale codes (double quant)
+};
+
+template <bool kDQ>
+__device__ __forceinline__ void load_step(StepData& d, const uint8_t* __restrict__ packed, const Scales& s,
+                                          int64_t row0, int64_t cols, int64_t blk, bool valid) {
+  if (!valid) {
+    d.w0[0] = d.w0[1] = d.w1[0] = d.w1[1] = make_uint4(0x77777777u, 0x77777777u, 0x77777777u, 0x77777777u);
+    d.s0 = d.s1 = 0.0f;
+    d.q0 = d.q1 = 0;
+    return;
+  }
+  const int64_t rb = cols / kBlock;  // blocks per row
+  const uint4* p0 = reinterpret_cast<const uint4*>(packed + row0 * (cols / 2) + blk * 32);
+  const uint4* p1 = reinterpret_cast<const uint4*>(packed + (row0 + 8) * (cols / 2) + blk * 32);
+  d.w0[0] = __ldcs(p0);
+  d.w0[1] = __ldcs(p0 + 1);
+  d.w1[0] = __ldcs(p1);
+  d.w1[1] = __ldcs(p1 + 1);
+  const int64_t b0 = row0 * rb + blk, b1 = (row0 + 8) * rb + blk;
+  if (kDQ) {
+    d.q0 = s.q[b0];
+    d.q1 = s.q[b1];
+    d.s0 = s.scale[b0 / kDqBlock];
+    d.s1 = s.scale[b1 / kDqBlock];
+  } else {
+    d.s0 = __ldcs(s.absmax + b0);
+    d.s1 = __ldcs(s.absmax + b1);
+  }
+}
+
+template <int NT, bool kDQ>
+__global__ void __launch_bounds__(kWarps * 32, NT >= 4 ? 1 : 2)
+    gemv_kernel(const uint8_t* __restrict__ packed, Scales s, int64_t rows, int64_t cols,
+                const __nv_bfloat16* __restrict__ x, int batch, __nv_bfloat16* __restrict__ y) {
+  __shared__ float unit_lut[kDQ ? 256 : 1];
+  __shared__ float red[kWarps][16][8 * NT];
+  if (kDQ) unit_lut[threadIdx.x & 255] = dq_unit(threadIdx.x & 255, s.dq_code);
+  __syncthreads();
+  const float mu = kDQ ? *s.mean : 0.0f;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int64_t row0 = (int64_t)blockIdx.x * 16 + g;
+  const int64_t nblk = cols / kBlock;
+  const int64_t nsteps = (cols + kStepK - 1) / kStepK;
+
+  float acc[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[nt][j] = 0.0f;
+
+  // activation rows fed by this lane, one per n-tile (null: padding row)
+  const __nv_bfloat16* xrow[NT];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) xrow[nt] = (8 * nt + g < batch) ? x + (int64_t)(8 * nt + g) * cols : nullptr;
+
+  StepData cur, nxt;
+  int64_t st = warp;
+  if (st < nsteps) load_step<kDQ>(cur, packed, s, row0, cols, st * 4 + t, st * 4 + t < nblk);
+  for (; st < nsteps; st += kWarps) {
+    const int64_t blk = st * 4 + t;
+    const bool valid = blk < nblk;
+    if (st + kWarps < nsteps) load_step<kDQ>(nxt, packed, s, row0, cols, (st + kWarps) * 4 + t, (st + kWarps) * 4 + t < nblk);
+    float a0 = cur.s0, a1 = cur.s1;
+    if (kDQ) {
+      a0 = dq_absmax(unit_lut[cur.q0], cur.s0, mu);
+      a1 = dq_absmax(unit_lut[cur.q1], cur.s1, mu);
+    }
+    const Table T0 = make_table(a0), T1 = make_table(a1);
+    const uint32_t w0[8] = {cur.w0[0].x, cur.w0[0].y, cur.w0[0].z, cur.w0[0].w,
+                            cur.w0[1].x, cur.w0[1].y, cur.w0[1].z, cur.w0[1].w};
+    const uint32_t w1[8] = {cur.w1[0].x, cur.w1[0].y, cur.w1[0].z, cur.w1[0].w,
+                            cur.w1[1].x, cur.w1[1].y, cur.w1[1].z, cur.w1[1].w};
+    const int64_t kbase = blk * kBlock;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      uint32_t d0[4], d1[4];
+      decode_word(w0[j], T0, d0);
+      decode_word(w1[j], T1, d1);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        uint4 xv = make_uint4(0, 0, 0, 0);
+        if (xrow[nt] != nullptr && valid) xv = __ldg(reinterpret_cast<const uint4*>(xrow[nt] + kbase + 8 * j));
+        // k positions 8j..8j+3: A = (row g: d0[0], d0[1]; row g+8: d1[0], d1[1])
+        const uint32_t alo[4] = {d0[0], d1[0], d0[1], d1[1]};
+        mma_bf16(acc[nt], alo, xv.x, xv.y);
+        const uint32_t ahi[4] = {d0[2], d1[2], d0[3], d1[3]};
+        mma_bf16(acc[nt], ahi, xv.z, xv.w);
+      }
+    }
+    cur = nxt;
+  }
+
+  // accumulator fragment: c0 (row g, col 2t), c1 (g, 2t+1), c2 (g+8, 2t), c3 (g+8, 2t+1)
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    red[warp][g][8 * nt + 2 * t] = acc[nt][0];
+    red[warp][g][8 * nt + 2 * t + 1] = acc[nt][1];
+    red[warp][g + 8][8 * nt + 2 * t] = acc[nt][2];
+    red[warp][g + 8][8 * nt + 2 * t + 1] = acc[nt][3];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < 16 * batch; i += blockDim.x) {
+    const int r = i & 15, b = i >> 4;
+    float sum = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) sum += red[w][r][b];
+    y[(int64_t)b * rows + (int64_t)blockIdx.x * 16 + r] = __float2bfloat16_rn(sum);
+  }
+}
+
+template <int NT>
+cudaError_t launch_nt(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x, int batch,
+                      void* y, cudaStream_t stream) {
+  const unsigned grid = (unsigned)(rows / 16);
+  const auto* xb = static_cast<const __nv_bfloat16*>(x);
+  auto* yb = static_cast<__nv_bfloat16*>(y);
+  if (s.absmax == nullptr)
+    gemv_kernel<NT, true><<<grid, kWarps * 32, 0, stream>>>(packed, s, rows, cols, xb, batch, yb);
+  else
+    gemv_kernel<NT, false><<<grid, kWarps * 32, 0, stream>>>(packed, s, rows, cols, xb, batch, yb);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// batch <= 64: the activation rows are spread over ceil(batch / 8) n-tiles
+cudaError_t launch_gemv(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x, int batch,
+                        void* y, cudaStream_t stream, int /*num_sms*/) {
+  if (batch <= 8) return launch_nt<1>(packed, s, rows, cols, x, batch, y, stream);
+  if (batch <= 16) return launch_nt<2>(packed, s, rows, cols, x, batch, y, stream);
+  if (batch <= 32) return launch_nt<4>(packed, s, rows, cols, x, batch, y, stream);
+  return launch_nt<8>(packed, s, rows, cols, x, batch, y, stream);
+}
+
+}  // namespace nf4

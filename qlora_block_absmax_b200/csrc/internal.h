@@ -1,0 +1,39 @@
+// internal.h -- launchers behind the C ABI (see include/nf4.h for semantics).
+// Arguments are validated by the callers in api.cu; launchers only size grids.
+#pragma once
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace nf4 {
+
+constexpr int kBlock = 64;      // level-1 block (elements per absmax)
+constexpr int kDqBlock = 256;   // level-2 block (absmax values per second-level scale)
+
+// Level-1 scales as the kernels see them: plain fp32 absmax, or the
+// double-quantized record (8-bit codes + second-level block absmax + mean).
+struct Scales {
+  const float* absmax;   // non-null: plain scales
+  const uint8_t* q;      // double-quantized codes
+  const float* scale;    // second-level block absmax
+  const float* mean;     // device pointer to the removed mean
+  int dq_code;           // 0 = E4M3, 1 = int8
+};
+
+cudaError_t launch_quantize(const void* src, bool bf16, int64_t n, uint8_t* packed, float* absmax,
+                            cudaStream_t stream, int num_sms);
+
+cudaError_t launch_double_quant(const float* absmax, int64_t nb, int dq_code, uint8_t* q, float* scale,
+                                float* mean, void* workspace, cudaStream_t stream, int num_sms);
+constexpr size_t kDoubleQuantWorkspace = 256;
+
+cudaError_t launch_dequantize(const uint8_t* packed, const Scales& s, int64_t n, void* out, bool out_bf16,
+                              cudaStream_t stream, int num_sms);
+
+cudaError_t launch_gemv(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x,
+                        int batch, void* y, cudaStream_t stream, int num_sms);
+
+size_t gemm_workspace_bytes(int64_t rows, int64_t cols, int64_t m);
+cudaError_t launch_gemm(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x,
+                        int64_t m, void* y, void* workspace, unsigned* err, cudaStream_t stream, int num_sms);
+
+}  // namespace nf4

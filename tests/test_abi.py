@@ -1,0 +1,108 @@
+"""The C-ABI library loads on a machine without a GPU, exports every function
+include/nf4.h declares, and rejects bad arguments on the host before touching
+CUDA.  No compute calls here."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from qlora_block_absmax_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "nf4.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nf4_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return _lib.load()
+
+
+def test_every_declared_symbol_is_exported_and_bound(lib):
+    names = declared_functions()
+    assert len(names) >= 12
+    for name in names:
+        assert hasattr(lib, name), name
+        assert name in _lib.SIGNATURES, f"binding lacks {name}"
+
+
+def test_status_strings(lib):
+    for code, name in _lib.STATUS_NAMES.items():
+        assert lib.nf4_status_string(code).decode() == name
+
+
+def test_code_table_matches_oracle_bitwise(lib):
+    buf = (ctypes.c_float * 16)()
+    lib.nf4_code_table(buf)
+    _, c32 = oracle.codebook()
+    assert np.array_equal(np.array(buf[:], np.float32).view(np.uint32), c32.view(np.uint32))
+
+
+def test_storage_bytes(lib):
+    n = 4096 * 4096
+    nb = n // 64
+    assert lib.nf4_storage_bytes(n, 64, 0, 256) == n // 2 + 4 * nb
+    assert lib.nf4_storage_bytes(n, 64, 1, 256) == n // 2 + nb + 4 * (nb // 256) + 4
+    assert lib.nf4_storage_bytes(65, 64, 1, 256) == 33 + 2 + 4 + 4
+    assert lib.nf4_storage_bytes(0, 64, 1, 256) == 0
+
+
+def weight(rows=128, cols=128, packed=0x1000, absmax=0x2000, q=0, scale=0, mean=0, bs=64, dqbs=256, code=0):
+    return _lib.NF4Weight(packed, absmax, q, scale, mean, rows, cols, bs, dqbs, code)
+
+
+def test_host_validation_before_cuda(lib):
+    E = {v: k for k, v in _lib.STATUS_NAMES.items()}
+    s = None
+    # quantize
+    assert lib.nf4_quantize(0x1000, 0, -1, 64, 0x2000, 0x3000, s) == E["NF4_ERR_INVALID_ARG"]
+    assert lib.nf4_quantize(0x1000, 7, 10, 64, 0x2000, 0x3000, s) == E["NF4_ERR_INVALID_ARG"]
+    assert lib.nf4_quantize(0x1000, 0, 10, 32, 0x2000, 0x3000, s) == E["NF4_ERR_UNSUPPORTED"]
+    assert lib.nf4_quantize(0x1000, 0, 0, 64, 0x2000, 0x3000, s) == E["NF4_OK"]  # empty: nothing launched
+    assert lib.nf4_quantize(None, 0, 10, 64, 0x2000, 0x3000, s) == E["NF4_ERR_INVALID_ARG"]
+    assert lib.nf4_quantize(0x1008, 0, 10, 64, 0x2000, 0x3000, s) == E["NF4_ERR_MISALIGNED"]
+    # double quant
+    assert lib.nf4_double_quant(0x1000, 10, 128, 0, 0x2000, 0x3000, 0x4000, 0x5000, 256, s) == E["NF4_ERR_UNSUPPORTED"]
+    assert lib.nf4_double_quant(0x1000, 10, 256, 5, 0x2000, 0x3000, 0x4000, 0x5000, 256, s) == E["NF4_ERR_INVALID_ARG"]
+    assert lib.nf4_double_quant(0x1000, 10, 256, 0, 0x2000, 0x3000, 0x4000, 0x5000, 8, s) == E["NF4_ERR_INVALID_ARG"]
+    assert lib.nf4_double_quant(0x1000, 0, 256, 0, 0x2000, 0x3000, 0x4000, 0x5000, 256, s) == E["NF4_OK"]
+    assert lib.nf4_double_quant_workspace_bytes(1 << 20) >= 128
+    # weight descriptor checks
+    w = weight(bs=32)
+    assert lib.nf4_dequantize(ctypes.byref(w), 0x9000, 0, s) == E["NF4_ERR_UNSUPPORTED"]
+    w = weight(packed=0x1001)
+    assert lib.nf4_dequantize(ctypes.byref(w), 0x9000, 0, s) == E["NF4_ERR_MISALIGNED"]
+    w = weight(absmax=0)  # neither plain scales nor a double-quant record
+    assert lib.nf4_dequantize(ctypes.byref(w), 0x9000, 0, s) == E["NF4_ERR_INVALID_ARG"]
+    w = weight(absmax=0, q=0x3000, scale=0x4000, mean=0x5000, code=9)
+    assert lib.nf4_dequantize(ctypes.byref(w), 0x9000, 0, s) == E["NF4_ERR_INVALID_ARG"]
+    w = weight()
+    assert lib.nf4_dequantize(ctypes.byref(w), 0x9000, 4, s) == E["NF4_ERR_INVALID_ARG"]
+    assert lib.nf4_dequantize(None, 0x9000, 0, s) == E["NF4_ERR_INVALID_ARG"]
+    # gemv / gemm shape rules
+    assert lib.nf4_gemv(ctypes.byref(w), 0x9000, 9, 0xa000, s) == E["NF4_ERR_INVALID_ARG"]
+    assert lib.nf4_gemv(ctypes.byref(w), 0x9000, 0, 0xa000, s) == E["NF4_ERR_INVALID_ARG"]
+    w = weight(cols=96)
+    assert lib.nf4_gemv(ctypes.byref(w), 0x9000, 1, 0xa000, s) == E["NF4_ERR_UNSUPPORTED"]
+    w = weight(rows=120)
+    assert lib.nf4_gemv(ctypes.byref(w), 0x9000, 1, 0xa000, s) == E["NF4_ERR_UNSUPPORTED"]
+    w = weight(rows=112)
+    assert lib.nf4_gemm(ctypes.byref(w), 0x9000, 4, 0xa000, None, 0, s) == E["NF4_ERR_UNSUPPORTED"]
+    w = weight()
+    assert lib.nf4_gemm(ctypes.byref(w), 0x9000, -1, 0xa000, None, 0, s) == E["NF4_ERR_INVALID_ARG"]
+    assert lib.nf4_gemm(ctypes.byref(w), 0x9000, 0, 0xa000, None, 0, s) == E["NF4_OK"]
+    assert lib.nf4_gemm(ctypes.byref(w), 0x9008, 4, 0xa000, None, 0, s) == E["NF4_ERR_MISALIGNED"]
+
+
+def test_device_query_without_gpu_is_safe(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("GPU present")
+    assert lib.nf4_device_supported() == 0

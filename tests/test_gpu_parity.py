@@ -1,0 +1,275 @@
+"""Parity of the CUDA library (through its C ABI) with the CPU oracle.
+
+Bit-exact: packed codes, fp32 absmax, double-quant codes/scales/mean, fp32 and
+bf16 dequantization.  GEMV/GEMM outputs: per-output relative error <= 1e-2
+against the fp64-accumulated oracle, with a floor of 1e-3 * rms(y_ref) on the
+denominator (outputs whose exact value is near zero cannot be judged
+relatively; fp32 accumulation alone gives errors of ~1e-6 * rms there).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import qlora_block_absmax_b200 as nf4
+from qlora_block_absmax_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+REL_TOL = 1e-2
+FLOOR = 1e-3
+
+
+def dev(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def dev_bf16(bits: np.ndarray) -> torch.Tensor:
+    return dev(bits.view(np.int16)).view(torch.bfloat16)
+
+
+def host_bf16_bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def near_threshold_count(w_f32: np.ndarray, absmax: np.ndarray) -> int:
+    """elements whose normalised value lies within 1e-6 of a code midpoint"""
+    _, c = oracle.codebook()
+    mids = (c[:-1].astype(np.float64) + c[1:]) / 2
+    a = np.repeat(absmax, 64)[:w_f32.size].astype(np.float64)
+    x = np.divide(w_f32.astype(np.float64), a, out=np.zeros_like(a), where=a > 0)
+    return int((np.abs(x[:, None] - mids[None, :]) <= 1e-6).any(axis=1).sum())
+
+
+def check_matmul(y_gpu: torch.Tensor, y_ref: np.ndarray, what: str):
+    y = y_gpu.float().cpu().numpy().astype(np.float64)
+    rms = np.sqrt(np.mean(y_ref ** 2)) if y_ref.size else 0.0
+    denom = np.maximum(np.abs(y_ref), FLOOR * rms)
+    err = np.abs(y - y_ref)
+    bad = err > REL_TOL * denom
+    floored = int((np.abs(y_ref) < FLOOR * rms).sum())
+    assert not bad.any(), (f"{what}: {bad.sum()} of {y.size} outputs beyond 1e-2 (max rel "
+                           f"{(err / np.maximum(denom, 1e-300)).max():.3e}, floored {floored})")
+    return float((err / np.maximum(denom, 1e-300)).max()), floored
+
+
+def special_weights(n_blocks: int, seed: int) -> np.ndarray:
+    """normal weights with hand-made blocks: zeros, signed zeros, negative max,
+    constants, exact code values, values on thresholds, tiny (subnormal) scales"""
+    w = synth.normal_weights((n_blocks * 64,), seed)
+    _, c = oracle.codebook()
+    blocks = w.reshape(-1, 64)
+    blocks[0] = 0.0
+    blocks[1, ::2] = -0.0
+    blocks[1, 1::2] = 0.0
+    blocks[2] = -np.abs(blocks[2])
+    blocks[3] = np.float32(0.25)
+    blocks[4, :16] = c
+    blocks[4, 16:] = c[np.arange(48) % 16] * np.float32(0.5)
+    mids = np.array([(float(c[i]) + float(c[i + 1])) / 2 for i in range(15)], np.float32)
+    blocks[5, :15] = mids
+    blocks[5, 15] = 1.0
+    blocks[6] = blocks[6] * np.float32(1e-38)     # tiny scale: exact-division path
+    blocks[7] = blocks[7] * np.float32(3e-42)     # subnormal scale
+    return w
+
+
+# --------------------------------------------------------------------------- quantize
+
+@pytest.mark.parametrize("n", [1, 2, 63, 64, 65, 127, 129, 4097, 64 * 1000 + 33])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_quantize_bit_exact_small(n, dtype):
+    w = synth.normal_weights((n,), 7000 + n)
+    if dtype == "bf16":
+        bits = synth.f32_to_bf16_bits(w)
+        p_ref, a_ref = oracle.quantize(bits)
+        p, a = nf4.quantize(dev_bf16(bits))
+    else:
+        p_ref, a_ref = oracle.quantize(w)
+        p, a = nf4.quantize(dev(w))
+    assert np.array_equal(a.cpu().numpy().view(np.uint32), a_ref.view(np.uint32))
+    assert np.array_equal(p.cpu().numpy(), p_ref)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_quantize_special_blocks(dtype):
+    w = special_weights(40, 77)
+    if dtype == "bf16":
+        bits = synth.f32_to_bf16_bits(w)
+        p_ref, a_ref = oracle.quantize(bits)
+        p, a = nf4.quantize(dev_bf16(bits))
+    else:
+        p_ref, a_ref = oracle.quantize(w)
+        p, a = nf4.quantize(dev(w))
+    assert np.array_equal(a.cpu().numpy().view(np.uint32), a_ref.view(np.uint32))
+    assert np.array_equal(p.cpu().numpy(), p_ref)
+
+
+def test_quantize_config1_roundtrip():
+    """fp32 1024x1024 ~N(0,0.02): codes, absmax, fp32 dequantization and
+    re-quantization all bit-exact."""
+    w = synth.config1_weight().reshape(-1)
+    p_ref, a_ref = oracle.quantize(w)
+    p, a = nf4.quantize(dev(w))
+    assert np.array_equal(p.cpu().numpy(), p_ref)
+    assert np.array_equal(a.cpu().numpy(), a_ref)
+    qw = nf4.QuantizedWeight(packed=p, rows=1024, cols=1024, absmax=a)
+    wh = nf4.dequantize(qw, torch.float32)
+    wh_ref = oracle.dequantize(p_ref, a_ref, w.size)
+    assert np.array_equal(wh.cpu().numpy().reshape(-1).view(np.uint32), wh_ref.view(np.uint32))
+    p2, a2 = nf4.quantize(wh.reshape(-1))
+    assert np.array_equal(p2.cpu().numpy(), p_ref) and np.array_equal(a2.cpu().numpy(), a_ref)
+    print(f"config1: near-midpoint elements {near_threshold_count(w, a_ref)}")
+
+
+def test_quantize_config2_bf16_outliers():
+    bits = synth.config2_weight().reshape(-1)
+    p_ref, a_ref = oracle.quantize(bits)
+    p, a = nf4.quantize(dev_bf16(bits))
+    assert np.array_equal(a.cpu().numpy(), a_ref)
+    assert np.array_equal(p.cpu().numpy(), p_ref)
+    print(f"config2: near-midpoint elements {near_threshold_count(synth.bf16_bits_to_f32(bits), a_ref)}")
+
+
+# --------------------------------------------------------------------------- double quant
+
+def dq_cases():
+    r = synth.rng(99)
+    _, a2 = oracle.quantize(synth.config2_weight().reshape(-1))
+    return {
+        "config2": a2,
+        "one": np.array([0.3], np.float32),
+        "255": np.abs(r.standard_normal(255)).astype(np.float32),
+        "257": np.abs(r.standard_normal(257)).astype(np.float32),
+        "constant": np.full(700, 0.0625, np.float32),
+        "wide": (np.abs(r.standard_normal(3000)) * np.exp(r.uniform(-80, 80, 3000))).astype(np.float32),
+        "signed": r.standard_normal(1000).astype(np.float32),
+        "zeros_and_tiny": np.concatenate([np.zeros(300, np.float32), np.full(212, 1e-40, np.float32)]),
+    }
+
+
+@pytest.mark.parametrize("case", list(dq_cases().keys()))
+@pytest.mark.parametrize("code", ["e4m3", "int8"])
+def test_double_quant_bit_exact(case, code):
+    a = dq_cases()[case]
+    c = oracle.DQ_E4M3 if code == "e4m3" else oracle.DQ_INT8
+    q_ref, s_ref, m_ref = oracle.double_quant(a, 256, c)
+    q, s, m = nf4.double_quant(dev(a), code)
+    assert np.float32(m.item()).view(np.uint32) == np.float32(m_ref).view(np.uint32)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+# --------------------------------------------------------------------------- dequantize
+
+@pytest.mark.parametrize("use_dq,code", [(False, "e4m3"), (True, "e4m3"), (True, "int8")])
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+@pytest.mark.parametrize("rows,cols", [(1, 1), (3, 21), (16, 64), (37, 129), (128, 640)])
+def test_dequantize_bit_exact(use_dq, code, out, rows, cols):
+    w = special_weights((rows * cols + 63) // 64 + 8, 5 + rows)[:rows * cols].reshape(rows, cols)
+    qw = nf4.quantize_weight(dev(w), use_double_quant=use_dq, code=code)
+    p_ref, a_ref = oracle.quantize(w.reshape(-1))
+    if use_dq:
+        c = oracle.DQ_E4M3 if code == "e4m3" else oracle.DQ_INT8
+        q_ref, s_ref, m_ref = oracle.double_quant(a_ref, 256, c)
+        a_ref = oracle.absmax_reconstruct(q_ref, s_ref, m_ref, 256, c)
+    ref = oracle.dequantize(p_ref, a_ref, rows * cols, 64, out)
+    got = nf4.dequantize(qw, torch.float32 if out == "f32" else torch.bfloat16)
+    if out == "f32":
+        assert np.array_equal(got.cpu().numpy().reshape(-1).view(np.uint32), ref.view(np.uint32))
+    else:
+        assert np.array_equal(host_bf16_bits(got).reshape(-1), ref)
+
+
+def test_dequantize_config2_double_quant_bf16():
+    bits = synth.config2_weight()
+    qw = nf4.quantize_weight(dev_bf16(bits), use_double_quant=True, code="e4m3")
+    p_ref, a_ref = oracle.quantize(bits.reshape(-1))
+    q_ref, s_ref, m_ref = oracle.double_quant(a_ref, 256, oracle.DQ_E4M3)
+    ah = oracle.absmax_reconstruct(q_ref, s_ref, m_ref, 256, oracle.DQ_E4M3)
+    ref = oracle.dequantize(p_ref, ah, bits.size, 64, "bf16")
+    got = nf4.dequantize(qw, torch.bfloat16)
+    assert np.array_equal(host_bf16_bits(got).reshape(-1), ref)
+
+
+# --------------------------------------------------------------------------- matmul
+
+def quantized_pair(rows, cols, seed, use_dq, code="e4m3"):
+    w = synth.normal_weights((rows, cols), seed)
+    qw = nf4.quantize_weight(dev(w), use_double_quant=use_dq, code=code)
+    p_ref, a_ref = oracle.quantize(w.reshape(-1))
+    if use_dq:
+        c = oracle.DQ_E4M3 if code == "e4m3" else oracle.DQ_INT8
+        q_ref, s_ref, m_ref = oracle.double_quant(a_ref, 256, c)
+        a_ref = oracle.absmax_reconstruct(q_ref, s_ref, m_ref, 256, c)
+    return qw, p_ref, a_ref
+
+
+@pytest.mark.parametrize("rows,cols", [(16, 64), (16, 192), (48, 320), (128, 256), (256, 4160)])
+@pytest.mark.parametrize("batch", [1, 3, 8])
+@pytest.mark.parametrize("use_dq", [False, True])
+def test_gemv_small(rows, cols, batch, use_dq):
+    qw, p_ref, a_ref = quantized_pair(rows, cols, rows + cols + batch, use_dq)
+    x = synth.activations((batch, cols), 31 + batch)
+    y = nf4.gemv(qw, dev_bf16(x))
+    check_matmul(y, oracle.matmul(p_ref, a_ref, rows, cols, x), f"gemv {rows}x{cols} b{batch}")
+
+
+@pytest.mark.parametrize("shape", [(4096, 4096), (14336, 4096), (4096, 14336), (1024, 4096)])
+@pytest.mark.parametrize("batch", [1, 4, 8])
+def test_gemv_config3_shapes(shape, batch):
+    rows, cols = shape
+    qw, p_ref, a_ref = quantized_pair(rows, cols, 1010 + rows // 1024 + cols // 1024, True)
+    x = synth.activations((batch, cols), 1013)
+    y = nf4.gemv(qw, dev_bf16(x))
+    mx, floored = check_matmul(y, oracle.matmul(p_ref, a_ref, rows, cols, x), f"gemv {shape} b{batch}")
+    print(f"gemv {shape} b{batch}: max floored-rel err {mx:.2e}, floored {floored}")
+
+
+def test_gemv_one_hot_pins_bit_exact():
+    rows, cols = 64, 256
+    qw, p_ref, a_ref = quantized_pair(rows, cols, 3, True)
+    wc = oracle.dequantize(p_ref, a_ref, rows * cols, 64, "bf16").reshape(rows, cols)
+    ks = [0, 1, 63, 64, 130, 255, 7, 200]
+    x = synth.f32_to_bf16_bits(np.eye(cols, dtype=np.float32)[ks])
+    y = nf4.gemv(qw, dev_bf16(x))
+    assert np.array_equal(host_bf16_bits(y), wc[:, ks].T)
+
+
+def test_gemv_zero_codes_give_zero():
+    rows, cols = 32, 128
+    p = torch.full((rows * cols // 2,), 0x77, dtype=torch.uint8, device="cuda")
+    a = torch.rand(rows * cols // 64, device="cuda") + 0.5
+    qw = nf4.QuantizedWeight(packed=p, rows=rows, cols=cols, absmax=a)
+    x = dev_bf16(synth.activations((5, cols), 4))
+    y = nf4.gemv(qw, x)
+    assert torch.all(y == 0)
+
+
+@pytest.mark.parametrize("m", [1, 9, 16, 33, 64, 65, 128, 200, 256])
+def test_gemm_small(m):
+    rows, cols = 256, 512
+    qw, p_ref, a_ref = quantized_pair(rows, cols, 41 + m, True)
+    x = synth.activations((m, cols), 42 + m)
+    y = nf4.gemm(qw, dev_bf16(x))
+    check_matmul(y, oracle.matmul(p_ref, a_ref, rows, cols, x), f"gemm m{m}")
+
+
+@pytest.mark.parametrize("m", [16, 64, 256, 1024, 4096])
+def test_gemm_config4_sampled(m):
+    """W 14336x4096 NF4+DQ, X [m, 4096]: 2048 sampled outputs against the oracle,
+    plus every output of the first activation row."""
+    rows, cols = 14336, 4096
+    qw, p_ref, a_ref = quantized_pair(rows, cols, 1020, True)
+    x = synth.activations((m, cols), 1021 + m)
+    y = nf4.gemm(qw, dev_bf16(x))
+    r = synth.rng(5 + m)
+    bs = r.integers(0, m, 2048)
+    ns = r.integers(0, rows, 2048)
+    ref = oracle.matmul_sampled(p_ref, a_ref, rows, cols, x, bs, ns)
+    yh = y.float().cpu().numpy().astype(np.float64)
+    full_row = oracle.matmul(p_ref, a_ref, rows, cols, x[:1])
+    rms = np.sqrt(np.mean(full_row ** 2))
+    got = yh[bs, ns]
+    assert np.all(np.abs(got - ref) <= REL_TOL * np.maximum(np.abs(ref), FLOOR * rms))
+    check_matmul(y[:1], full_row, f"gemm m{m} row 0")
