@@ -1,0 +1,410 @@
+#!/usr/bin/env python
+"""Benchmark of the NF4 hot path on B200.
+
+One step = the whole path on one weight: quantize (bf16 -> NF4 codes + fp32
+absmax), double quantization (E4M3), dequantization (bf16 out), decode GEMV
+(batch 1) and prefill GEMM (M = 256), all through the C ABI of libnf4.so.
+
+Workload: the double-quantization case of the reference configs -- a bf16
+4096 x 4096 weight ~N(0, 0.02) with 0.1% of entries x20 (seeds 1002/1003) --
+with bf16 activations ~N(0, 1) (seeds 1013, 1277).  Inputs rotate over enough
+independent copies that every step's working set is cold in the 126 MB L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own replica
+(the path has no cross-GPU exchange); value = all ranks' bytes / max time.
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NF4 GEMV/dequant HBM GB/s (% of peak); NF4 GEMM TFLOPS; quantize Gelem/s"
+ROWS, COLS, GEMV_B, GEMM_M = 4096, 4096, 1, 256
+WORKLOAD = "nf4_path_bf16_4096x4096_outliers_gemv1_gemm256"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS = ("quantize", "double_quant", "dequantize", "gemv", "gemm")
+
+
+def work_per_step(rows=ROWS, cols=COLS, b=GEMV_B, m=GEMM_M):
+    """Algorithmic bytes (each operand read once, each output written once at
+    its stored width) and flops of every kernel in one step."""
+    n = rows * cols
+    nb = n // 64
+    nb2 = (nb + 255) // 256
+    w4 = n // 2 + nb + 4 * nb2 + 4           # NF4 codes + double-quant record
+    return {
+        "quantize": {"bytes": 2 * n + n // 2 + 4 * nb, "elems": n},
+        "double_quant": {"bytes": 4 * nb + nb + 4 * nb2 + 4},
+        "dequantize": {"bytes": w4 + 2 * n},
+        "gemv": {"bytes": w4 + 2 * b * cols + 2 * b * rows, "flops": 2 * b * n},
+        "gemm": {"bytes": w4 + 2 * m * cols + 2 * m * rows, "flops": 2 * m * n},
+    }
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].isdigit():
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = sorted(int(r[1]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": int(rows[0][2]), "samples": len(rows), "reasons": reasons}
+
+
+# ---------------------------------------------------------------------------- oracle baseline
+
+def oracle_sample_step(sample_rows: int, w_bits, x_bits, X_bits):
+    """The same step computed by the CPU oracle on the first `sample_rows` rows
+    of the weight (GEMM over all M activation rows).  Returns elapsed seconds
+    and the algorithmic bytes of the sample."""
+    import oracle
+    n = sample_rows * COLS
+    t0 = time.perf_counter()
+    p, a = oracle.quantize(w_bits[:sample_rows].reshape(-1))
+    q, s, mu = oracle.double_quant(a, 256, oracle.DQ_E4M3)
+    ah = oracle.absmax_reconstruct(q, s, mu, 256, oracle.DQ_E4M3)
+    oracle.dequantize(p, ah, n, 64, "bf16")
+    oracle.matmul(p, ah, sample_rows, COLS, x_bits)
+    oracle.matmul(p, ah, sample_rows, COLS, X_bits)
+    dt = time.perf_counter() - t0
+    work = work_per_step(rows=sample_rows)
+    return dt, sum(v["bytes"] for v in work.values())
+
+
+def cpu_baseline(sample_rows: int, reps: int = 1):
+    import oracle
+    from qlora_block_absmax_b200 import synth
+    w = synth.config2_weight()
+    x = synth.activations((GEMV_B, COLS), 1013)
+    X = synth.activations((GEMM_M, COLS), 1277)
+    oracle.build()
+    cores = oracle.get_threads()
+    total_t, total_b = 0.0, 0
+    for _ in range(reps):
+        dt, b = oracle_sample_step(sample_rows, w, x, X)
+        total_t += dt
+        total_b += b
+    return {"value": total_b / total_t / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"whole step on the first {sample_rows} of {ROWS} weight rows "
+                      f"(GEMM over all {GEMM_M} activation rows), {reps} rep(s), {total_t:.1f} s",
+            "seconds": total_t}
+
+
+# ---------------------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import qlora_block_absmax_b200 as nf4
+    from qlora_block_absmax_b200 import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+
+    # ---- inputs (identical values in every copy; distinct memory)
+    w_bits = synth.config2_weight()
+    x_bits = synth.activations((GEMV_B, COLS), 1013)
+    X_bits = synth.activations((GEMM_M, COLS), 1277)
+    host_w = torch.from_numpy(w_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    host_x = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    host_X = torch.from_numpy(X_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    n = ROWS * COLS
+    nb = n // 64
+    per_copy = 2 * n + n // 2 + 4 * nb + nb + 2 * n + 2 * GEMM_M * (ROWS + COLS)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    copies = max(4, -(-3 * l2 // per_copy))
+
+    class Copy:
+        pass
+
+    cs = []
+    for _ in range(copies):
+        c = Copy()
+        c.w = host_w.to(dev)
+        c.x = host_x.to(dev)
+        c.X = host_X.to(dev)
+        c.packed = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+        c.absmax = torch.empty(nb, dtype=torch.float32, device=dev)
+        c.q = torch.empty(nb, dtype=torch.uint8, device=dev)
+        c.scale = torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev)
+        c.mean = torch.empty(1, dtype=torch.float32, device=dev)
+        c.ws = torch.empty(256, dtype=torch.uint8, device=dev)
+        c.deq = torch.empty(ROWS, COLS, dtype=torch.bfloat16, device=dev)
+        c.y = torch.empty(GEMV_B, ROWS, dtype=torch.bfloat16, device=dev)
+        c.Y = torch.empty(GEMM_M, ROWS, dtype=torch.bfloat16, device=dev)
+        c.qw = nf4.QuantizedWeight(packed=c.packed, rows=ROWS, cols=COLS, absmax_q=c.q, absmax_scale=c.scale,
+                                   absmax_mean=c.mean, dq_code=nf4.NF4_DQ_E4M3)
+        cs.append(c)
+    stream = torch.cuda.current_stream()
+
+    def step(c, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        nf4.quantize(c.w, out=(c.packed, c.absmax))
+        if ev is not None:
+            ev[1].record(stream)
+        nf4.double_quant(c.absmax, "e4m3", out=(c.q, c.scale, c.mean), workspace=c.ws)
+        if ev is not None:
+            ev[2].record(stream)
+        nf4.dequantize(c.qw, torch.bfloat16, out=c.deq)
+        if ev is not None:
+            ev[3].record(stream)
+        nf4.gemv(c.qw, c.x, out=c.y)
+        if ev is not None:
+            ev[4].record(stream)
+        nf4.gemm(c.qw, c.X, out=c.Y)
+        if ev is not None:
+            ev[5].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for i in range(args.warmup):
+        step(cs[i % copies])
+    nf4.check_device_error()
+    barrier()
+
+    # ---- device-timed region: K steps, per-kernel events on the launching stream
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    launches0 = nf4.kernel_launches()
+    barrier()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(cs[i % copies], events[i])
+    t_end.record(stream)
+    barrier()
+    launches = nf4.kernel_launches() - launches0
+    clocks = sampler.stop()
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    per_kernel_ms = {k: 0.0 for k in KERNELS}
+    for ev in events:
+        for j, k in enumerate(KERNELS):
+            per_kernel_ms[k] += ev[j].elapsed_time(ev[j + 1])
+    nf4.check_device_error()
+
+    # ---- end to end through the public API with host buffers
+    host_out = {"packed": torch.empty(n // 2, dtype=torch.uint8).pin_memory(),
+                "q": torch.empty(nb, dtype=torch.uint8).pin_memory(),
+                "scale": torch.empty((nb + 255) // 256, dtype=torch.float32).pin_memory(),
+                "mean": torch.empty(1, dtype=torch.float32).pin_memory(),
+                "y": torch.empty(GEMV_B, ROWS, dtype=torch.bfloat16).pin_memory(),
+                "Y": torch.empty(GEMM_M, ROWS, dtype=torch.bfloat16).pin_memory()}
+    h2d = host_w.numel() * 2 + host_x.numel() * 2 + host_X.numel() * 2
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+
+    def e2e_step(c):
+        c.w.copy_(host_w, non_blocking=True)
+        c.x.copy_(host_x, non_blocking=True)
+        c.X.copy_(host_X, non_blocking=True)
+        step(c)
+        host_out["packed"].copy_(c.packed, non_blocking=True)
+        host_out["q"].copy_(c.q, non_blocking=True)
+        host_out["scale"].copy_(c.scale, non_blocking=True)
+        host_out["mean"].copy_(c.mean, non_blocking=True)
+        host_out["y"].copy_(c.y, non_blocking=True)
+        host_out["Y"].copy_(c.Y, non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(cs[i % copies])
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        e2e_step(cs[i % copies])
+    e1.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+
+    work = work_per_step()
+    step_bytes = sum(v["bytes"] for v in work.values())
+    ms_per_step = elapsed_ms / args.steps
+    value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
+    e2e_value = world * step_bytes / (e2e_ms / args.steps * 1e-3) / 1e9
+
+    peaks, peak_src = load_peaks()
+    breakdown = {}
+    for k in KERNELS:
+        t = per_kernel_ms[k] / args.steps * 1e-3
+        d = {"ms": round(t * 1e3, 5), "share": round(per_kernel_ms[k] / sum(per_kernel_ms.values()), 4),
+             "gbs": round(work[k]["bytes"] / t / 1e9, 1),
+             "frac_hbm": round(work[k]["bytes"] / t / 1e9 / peaks["hbm_gbs"], 4)}
+        if "flops" in work[k]:
+            d["tflops"] = round(work[k]["flops"] / t / 1e12, 2)
+            d["frac_bf16"] = round(work[k]["flops"] / t / 1e12 / peaks["bf16_tflops"], 4)
+        if "elems" in work[k]:
+            d["gelem_s"] = round(work[k]["elems"] / t / 1e9, 2)
+        breakdown[k] = d
+    dom = max(KERNELS, key=lambda k: per_kernel_ms[k])
+    t_dom = per_kernel_ms[dom] / args.steps * 1e-3
+    if dom == "gemm":
+        ach = work[dom]["flops"] / t_dom / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": round(ach, 2), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(ach / peaks["bf16_tflops"], 4)}
+    else:
+        ach = work[dom]["bytes"] / t_dom / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4)}
+    roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json burst)" if peak_src == "measured" else "fallback"
+    roof["traffic"] = TRAFFIC.get(dom)
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "rows": ROWS, "cols": COLS, "gemv_batch": GEMV_B, "gemm_m": GEMM_M,
+                   "weight": "bf16 ~N(0,0.02), 0.1% x20 outliers, seeds 1002/1003; NF4 blocksize 64, "
+                             "double quant E4M3 blocks of 256",
+                   "l2": f"inputs rotate over {copies} copies ({copies * per_copy / 1e6:.0f} MB > L2 "
+                         f"{l2 / 1e6:.0f} MB)",
+                   "parallelism": "replicas" if world > 1 else "single"},
+        "roofline": roof,
+        "breakdown": breakdown,
+        "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+        "impl": "ours",
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = {k: (round(v, 4) if isinstance(v, float) else v)
+                                for k, v in cpu_baseline(args.cpu_rows, args.cpu_reps).items()}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ncu dram bytes per launch of each kernel at this workload (see profiles/); None until captured
+TRAFFIC = {}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from qlora_block_absmax_b200 import synth
+    oracle.build()
+    w = synth.config2_weight()
+    x = synth.activations((GEMV_B, COLS), 1013)
+    X = synth.activations((GEMM_M, COLS), 1277)
+    rows = args.ref_rows
+    for _ in range(args.warmup):
+        oracle_sample_step(rows, w, x, X)
+    t_total, b_total = 0.0, 0
+    for _ in range(args.steps):
+        dt, b = oracle_sample_step(rows, w, x, X)
+        t_total += dt
+        b_total += b
+    value = b_total / t_total / 1e9
+    cores = oracle.get_threads()
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_total / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "rows": ROWS, "cols": COLS, "gemv_batch": GEMV_B, "gemm_m": GEMM_M},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: whole path on the first {rows} of {ROWS} weight rows "
+                                   f"(GEMM over all {GEMM_M} activation rows)"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-rows", type=int, default=ROWS, help="weight rows in the oracle CPU-baseline sample")
+    ap.add_argument("--cpu-reps", type=int, default=3, help="repetitions of the oracle CPU-baseline sample")
+    ap.add_argument("--ref-rows", type=int, default=1024, help="weight rows per oracle step for --impl reference")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

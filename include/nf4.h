@@ -163,6 +163,10 @@ NF4_API void nf4_code_table(float out[16]);
 /* 1 if the current CUDA device is sm_100 (B200 class), else 0. */
 NF4_API int32_t nf4_device_supported(void);
 
+/* Diagnostics: number of kernels this process has launched through the
+ * library so far (all devices, all threads).  Host only. */
+NF4_API uint64_t nf4_kernel_launches(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -23,7 +23,7 @@ from . import _lib
 from ._lib import NF4_BF16, NF4_DQ_E4M3, NF4_DQ_INT8, NF4_F32, NF4Error
 
 __all__ = ["QuantizedWeight", "quantize", "double_quant", "quantize_weight", "dequantize", "gemv", "gemm",
-           "storage_bytes", "code_table", "check_device_error", "NF4Error", "library_path"]
+           "storage_bytes", "code_table", "check_device_error", "kernel_launches", "NF4Error", "library_path"]
 
 BLOCKSIZE = 64
 DQ_BLOCKSIZE = 256
@@ -190,6 +190,11 @@ def code_table() -> list:
     buf = (ctypes.c_float * 16)()
     _lib.load().nf4_code_table(buf)
     return list(buf)
+
+
+def kernel_launches() -> int:
+    """Kernels launched through the library by this process so far."""
+    return int(_lib.load().nf4_kernel_launches())
 
 
 def check_device_error(stream=None) -> None:

@@ -43,6 +43,7 @@ SIGNATURES = {
     "nf4_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "nf4_code_table": (None, [ctypes.POINTER(ctypes.c_float)]),
     "nf4_device_supported": (I32, []),
+    "nf4_kernel_launches": (ctypes.c_uint64, []),
 }
 
 _lib = None

@@ -2,6 +2,7 @@
 // Host-side validation happens before any launch; kernels live in the other
 // translation units (quantize.cu, double_quant.cu, dequantize.cu, gemv.cu,
 // gemm_sm100.cu).
+#include <atomic>
 #include <mutex>
 
 #include "../../include/nf4.h"
@@ -22,6 +23,7 @@ struct DeviceInfo {
 };
 
 std::mutex g_mutex;
+std::atomic<uint64_t> g_launches{0};
 DeviceInfo g_info[kMaxDevices];
 
 // Info of the current device, filled on first use.
@@ -68,7 +70,13 @@ nf4_status check_weight(const nf4_weight* w, nf4::Scales* s) {
 
 }  // namespace
 
+namespace nf4 {
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace nf4
+
 extern "C" {
+
+uint64_t nf4_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 const char* nf4_status_string(nf4_status s) {
   switch (s) {

@@ -34,44 +34,58 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restri
   const int sub = threadIdx.x & 3;
   const int64_t nfull = n / kBlock;
   const int64_t nblocks = (n + kBlock - 1) / kBlock;
-  const int64_t stride = (int64_t)gridDim.x * (blockDim.x / 4);
+  const int64_t groups = (int64_t)gridDim.x * (blockDim.x / 4);
+  const int64_t gid = (int64_t)blockIdx.x * (blockDim.x / 4) + (threadIdx.x >> 2);
+  constexpr int kUnroll = 4;  // blocks per group per iteration: four loads in flight per lane
 
-  for (int64_t b = (int64_t)blockIdx.x * (blockDim.x / 4) + (threadIdx.x >> 2); b < nblocks; b += stride) {
-    const int64_t first = b * kBlock + sub * 16;
-    const float a = block_scale<kDQ>(s, unit_lut, b);
-    if (b < nfull) {
-      uint2 pk = __ldcs(reinterpret_cast<const uint2*>(packed + first / 2));
-      float v[16];
+  for (int64_t b0 = gid; b0 < nblocks; b0 += groups * kUnroll) {
+    uint2 pk[kUnroll];
+    float a[kUnroll];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t lo = (pk.x >> (8 * j)) & 0xffu, hi = (pk.y >> (8 * j)) & 0xffu;
-        v[2 * j] = __fmul_rn(code[lo >> 4], a);
-        v[2 * j + 1] = __fmul_rn(code[lo & 15], a);
-        v[8 + 2 * j] = __fmul_rn(code[hi >> 4], a);
-        v[8 + 2 * j + 1] = __fmul_rn(code[hi & 15], a);
-      }
-      if (kBF16) {
-        uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + first);
-        __stcs(o, make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                             pack_bf16x2(v[6], v[7])));
-        __stcs(o + 1, make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
-                                 pack_bf16x2(v[14], v[15])));
+    for (int u = 0; u < kUnroll; ++u) {  // issue every load first
+      const int64_t b = b0 + u * groups;
+      pk[u] = (b < nfull) ? __ldcs(reinterpret_cast<const uint2*>(packed + b * (kBlock / 2) + sub * 8))
+                          : make_uint2(0, 0);
+      a[u] = (b < nblocks) ? block_scale<kDQ>(s, unit_lut, b) : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t b = b0 + u * groups;
+      if (b >= nblocks) break;
+      const int64_t first = b * kBlock + sub * 16;
+      if (b < nfull) {
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t lo = (pk[u].x >> (8 * j)) & 0xffu, hi = (pk[u].y >> (8 * j)) & 0xffu;
+          v[2 * j] = __fmul_rn(code[lo >> 4], a[u]);
+          v[2 * j + 1] = __fmul_rn(code[lo & 15], a[u]);
+          v[8 + 2 * j] = __fmul_rn(code[hi >> 4], a[u]);
+          v[8 + 2 * j + 1] = __fmul_rn(code[hi & 15], a[u]);
+        }
+        if (kBF16) {
+          uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + first);
+          __stcs(o, make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                               pack_bf16x2(v[6], v[7])));
+          __stcs(o + 1, make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
+                                   pack_bf16x2(v[14], v[15])));
+        } else {
+          float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + first);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) __stcs(o + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+        }
       } else {
-        float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + first);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) __stcs(o + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
-      }
-    } else {
 #pragma unroll 1
-      for (int i = 0; i < 16; ++i) {
-        const int64_t e = first + i;
-        if (e >= n) break;
-        const uint8_t byte = packed[e / 2];
-        const float v = __fmul_rn(code[(e & 1) ? (byte & 15) : (byte >> 4)], a);
-        if (kBF16)
-          static_cast<uint16_t*>(out)[e] = (uint16_t)(pack_bf16x2(v, 0.0f) & 0xffffu);
-        else
-          static_cast<float*>(out)[e] = v;
+        for (int i = 0; i < 16; ++i) {
+          const int64_t e = first + i;
+          if (e >= n) break;
+          const uint8_t byte = packed[e / 2];
+          const float v = __fmul_rn(code[(e & 1) ? (byte & 15) : (byte >> 4)], a[u]);
+          if (kBF16)
+            static_cast<uint16_t*>(out)[e] = (uint16_t)(pack_bf16x2(v, 0.0f) & 0xffffu);
+          else
+            static_cast<float*>(out)[e] = v;
+        }
       }
     }
   }
@@ -82,7 +96,7 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restri
 cudaError_t launch_dequantize(const uint8_t* packed, const Scales& s, int64_t n, void* out, bool out_bf16,
                               cudaStream_t stream, int num_sms) {
   const int64_t nblocks = (n + kBlock - 1) / kBlock;
-  int64_t grid = (nblocks + 63) / 64;
+  int64_t grid = (nblocks + 255) / 256;
   const int64_t cap = (int64_t)num_sms * 8;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
@@ -91,6 +105,7 @@ cudaError_t launch_dequantize(const uint8_t* packed, const Scales& s, int64_t n,
   if (dq && !out_bf16) dequantize_kernel<true, false><<<(unsigned)grid, 256, 0, stream>>>(packed, s, n, out);
   if (!dq && out_bf16) dequantize_kernel<false, true><<<(unsigned)grid, 256, 0, stream>>>(packed, s, n, out);
   if (!dq && !out_bf16) dequantize_kernel<false, false><<<(unsigned)grid, 256, 0, stream>>>(packed, s, n, out);
+  count_launches(1);
   return cudaGetLastError();
 }
 

@@ -46,22 +46,31 @@ __device__ __forceinline__ void add_value(long long (&acc)[kLimbs], float x) {
   for (int L = 0; L < kLimbs; ++L) acc[L] += (L == li) ? lo : ((L == li + 1) ? hi : 0);
 }
 
-// bits [pos, pos + cnt) of the normalised limbs (cnt <= 32), as an integer
-__device__ uint64_t limb_bits(const uint32_t* d, int pos, int cnt) {
-  uint64_t r = 0;
-  for (int i = 0; i < cnt; ++i) {
-    const int p = pos + i;
-    if (p < 0 || p >= 32 * kLimbs) continue;
-    r |= (uint64_t)((d[p >> 5] >> (p & 31)) & 1u) << i;
-  }
-  return r;
+// limb i of d (0 <= i < kLimbs), else 0; unrolled so d stays in registers
+__device__ __forceinline__ uint32_t limb_at(const uint32_t (&d)[kLimbs], int i) {
+  uint32_t v = 0;
+#pragma unroll
+  for (int L = 0; L < kLimbs; ++L) v = (L == i) ? d[L] : v;
+  return v;
+}
+
+// bits [pos, pos + 64) of the 320-bit number d (pos may be negative)
+__device__ __forceinline__ uint64_t window64(const uint32_t (&d)[kLimbs], int pos) {
+  const int i = pos >> 5;  // floor division
+  const int s = pos & 31;
+  const uint32_t l0 = limb_at(d, i), l1 = limb_at(d, i + 1), l2 = limb_at(d, i + 2);
+  const uint64_t lo = ((uint64_t)l1 << 32) | l0;
+  if (s == 0) return lo;
+  return (lo >> s) | ((uint64_t)l2 << (64 - s));
 }
 
 // Normalise the signed limbs, round the total to fp64 (nearest even) and
-// return mu = fp32(fp64 sum / nb).  Single thread.
-__device__ float finish_mean(const long long* limb_in, int64_t nb) {
+// return mu = fp32(fp64 sum / nb).  Single thread, registers only.
+__device__ float finish_mean(const long long (&limb_in)[kLimbs], int64_t nb) {
   long long l[kLimbs];
+#pragma unroll
   for (int L = 0; L < kLimbs; ++L) l[L] = limb_in[L];
+#pragma unroll
   for (int L = 0; L < kLimbs - 1; ++L) {  // carry: limbs 0..8 into [0, 2^32)
     const long long carry = l[L] >> 32;   // arithmetic shift = floor division
     l[L] -= carry * (1LL << 32);
@@ -71,34 +80,43 @@ __device__ float finish_mean(const long long* limb_in, int64_t nb) {
   uint32_t d[kLimbs];
   if (neg) {  // magnitude of a negative total: subtract from zero
     long long borrow = 0;
+#pragma unroll
     for (int L = 0; L < kLimbs - 1; ++L) {
-      long long t = -l[L] - borrow;
+      const long long t = -l[L] - borrow;
       borrow = t < 0;
       d[L] = (uint32_t)(t + (borrow ? (1LL << 32) : 0));
     }
     d[kLimbs - 1] = (uint32_t)(-l[kLimbs - 1] - borrow);
   } else {
+#pragma unroll
     for (int L = 0; L < kLimbs; ++L) d[L] = (uint32_t)l[L];
   }
-  int top = -1;
-  for (int p = 32 * kLimbs - 1; p >= 0; --p)
-    if ((d[p >> 5] >> (p & 31)) & 1u) {
-      top = p;
-      break;
-    }
+  int top = -1;  // index of the highest set bit
+#pragma unroll
+  for (int L = 0; L < kLimbs; ++L)
+    if (d[L]) top = 32 * L + 31 - __clz(d[L]);
   double s = 0.0;
   if (top >= 0) {
     uint64_t m;
     int exp2;  // s = m * 2^exp2
     if (top < 53) {
-      m = limb_bits(d, 0, 32) | (limb_bits(d, 32, 21) << 32);
+      m = window64(d, 0);
       exp2 = -149;
     } else {
-      const int low = top - 52;
-      m = limb_bits(d, low, 32) | (limb_bits(d, low + 32, 21) << 32);
-      const bool round = limb_bits(d, low - 1, 1) != 0;
-      bool sticky = false;
-      for (int p = 0; p < low - 1 && !sticky; ++p) sticky = (d[p >> 5] >> (p & 31)) & 1u;
+      const int low = top - 52;  // lowest kept bit
+      const uint64_t w = window64(d, low - 1);  // round bit + 53 kept bits
+      m = (w >> 1) & ((1ull << 53) - 1);
+      const bool round = w & 1u;
+      bool sticky = false;  // any set bit below low - 1
+      const int sb = low - 1;
+#pragma unroll
+      for (int L = 0; L < kLimbs; ++L) {
+        const int base = 32 * L;
+        uint32_t mask = 0;
+        if (base + 32 <= sb) mask = 0xffffffffu;
+        else if (base < sb) mask = (1u << (sb - base)) - 1u;
+        sticky |= (d[L] & mask) != 0;
+      }
       if (round && (sticky || (m & 1u))) m += 1;  // may reach 2^53: still exact
       exp2 = low - 149;
     }
@@ -140,6 +158,7 @@ __global__ void __launch_bounds__(256) dq_sum_kernel(const float* __restrict__ a
   if (last && threadIdx.x == 0) {
     __threadfence();
     long long l[kLimbs];
+#pragma unroll
     for (int L = 0; L < kLimbs; ++L) l[L] = (long long)atomicAdd(&ws->limb[L], 0ull);
     *mean_out = finish_mean(l, nb);
   }
@@ -215,6 +234,7 @@ cudaError_t launch_double_quant(const float* absmax, int64_t nb, int dq_code, ui
   const int64_t ngroups = (nb + kDqBlock - 1) / kDqBlock;
   const int64_t grid2 = (ngroups + 7) / 8;
   dq_code_kernel<<<(unsigned)grid2, 256, 0, stream>>>(absmax, nb, dq_code, mean, q, scale);
+  count_launches(2);
   return cudaGetLastError();
 }
 

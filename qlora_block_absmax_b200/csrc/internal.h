@@ -11,6 +11,9 @@ constexpr int kDqBlock = 256;   // level-2 block (absmax values per second-level
 
 // Level-1 scales as the kernels see them: plain fp32 absmax, or the
 // double-quantized record (8-bit codes + second-level block absmax + mean).
+// count of kernels launched (read by nf4_kernel_launches)
+void count_launches(int n);
+
 struct Scales {
   const float* absmax;   // non-null: plain scales
   const uint8_t* q;      // double-quantized codes

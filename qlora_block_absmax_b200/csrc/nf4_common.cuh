@@ -24,8 +24,8 @@ constexpr float kInt8Top = 127.0f;
 // error word bits set by device code (read back by nf4_check_device_error)
 constexpr unsigned kErrTimeout = 1u;
 
-// bounded spin limit for mbarrier waits (about a second at B200 clocks)
-constexpr long long kSpinLimit = 1LL << 27;
+// wall-clock bound of every device-side wait (nanoseconds)
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t d;
@@ -104,12 +104,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for phase `parity` of a barrier, giving up after kSpinLimit polls: on
-// timeout the error word gets kErrTimeout and the function returns false so
-// the caller can leave the loop instead of hanging the GPU.
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for phase `parity` of a barrier, giving up after kWaitLimitNs of wall
+// clock: on timeout the error word gets kErrTimeout and the function returns
+// false so the caller can leave its loop instead of hanging the GPU.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, unsigned* err) {
-  for (long long i = 0; i < kSpinLimit; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) break;
+  }
   if (err) atomicOr(err, kErrTimeout);
   return false;
 }

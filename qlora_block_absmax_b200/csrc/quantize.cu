@@ -7,40 +7,44 @@
 //   Step 4  two 4-bit codes share one byte; the scales are stored beside them.
 //
 // Layout: four lanes own one 64-element block, 16 consecutive elements each
-// (two 16-byte loads for bf16, four for fp32).  The block absmax is a 4-lane
-// shuffle reduction.  The nearest code of x = RN(w / a) is the number of
-// thresholds below x; a 514-entry bucket table in shared memory turns that
-// into one lookup and one compare.  x is first estimated as w * RN(1/a); when
-// the estimate lies within 2^-19 of the bucket's threshold (where the estimate
-// and the IEEE quotient could fall on different sides) the exact quotient
-// __fdiv_rn(w, a) decides, so every code equals the one of the IEEE quotient.
+// (two 16-byte loads for bf16, four for fp32); a warp covers 8 consecutive
+// blocks per iteration and iterates uniformly (the lookup is a warp shuffle).
+// The block absmax is a 4-lane shuffle reduction.
+//
+// Nearest code of x = RN(w / a): the number of thresholds (exact code
+// midpoints rounded down to fp32) below x.  A 32-bucket table covers [-1, 1];
+// lane j of every warp holds bucket j: the one threshold inside it (2.0 if
+// none) with the count of thresholds below the bucket in its low 4 mantissa
+// bits.  x is first estimated as q = w * RN(1/a) (within 3 * 2^-24 of x); q
+// picks the bucket, a shuffle fetches the entry, and code = base + (q > entry).
+// When q lies within 2^-19 of the entry -- where the estimate, or the 4 bits
+// stored in the entry, could change the decision -- the exact quotient
+// __fdiv_rn(w, a) is compared with the exact threshold instead.  Every code is
+// therefore the one of the IEEE quotient.
 #include "nf4_common.cuh"
 #include "internal.h"
 
 namespace nf4 {
 namespace {
 
-__constant__ float c_bucket_thr[NF4_NUM_BUCKETS] = NF4_BUCKET_THRESHOLD_INIT;
-__constant__ unsigned char c_bucket_base[NF4_NUM_BUCKETS] = NF4_BUCKET_BASE_INIT;
+__constant__ uint32_t c_q32[32] = NF4_Q32_INIT;
+__constant__ float c_threshold[15] = NF4_THRESHOLD_INIT;
 
-struct Bucket {
-  float thr;
-  int base;
-};
+constexpr float kNearThreshold = 0x1p-19f;
+constexpr float kTinyScale = 0x1p-120f;  // below this 1/a may overflow: divide exactly
 
-constexpr float kNearThreshold = 0x1p-19f;   // estimate is within 3 * 2^-24 of the quotient
-constexpr float kTinyScale = 0x1p-120f;      // below this 1/a may overflow: divide exactly
-
-__device__ __forceinline__ int code_of(const Bucket* tab, float w, float a, float r, bool exact) {
-  float q = exact ? __fdiv_rn(w, a) : __fmul_rn(w, r);
-  float v = __fmaf_rn(q, 0.5f, NF4_BUCKET_BIAS);
-  unsigned bk = (unsigned)((__float_as_int(v) >> NF4_BUCKET_SHIFT) - (0x40000000 >> NF4_BUCKET_SHIFT));
-  bk = min(bk, (unsigned)(NF4_NUM_BUCKETS - 1));  // NaN/Inf inputs stay in bounds
-  Bucket e = tab[bk];
-  int code = e.base + (q > e.thr ? 1 : 0);
-  if (!exact && fabsf(q - e.thr) <= kNearThreshold) {
-    float x = __fdiv_rn(w, a);
-    code = e.base + (x > e.thr ? 1 : 0);
+// `entry` is this lane's bucket word; every lane of the warp must call this
+__device__ __forceinline__ int code_of(uint32_t entry, float w, float a, float r, bool exact) {
+  const float q = exact ? __fdiv_rn(w, a) : __fmul_rn(w, r);
+  const float v = __fmaf_rn(q, NF4_Q32_SCALE, 3.0f);
+  const int bk = (__float_as_int(v) >> 18) & 31;  // NaN/Inf inputs still land in 0..31
+  const uint32_t e = __shfl_sync(0xffffffffu, entry, bk);
+  const int base = (int)(e & 15u);
+  const float thr = __uint_as_float(e);
+  int code = base + (q > thr ? 1 : 0);
+  if (fabsf(q - thr) <= kNearThreshold) {
+    const float x = exact ? q : __fdiv_rn(w, a);
+    code = base + (x > c_threshold[base < 15 ? base : 14] ? 1 : 0);
   }
   return code;
 }
@@ -79,74 +83,68 @@ template <bool kBF16>
 __global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ src, int64_t n,
                                                        uint8_t* __restrict__ packed,
                                                        float* __restrict__ absmax) {
-  __shared__ Bucket tab[NF4_NUM_BUCKETS];
-  for (int i = threadIdx.x; i < NF4_NUM_BUCKETS; i += blockDim.x) tab[i] = Bucket{c_bucket_thr[i], (int)c_bucket_base[i]};
-  __syncthreads();
-
   const int lane = threadIdx.x & 31;
+  const uint32_t entry = c_q32[lane];
   const int sub = lane & 3;                                  // which 16 of the block's 64
   const unsigned gmask = 0xfu << (lane & ~3);                // the 4 lanes of this block
   const int64_t nfull = n / kBlock;
   const int64_t nblocks = (n + kBlock - 1) / kBlock;
-  const int64_t stride = (int64_t)gridDim.x * (blockDim.x / 4);
+  const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int64_t warp_id = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
 
-  for (int64_t b = (int64_t)blockIdx.x * (blockDim.x / 4) + (threadIdx.x >> 2); b < nblocks; b += stride) {
+  for (int64_t wb = warp_id * 8; wb < nblocks; wb += warps_total * 8) {  // uniform per warp
+    const int64_t b = wb + (lane >> 2);
+    const bool live = b < nblocks;
     const int64_t first = b * kBlock + sub * 16;
     float w[16];
-    if (b < nfull) {
+    if (live && b < nfull) {
       load16<kBF16>(src, first, w);
-    } else {  // short last block: missing elements read as 0 (they do not change the absmax)
+    } else {  // short last block (or no block): missing elements read as 0
 #pragma unroll
-      for (int i = 0; i < 16; ++i) w[i] = (first + i < n) ? load1<kBF16>(src, first + i) : 0.0f;
+      for (int i = 0; i < 16; ++i) w[i] = (live && first + i < n) ? load1<kBF16>(src, first + i) : 0.0f;
     }
     // Step 2: block absmax (exact; max is order-free)
     float a = 0.0f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(w[i]));
-    a = fmaxf(a, __shfl_xor_sync(gmask, a, 1));
-    a = fmaxf(a, __shfl_xor_sync(gmask, a, 2));
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
 
-    // Step 3: nearest code of RN(w / a); all-zero block -> zero code (7)
-    uint32_t lo = 0x77777777u, hi = 0x77777777u;
-    if (a > 0.0f) {
-      const bool exact = a < kTinyScale;
-      const float r = exact ? 0.0f : __frcp_rn(a);
-      int c[16];
+    // Step 3: nearest code of RN(w / a); an all-zero block takes the zero code (7)
+    const bool zero = !(a > 0.0f);
+    const bool exact = a < kTinyScale;
+    const float r = exact ? 0.0f : __frcp_rn(a);
+    const float as = zero ? 1.0f : a;  // keeps the (discarded) zero-block arithmetic finite
+    int c[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) c[i] = code_of(tab, w[i], a, r, exact);
-      // Step 4: element 2j -> high nibble of byte j
-      lo = 0;
-      hi = 0;
+    for (int i = 0; i < 16; ++i) c[i] = code_of(entry, w[i], as, r, exact && !zero);
+    // Step 4: element 2j -> high nibble of byte j
+    uint32_t lo = 0, hi = 0;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        lo |= (uint32_t)((c[2 * j] << 4) | c[2 * j + 1]) << (8 * j);
-        hi |= (uint32_t)((c[8 + 2 * j] << 4) | c[8 + 2 * j + 1]) << (8 * j);
-      }
+    for (int j = 0; j < 4; ++j) {
+      lo |= (uint32_t)((c[2 * j] << 4) | c[2 * j + 1]) << (8 * j);
+      hi |= (uint32_t)((c[8 + 2 * j] << 4) | c[8 + 2 * j + 1]) << (8 * j);
     }
+    if (zero) lo = hi = 0x77777777u;
+    if (!live) continue;
     if (b < nfull) {
       *reinterpret_cast<uint2*>(packed + first / 2) = make_uint2(lo, hi);
     } else {
-      // short block: write only the bytes that hold real elements; an odd
-      // tail keeps the zero code (7) in its low nibble
-      const int64_t nbytes = (n + 1) / 2;
-      uint8_t bytes[8];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        bytes[j] = (uint8_t)(lo >> (8 * j));
-        bytes[4 + j] = (uint8_t)(hi >> (8 * j));
-      }
+      // short block: write only bytes holding real elements; an odd tail keeps
+      // the zero code (7) in its low nibble
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int64_t e = first + 2 * j;  // element in the high nibble
         if (e < n) {
-          uint8_t v = bytes[j];
+          uint8_t v = (uint8_t)((j < 4 ? lo : hi) >> (8 * (j & 3)));
           if (e + 1 >= n) v = (uint8_t)((v & 0xf0u) | 0x7u);
-          if (first / 2 + j < nbytes) packed[first / 2 + j] = v;
+          packed[first / 2 + j] = v;
         }
       }
     }
     if (sub == 0) absmax[b] = a;
   }
+  (void)gmask;
 }
 
 }  // namespace
@@ -163,6 +161,7 @@ cudaError_t launch_quantize(const void* src, bool bf16, int64_t n, uint8_t* pack
     quantize_kernel<true><<<(unsigned)grid, 256, 0, stream>>>(src, n, packed, absmax);
   else
     quantize_kernel<false><<<(unsigned)grid, 256, 0, stream>>>(src, n, packed, absmax);
+  count_launches(1);
   return cudaGetLastError();
 }
 
