@@ -23,7 +23,7 @@ from . import _lib
 from ._lib import NF4_BF16, NF4_DQ_E4M3, NF4_DQ_INT8, NF4_F32, NF4Error
 
 __all__ = ["QuantizedWeight", "quantize", "double_quant", "quantize_weight", "dequantize", "gemv", "gemm",
-           "storage_bytes", "code_table", "check_device_error", "kernel_launches", "NF4Error", "library_path"]
+           "storage_bytes", "gemm_workspace_bytes", "code_table", "check_device_error", "kernel_launches", "NF4Error", "library_path"]
 
 BLOCKSIZE = 64
 DQ_BLOCKSIZE = 256
@@ -180,6 +180,12 @@ def gemm(qw: QuantizedWeight, x: torch.Tensor, out=None, workspace: Optional[tor
                       workspace.numel() if workspace is not None else 0, _stream(stream))
     _lib.check(st, "nf4_gemm")
     return out
+
+
+def gemm_workspace_bytes(qw: QuantizedWeight, m: int) -> int:
+    """Scratch bytes nf4_gemm needs for `m` activation rows (0 when none)."""
+    d = qw.descriptor()
+    return int(_lib.load().nf4_gemm_workspace_bytes(ctypes.byref(d), m))
 
 
 def storage_bytes(n: int, use_double_quant: bool = True) -> int:

@@ -149,7 +149,7 @@ nf4_status nf4_double_quant(const float* absmax, int64_t nb, int32_t dq_blocksiz
   nf4_status st = device_info(&d);
   if (st != NF4_OK) return st;
   return from_cuda(nf4::launch_double_quant(absmax, nb, dq_code, q_out, scale_out, mean_out, workspace,
-                                            reinterpret_cast<cudaStream_t>(stream), d.num_sms));
+                                            d.error_word, reinterpret_cast<cudaStream_t>(stream), d.num_sms));
 }
 
 nf4_status nf4_dequantize(const nf4_weight* w, void* out, int32_t out_dtype, nf4_stream_t stream) {

@@ -9,13 +9,13 @@
 // or int8 (Q = 127, half away from zero, clamped).  The mean is removed first
 // (one fp32 per tensor): mu = fp32(fp64(exact sum) / nb).
 //
-// Kernel 1 (sum): every fp32 value is an integer multiple of 2^-149, so each
-// thread adds its values into ten signed 64-bit limbs holding 32 bits each of
-// a 320-bit fixed-point number; integer addition makes the total exact and
-// independent of order.  Warp shuffles and shared memory combine threads,
-// 64-bit atomics combine CTAs, and the last CTA to finish normalises the limbs,
-// rounds the sum once to fp64 and writes mu.
-// Kernel 2 (codes): one warp per 256-value block.
+// Sum: every fp32 value is an integer multiple of 2^-149, so each thread adds
+// its values into ten signed 64-bit limbs holding 32 bits each of a 320-bit
+// fixed-point number; integer addition makes the total exact and independent
+// of order.  Warp shuffles and shared memory combine threads, 64-bit atomics
+// combine CTAs.  After a grid barrier every CTA normalises the same limbs,
+// rounds the sum once to fp64 and derives mu.
+// Codes: one warp per 256-value block.
 #include "nf4_common.cuh"
 #include "internal.h"
 
@@ -127,20 +127,35 @@ __device__ float finish_mean(const long long (&limb_in)[kLimbs], int64_t nb) {
   return __double2float_rn(__ddiv_rn(s, (double)nb));
 }
 
-__global__ void __launch_bounds__(256) dq_sum_kernel(const float* __restrict__ a, int64_t nb,
-                                                     SumWorkspace* __restrict__ ws, float* __restrict__ mean_out) {
+// One cooperative launch (every CTA resident): exact sum -> grid barrier ->
+// codes.  The barrier spins on a counter with a wall-clock bound; if it runs
+// out the error word is set and the codes are skipped.
+__global__ void __launch_bounds__(256) dq_fused_kernel(const float* __restrict__ a, int64_t nb, int dq_code,
+                                                       uint8_t* __restrict__ q, float* __restrict__ scale,
+                                                       float* __restrict__ mean_out, SumWorkspace* __restrict__ ws,
+                                                       unsigned* __restrict__ err) {
+  // ---- phase 1: this thread's values into the integer limbs
   long long acc[kLimbs];
 #pragma unroll
   for (int L = 0; L < kLimbs; ++L) acc[L] = 0;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nb; i += (int64_t)gridDim.x * blockDim.x)
-    add_value(acc, a[i]);
+  const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t n4 = nb / 4;  // absmax is 16-byte aligned: float4 loads for the body
+  for (int64_t i = tid; i < n4; i += nthreads) {
+    const float4 v = reinterpret_cast<const float4*>(a)[i];
+    add_value(acc, v.x);
+    add_value(acc, v.y);
+    add_value(acc, v.z);
+    add_value(acc, v.w);
+  }
+  for (int64_t i = 4 * n4 + tid; i < nb; i += nthreads) add_value(acc, a[i]);
 #pragma unroll
   for (int L = 0; L < kLimbs; ++L)
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc[L] += __shfl_xor_sync(0xffffffffu, acc[L], off);
-
   __shared__ long long red[8][kLimbs];
-  __shared__ bool last;
+  __shared__ float s_mu;
+  __shared__ int s_ok;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (lane == 0)
 #pragma unroll
@@ -153,89 +168,111 @@ __global__ void __launch_bounds__(256) dq_sum_kernel(const float* __restrict__ a
   }
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) last = atomicAdd(&ws->done, 1u) == gridDim.x - 1;
-  __syncthreads();
-  if (last && threadIdx.x == 0) {
-    __threadfence();
-    long long l[kLimbs];
-#pragma unroll
-    for (int L = 0; L < kLimbs; ++L) l[L] = (long long)atomicAdd(&ws->limb[L], 0ull);
-    *mean_out = finish_mean(l, nb);
-  }
-}
 
-__global__ void __launch_bounds__(256) dq_code_kernel(const float* __restrict__ a, int64_t nb, int dq_code,
-                                                      const float* __restrict__ mean, uint8_t* __restrict__ q,
-                                                      float* __restrict__ scale) {
-  const int lane = threadIdx.x & 31;
-  const int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  // ---- grid barrier (bounded)
+  if (threadIdx.x == 0) {
+    atomicAdd(&ws->done, 1u);
+    int ok = 1;
+    const unsigned long long t0 = global_ns();
+    while (atomicAdd(&ws->done, 0u) < gridDim.x) {
+      if (global_ns() - t0 > kWaitLimitNs) {
+        atomicOr(err, kErrTimeout);
+        ok = 0;
+        break;
+      }
+    }
+    __threadfence();
+    if (ok) {
+      long long l[kLimbs];
+#pragma unroll
+      for (int L = 0; L < kLimbs; ++L) l[L] = (long long)atomicAdd(&ws->limb[L], 0ull);
+      s_mu = finish_mean(l, nb);  // the same integers in every CTA: the same mu
+      if (blockIdx.x == 0) *mean_out = s_mu;
+    }
+    s_ok = ok;
+  }
+  __syncthreads();
+  if (!s_ok) return;
+  const float mu = s_mu;
+
+  // ---- phase 2: one warp per block of kDqBlock residuals
   const int64_t ngroups = (nb + kDqBlock - 1) / kDqBlock;
-  if (g >= ngroups) return;  // whole warp leaves together
-  const float mu = *mean;
-  const int64_t first = g * kDqBlock + lane * 8;
-  const bool full = (g + 1) * kDqBlock <= nb;
-  float r[8];
-  if (full) {
-    const float4* p = reinterpret_cast<const float4*>(a + first);
-    float4 v0 = p[0], v1 = p[1];
-    r[0] = v0.x; r[1] = v0.y; r[2] = v0.z; r[3] = v0.w;
-    r[4] = v1.x; r[5] = v1.y; r[6] = v1.z; r[7] = v1.w;
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) r[i] = (first + i < nb) ? a[first + i] : mu;  // mu -> residual 0
-  }
-  float m = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    r[i] = __fsub_rn(r[i], mu);  // residual after removing the mean
-    m = fmaxf(m, fabsf(r[i]));
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-  if (lane == 0) scale[g] = m;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
   const float Q = dq_code == 0 ? kE4M3Top : kInt8Top;
-  float y[8];
+  for (int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp; g < ngroups; g += nwarps) {
+    const int64_t first = g * kDqBlock + lane * 8;
+    const bool full = (g + 1) * kDqBlock <= nb;
+    float r[8];
+    if (full) {
+      const float4* p = reinterpret_cast<const float4*>(a + first);
+      const float4 v0 = p[0], v1 = p[1];
+      r[0] = v0.x; r[1] = v0.y; r[2] = v0.z; r[3] = v0.w;
+      r[4] = v1.x; r[5] = v1.y; r[6] = v1.z; r[7] = v1.w;
+    } else {
 #pragma unroll
-  for (int i = 0; i < 8; ++i) y[i] = (m != 0.0f) ? __fmul_rn(__fdiv_rn(r[i], m), Q) : 0.0f;
-  uint32_t lo, hi;
-  if (dq_code == 0) {
-    lo = pack_e4m3x2(y[0], y[1]) | (pack_e4m3x2(y[2], y[3]) << 16);
-    hi = pack_e4m3x2(y[4], y[5]) | (pack_e4m3x2(y[6], y[7]) << 16);
-  } else {
-    uint32_t b[8];
+      for (int i = 0; i < 8; ++i) r[i] = (first + i < nb) ? a[first + i] : mu;  // mu -> residual 0
+    }
+    float m = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      float t = fminf(fmaxf(roundf(y[i]), -127.0f), 127.0f);  // half away from zero, clamp
-      b[i] = (uint32_t)(uint8_t)(int8_t)(int)t;
+      r[i] = __fsub_rn(r[i], mu);  // residual after removing the mean
+      m = fmaxf(m, fabsf(r[i]));
     }
-    lo = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
-    hi = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
-  }
-  if (full) {
-    *reinterpret_cast<uint2*>(q + first) = make_uint2(lo, hi);
-  } else {
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if (first + i < nb) q[first + i] = (uint8_t)((i < 4 ? lo : hi) >> (8 * (i & 3)));
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if (lane == 0) scale[g] = m;
+    float y[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = (m != 0.0f) ? __fmul_rn(__fdiv_rn(r[i], m), Q) : 0.0f;
+    uint32_t lo, hi;
+    if (dq_code == 0) {
+      lo = pack_e4m3x2(y[0], y[1]) | (pack_e4m3x2(y[2], y[3]) << 16);
+      hi = pack_e4m3x2(y[4], y[5]) | (pack_e4m3x2(y[6], y[7]) << 16);
+    } else {
+      uint32_t bb[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float t = fminf(fmaxf(roundf(y[i]), -127.0f), 127.0f);  // half away from zero, clamp
+        bb[i] = (uint32_t)(uint8_t)(int8_t)(int)t;
+      }
+      lo = bb[0] | (bb[1] << 8) | (bb[2] << 16) | (bb[3] << 24);
+      hi = bb[4] | (bb[5] << 8) | (bb[6] << 16) | (bb[7] << 24);
+    }
+    if (full) {
+      *reinterpret_cast<uint2*>(q + first) = make_uint2(lo, hi);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (first + i < nb) q[first + i] = (uint8_t)((i < 4 ? lo : hi) >> (8 * (i & 3)));
+    }
   }
 }
 
 }  // namespace
 
 cudaError_t launch_double_quant(const float* absmax, int64_t nb, int dq_code, uint8_t* q, float* scale,
-                                float* mean, void* workspace, cudaStream_t stream, int num_sms) {
-  cudaError_t err = cudaMemsetAsync(workspace, 0, sizeof(SumWorkspace), stream);
-  if (err != cudaSuccess) return err;
-  int64_t grid1 = (nb + 256 * 8 - 1) / (256 * 8);
-  if (grid1 > num_sms) grid1 = num_sms;
-  if (grid1 < 1) grid1 = 1;
-  dq_sum_kernel<<<(unsigned)grid1, 256, 0, stream>>>(absmax, nb, static_cast<SumWorkspace*>(workspace), mean);
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  const int64_t ngroups = (nb + kDqBlock - 1) / kDqBlock;
-  const int64_t grid2 = (ngroups + 7) / 8;
-  dq_code_kernel<<<(unsigned)grid2, 256, 0, stream>>>(absmax, nb, dq_code, mean, q, scale);
-  count_launches(2);
-  return cudaGetLastError();
+                                float* mean, void* workspace, unsigned* err, cudaStream_t stream, int num_sms) {
+  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(SumWorkspace), stream);
+  if (e != cudaSuccess) return e;
+  // one CTA per SM: 256 threads and ~1 KB of shared memory, so all are resident
+  int64_t grid = (nb + 256 * 4 - 1) / (256 * 4);
+  if (grid > num_sms) grid = num_sms;
+  if (grid < 1) grid = 1;
+  auto* ws = static_cast<SumWorkspace*>(workspace);
+  void* args[] = {(void*)&absmax, (void*)&nb, (void*)&dq_code, (void*)&q, (void*)&scale, (void*)&mean, (void*)&ws,
+                  (void*)&err};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelExC(&cfg, (const void*)dq_fused_kernel, args);
+  count_launches(1);
+  return e;
 }
 
 }  // namespace nf4

@@ -22,6 +22,8 @@
 // the roles leave their loops, so a fault cannot hang the GPU.
 #include <cuda.h>
 
+#include <atomic>
+
 #include "nf4_common.cuh"
 #include "nf4_decode.cuh"
 #include "internal.h"
@@ -32,25 +34,38 @@ namespace {
 constexpr int kTileN = 128;       // weight rows per tile (UMMA M)
 constexpr int kTileM = 256;       // activation rows per tile (UMMA N)
 constexpr int kTileK = 64;        // k per stage (128 bytes of bf16: one swizzle atom)
-constexpr int kStages = 4;
-constexpr int kABytes = kTileN * kTileK * 2;  // 16 KB
-constexpr int kBBytes = kTileM * kTileK * 2;  // 32 KB
+constexpr int kXStages = 4;  // activation-tile ring (TMA from L2/HBM)
+constexpr int kAStages = 3;  // decoded weight-tile ring (written by the producer warps)
+constexpr int kWStages = 6;  // packed-code + scale ring (TMA from HBM), deeper to hide its latency
+constexpr int kABytes = kTileN * kTileK * 2;  // 16 KB: decoded bf16 weight tile (operand A)
+constexpr int kBBytes = kTileM * kTileK * 2;  // 32 KB: activation tile (operand B)
+constexpr int kWBytes = kTileN * kTileK / 2;  // 4 KB: packed codes of the weight tile
+constexpr int kSBytes = kTileN * 16;          // 2 KB: 16-byte scale chunk per weight row
+constexpr int kRingBytes = kAStages * kABytes + kXStages * kBBytes + kWStages * (kWBytes + kSBytes);
 constexpr int kAccCols = kTileM;              // fp32 columns per accumulator
 constexpr int kTmemCols = 2 * kAccCols;       // 512
-constexpr int kThreads = 14 * 32;
+constexpr int kThreads = 15 * 32;
 constexpr int kEpiWarps = 4;
 constexpr int kProdWarp0 = 4;                 // producers: warps 4..11
-constexpr int kTmaWarp = 12;
+constexpr int kTmaWarp = 12;                  // activation tiles
 constexpr int kMmaWarp = 13;
-constexpr size_t kSmemBytes = (size_t)kStages * (kABytes + kBBytes) + 1024 /*align*/ + 2048 /*barriers, lut*/;
+constexpr int kTmaWWarp = 14;                 // packed codes and scales
+constexpr int kStageOutBytes = 32 * 32 * 2;    // per epilogue warp: 32 rows x 32 columns of bf16
+constexpr size_t kSmemBytes = (size_t)kRingBytes + kEpiWarps * kStageOutBytes + 1024 /*align*/ +
+                              2048 /*barriers, lut*/;
 
 struct Smem {  // placed after the 1024-aligned stage buffers
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t wfull[kWStages];   // packed codes + scale chunk landed (TMA)
+  uint64_t wempty[kWStages];  // codes read by the producer warps
+  uint64_t xfull[kXStages];   // activation tile landed (TMA)
+  uint64_t xempty[kXStages];  // activation tile consumed by the MMAs (tcgen05.commit)
+  uint64_t afull[kAStages];   // decoded weight tile written (producer warps)
+  uint64_t aempty[kAStages];  // decoded tile consumed by the MMAs (tcgen05.commit)
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint32_t tmem_base;
   int abort;
+  int last;
   float unit_lut[256];
 };
 
@@ -121,28 +136,64 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Sm
 
 // ------------------------------------------------------------------ kernel
 
-template <bool kDQ>
+#ifdef NF4_TRACE  // diagnostics build only: per-CTA wall-clock stamps of pipeline milestones
+__device__ unsigned long long g_trace[1024 * 16];
+#define NF4_STAMP(slot) (g_trace[blockIdx.x * 16 + (slot)] = global_ns())
+#else
+#define NF4_STAMP(slot) ((void)0)
+#endif
+
+// Work unit u = tile * splits + split: the split takes k stages
+// [split * kps, (split + 1) * kps).  With splits > 1 the epilogue writes an
+// fp32 partial tile to the workspace and the last split to finish a tile adds
+// the partials in split order (deterministic) and writes bf16 Y.
+struct Work {
+  int ntiles_m, units, splits, kps;
+  __device__ int tile(int u) const { return u / splits; }
+  __device__ int split(int u) const { return u % splits; }
+  __device__ int n0(int u) const { return (tile(u) / ntiles_m) * kTileN; }
+  __device__ int m0(int u) const { return (tile(u) % ntiles_m) * kTileM; }
+};
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory"); }
+
+template <bool kDQ, bool kScaleTma>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_kernel(const uint8_t* __restrict__ packed, Scales s, int rows, int cols, int m_total,
-                const __grid_constant__ CUtensorMap xmap, __nv_bfloat16* __restrict__ y, unsigned* err) {
+    gemm_kernel(Scales s, int rows, int cols, int m_total, int splits, const __grid_constant__ CUtensorMap xmap,
+                const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
+                __nv_bfloat16* __restrict__ y, float* __restrict__ part, unsigned* __restrict__ tile_count,
+                unsigned* err) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;  // 1024-aligned stage buffers (swizzle atoms)
   uint8_t* gbase = smem_raw + (base - raw);
-  const uint32_t a_smem0 = base, b_smem0 = base + kStages * kABytes;
+  const uint32_t a_smem0 = base, b_smem0 = base + kAStages * kABytes;
+  const uint32_t w_smem0 = b_smem0 + kXStages * kBBytes, s_smem0 = w_smem0 + kWStages * kWBytes;
   uint8_t* a_gen0 = gbase;
-  Smem* sm = reinterpret_cast<Smem*>(gbase + kStages * (kABytes + kBBytes));
+  const uint8_t* w_gen0 = gbase + (w_smem0 - base);
+  const uint8_t* s_gen0 = gbase + (s_smem0 - base);
+  uint16_t* out_stage = reinterpret_cast<uint16_t*>(gbase + kRingBytes);  // epilogue transpose
+  Smem* sm = reinterpret_cast<Smem*>(gbase + kRingBytes + kEpiWarps * kStageOutBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ntiles_n = rows / kTileN;
-  const int ntiles_m = (m_total + kTileM - 1) / kTileM;
-  const int ntiles = ntiles_n * ntiles_m;
-  const int kstages = cols / kTileK;
+  Work wk;
+  wk.ntiles_m = (m_total + kTileM - 1) / kTileM;
+  wk.splits = splits;
+  wk.units = (rows / kTileN) * wk.ntiles_m * splits;
+  wk.kps = cols / kTileK / splits;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&sm->full[i], 4 + 1);  // 4 producer warps + the TMA arrive.expect_tx
-      mbar_init(&sm->empty[i], 1);     // tcgen05.commit
+    for (int i = 0; i < kWStages; ++i) {
+      mbar_init(&sm->wfull[i], 1);   // TMA arrive.expect_tx
+      mbar_init(&sm->wempty[i], 4);  // the 4 producer warps of the stage's group
+    }
+    for (int i = 0; i < kXStages; ++i) {
+      mbar_init(&sm->xfull[i], 1);   // TMA arrive.expect_tx
+      mbar_init(&sm->xempty[i], 1);  // tcgen05.commit
+    }
+    for (int i = 0; i < kAStages; ++i) {
+      mbar_init(&sm->afull[i], 4);   // the 4 producer warps of the stage's group
+      mbar_init(&sm->aempty[i], 1);  // tcgen05.commit
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm->acc_full[i], 1);
@@ -162,6 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm->tmem_base;
+  if (threadIdx.x == 0) NF4_STAMP(0);
 
   if (warp >= kProdWarp0 && warp < kTmaWarp) {
     // ------------------------------------------------ dequant producers
@@ -170,24 +222,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float mu = kDQ ? *s.mean : 0.0f;
     const int64_t rb = cols / kBlock;
     uint32_t it = 0;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-      const int64_t row = (int64_t)(tile / ntiles_m) * kTileN + p;
-      for (int ks = 0; ks < kstages; ++ks, ++it) {
+    for (int u = blockIdx.x; u < wk.units; u += gridDim.x) {
+      const int64_t row = (int64_t)wk.n0(u) + p;
+      const int ks0 = wk.split(u) * wk.kps;
+      for (int ks = ks0; ks < ks0 + wk.kps; ++ks, ++it) {
         if ((int)(it & 1) != group) continue;
-        const int st = it % kStages;
-        const uint32_t ph = (it / kStages) & 1;
-        // issue the global loads before waiting for the stage to drain
-        const uint4* src = reinterpret_cast<const uint4*>(packed + row * (cols / 2) + (int64_t)ks * 32);
-        const uint4 w0 = __ldg(src), w1 = __ldg(src + 1);
-        const int64_t b = row * rb + ks;
+        const int ws = it % kWStages, as = it % kAStages;
+        const uint32_t wph = (it / kWStages) & 1, aph = (it / kAStages) & 1;
+        if (!wait_or_abort(&sm->wfull[ws], wph, sm, err)) break;  // codes + scale chunk landed
+        const uint4* wsrc = reinterpret_cast<const uint4*>(w_gen0 + ws * kWBytes + p * 32);
+        const uint4 w0 = wsrc[0], w1 = wsrc[1];
+        const uint8_t* sc = s_gen0 + ws * kSBytes + p * 16;
+        const int64_t b = row * rb + ks;  // level-1 block of this row and stage
+        const uint32_t qcode = kDQ && kScaleTma ? sc[ks & 15] : 0u;
+        const float plain = !kDQ && kScaleTma ? reinterpret_cast<const float*>(sc)[ks & 3] : 0.0f;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm->wempty[ws]);  // the code slot may be refilled
         float a;
         if (kDQ)
-          a = dq_absmax(sm->unit_lut[s.q[b]], s.scale[b / kDqBlock], mu);
+          a = dq_absmax(sm->unit_lut[kScaleTma ? qcode : s.q[b]], __ldg(s.scale + b / kDqBlock), mu);
         else
-          a = __ldg(s.absmax + b);
+          a = kScaleTma ? plain : __ldg(s.absmax + b);
         const Table T = make_table(a);
-        if (!wait_or_abort(&sm->empty[st], ph ^ 1, sm, err)) break;
-        uint8_t* dst = a_gen0 + st * kABytes + p * 128;
+        if (!wait_or_abort(&sm->aempty[as], aph ^ 1, sm, err)) break;  // the MMAs left this slot
+        uint8_t* dst = a_gen0 + as * kABytes + p * 128;
         const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
@@ -197,87 +255,190 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm->full[st]);
+        if (lane == 0) mbar_arrive(&sm->afull[as]);
       }
       if (aborted(sm)) break;
     }
   } else if (warp == kTmaWarp) {
-    // ------------------------------------------------ activation tiles via TMA
+    // ------------------------------------------------ TMA: activation tiles
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
       uint32_t it = 0;
-      for (int tile = blockIdx.x; tile < ntiles && !aborted(sm); tile += gridDim.x) {
-        const int m0 = (tile % ntiles_m) * kTileM;
-        for (int ks = 0; ks < kstages; ++ks, ++it) {
-          const int st = it % kStages;
-          const uint32_t ph = (it / kStages) & 1;
-          if (!wait_or_abort(&sm->empty[st], ph ^ 1, sm, err)) break;
-          mbar_expect_tx(&sm->full[st], kBBytes);
-          tma_load_2d(b_smem0 + st * kBBytes, &xmap, ks * kTileK, m0, &sm->full[st]);
+      for (int u = blockIdx.x; u < wk.units && !aborted(sm); u += gridDim.x) {
+        const int ks0 = wk.split(u) * wk.kps;
+        const int m0 = wk.m0(u);
+        for (int ks = ks0; ks < ks0 + wk.kps; ++ks, ++it) {
+          const int xs = it % kXStages;
+          if (!wait_or_abort(&sm->xempty[xs], ((it / kXStages) & 1) ^ 1, sm, err)) break;
+          if (it == 0) NF4_STAMP(1);
+          mbar_expect_tx(&sm->xfull[xs], kBBytes);
+          tma_load_2d(b_smem0 + xs * kBBytes, &xmap, ks * kTileK, m0, &sm->xfull[xs]);
         }
       }
-      // drain: wait for the copies still in flight into the stages
-      const uint32_t issued = it;
-      for (uint32_t j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
-        mbar_wait_bounded(&sm->full[j % kStages], (j / kStages) & 1, err);
+      const uint32_t issued = it;  // drain the copies still in flight
+      for (uint32_t j = (issued > kXStages ? issued - kXStages : 0); j < issued; ++j)
+        mbar_wait_bounded(&sm->xfull[j % kXStages], (j / kXStages) & 1, err);
+    }
+  } else if (warp == kTmaWWarp) {
+    // ------------------------------------------------ TMA: packed codes and scale chunks
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&wmap)) : "memory");
+      if (kScaleTma) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&smap)) : "memory");
+      uint32_t it = 0;
+      for (int u = blockIdx.x; u < wk.units && !aborted(sm); u += gridDim.x) {
+        const int ks0 = wk.split(u) * wk.kps;
+        const int n0 = wk.n0(u);
+        for (int ks = ks0; ks < ks0 + wk.kps; ++ks, ++it) {
+          const int ws = it % kWStages;
+          if (!wait_or_abort(&sm->wempty[ws], ((it / kWStages) & 1) ^ 1, sm, err)) break;
+          mbar_expect_tx(&sm->wfull[ws], kWBytes + (kScaleTma ? kSBytes : 0));
+          tma_load_2d(w_smem0 + ws * kWBytes, &wmap, ks * (kTileK / 2), n0, &sm->wfull[ws]);
+          // the 16-byte scale chunk holding this stage's block: 16 codes or 4 fp32
+          if (kScaleTma)
+            tma_load_2d(s_smem0 + ws * kSBytes, &smap, kDQ ? (ks & ~15) : (ks & ~3), n0, &sm->wfull[ws]);
+        }
+      }
+      const uint32_t issued = it;  // drain the copies still in flight
+      for (uint32_t j = (issued > kWStages ? issued - kWStages : 0); j < issued; ++j)
+        mbar_wait_bounded(&sm->wfull[j % kWStages], (j / kWStages) & 1, err);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = instr_desc(kTileN, kTileM);
-      uint32_t it = 0, tcount = 0;
-      for (int tile = blockIdx.x; tile < ntiles && !aborted(sm); tile += gridDim.x, ++tcount) {
-        const int acc = tcount & 1;
-        if (!wait_or_abort(&sm->acc_empty[acc], ((tcount >> 1) & 1) ^ 1, sm, err)) break;
+      uint32_t it = 0, ucount = 0;
+      for (int u = blockIdx.x; u < wk.units && !aborted(sm); u += gridDim.x, ++ucount) {
+        const int acc = ucount & 1;
+        if (!wait_or_abort(&sm->acc_empty[acc], ((ucount >> 1) & 1) ^ 1, sm, err)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + acc * kAccCols;
         bool ok = true;
-        for (int ks = 0; ks < kstages; ++ks, ++it) {
-          const int st = it % kStages;
-          const uint32_t ph = (it / kStages) & 1;
-          if (!wait_or_abort(&sm->full[st], ph, sm, err)) {
+        for (int j = 0; j < wk.kps; ++j, ++it) {
+          const int as = it % kAStages, xs = it % kXStages;
+          if (!wait_or_abort(&sm->afull[as], (it / kAStages) & 1, sm, err) ||
+              !wait_or_abort(&sm->xfull[xs], (it / kXStages) & 1, sm, err)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = a_smem0 + st * kABytes, b_addr = b_smem0 + st * kBBytes;
+          if (it == 0) NF4_STAMP(2);
+          const uint32_t a_addr = a_smem0 + as * kABytes, b_addr = b_smem0 + xs * kBBytes;
 #pragma unroll
           for (int kk = 0; kk < kTileK / 16; ++kk)  // 16 bf16 = 32 bytes per MMA along k
             tc_mma(d_tmem, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32), idesc,
-                   (ks | kk) != 0);
-          tc_commit(&sm->empty[st]);  // stage free once these MMAs have read it
+                   (j | kk) != 0);
+          tc_commit(&sm->aempty[as]);  // slots free once these MMAs have read them
+          tc_commit(&sm->xempty[xs]);
         }
         if (!ok) break;
+        NF4_STAMP(3);
         tc_commit(&sm->acc_full[acc]);  // accumulator ready for the epilogue
       }
     }
   } else if (warp < kEpiWarps) {
-    // ------------------------------------------------ epilogue: TMEM -> bf16 -> Y
-    uint32_t tcount = 0;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tcount) {
-      const int acc = tcount & 1;
-      if (!wait_or_abort(&sm->acc_full[acc], (tcount >> 1) & 1, sm, err)) break;
+    // ------------------------------------------------ epilogue: TMEM -> Y (or fp32 partials)
+    uint32_t ucount = 0;
+    for (int u = blockIdx.x; u < wk.units; u += gridDim.x, ++ucount) {
+      const int acc = ucount & 1;
+      if (!wait_or_abort(&sm->acc_full[acc], (ucount >> 1) & 1, sm, err)) break;
       tc_fence_after();
-      const int64_t n = (int64_t)(tile / ntiles_m) * kTileN + warp * 32 + lane;
-      const int m0 = (tile % ntiles_m) * kTileM;
-#pragma unroll 1
-      for (int c = 0; c < kTileM / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + acc * kAccCols + c * 32, v);
+      if (threadIdx.x == 0) NF4_STAMP(4);
+      const int nl = warp * 32 + lane;  // weight row within the tile
+      const int64_t n = (int64_t)wk.n0(u) + nl;
+      const int m0 = wk.m0(u);
+      const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + acc * kAccCols;
+      uint16_t* st = out_stage + warp * (32 * 32);  // this warp's [32 m][32 n] bf16 tile
+      // Y rows m0 + c*32 + r, columns n0 + warp*32 .. +31: the warp's 32x32 block goes
+      // through shared memory so each lane stores 16 contiguous bytes of a Y row
+      auto store_block = [&](int c) {
+        __syncwarp();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int m = m0 + c * 32 + j;
-          if (m < m_total) y[(int64_t)m * rows + n] = __float2bfloat16_rn(__uint_as_float(v[j]));
+        for (int i = 0; i < 4; ++i) {
+          const int piece = lane + 32 * i;  // 128 pieces of 8 bf16
+          const int r = piece >> 2, q = piece & 3;
+          const int m = m0 + c * 32 + r;
+          const uint4 v = *reinterpret_cast<const uint4*>(st + r * 32 + q * 8);
+          if (m < m_total)
+            *reinterpret_cast<uint4*>(y + (int64_t)m * rows + (n - lane) + q * 8) = v;
+        }
+        __syncwarp();
+      };
+      if (wk.splits == 1) {
+#pragma unroll 1
+        for (int c = 0; c < kTileM / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(taddr + c * 32, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) st[j * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
+          store_block(c);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm->acc_empty[acc]);
+      } else {
+        // fp32 partial tile of this unit, laid out [m/4][n_local][4]: each 16-byte
+        // access of a warp covers 32 consecutive n (512 contiguous bytes)
+        float* mine = part + (size_t)u * (kTileN * kTileM);
+#pragma unroll 1
+        for (int c = 0; c < kTileM / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(taddr + c * 32, v);
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            __stcg(reinterpret_cast<float4*>(mine + ((size_t)((c * 32 + j) / 4) * kTileN + nl) * 4),
+                   make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
+                               __uint_as_float(v[j + 3])));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm->acc_empty[acc]);  // TMEM no longer needed
+        __threadfence();
+        epi_bar();
+        if (threadIdx.x == 0) sm->last = atomicAdd(&tile_count[wk.tile(u)], 1u) == (unsigned)(wk.splits - 1);
+        epi_bar();
+        if (threadIdx.x == 0) NF4_STAMP(5);
+        if (sm->last) {
+          __threadfence();
+          const float* tp = part + (size_t)wk.tile(u) * wk.splits * (kTileN * kTileM);
+#pragma unroll 1
+          for (int c = 0; c < kTileM / 32; ++c) {
+            float4 acc4[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              acc4[j] = __ldcg(reinterpret_cast<const float4*>(tp + ((size_t)(c * 8 + j) * kTileN + nl) * 4));
+            for (int sp = 1; sp < wk.splits; ++sp) {  // partials added in split order
+              const float* q = tp + (size_t)sp * (kTileN * kTileM);
+              float4 t[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                t[j] = __ldcg(reinterpret_cast<const float4*>(q + ((size_t)(c * 8 + j) * kTileN + nl) * 4));
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                acc4[j].x += t[j].x;
+                acc4[j].y += t[j].y;
+                acc4[j].z += t[j].z;
+                acc4[j].w += t[j].w;
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              st[(4 * j + 0) * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(acc4[j].x));
+              st[(4 * j + 1) * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(acc4[j].y));
+              st[(4 * j + 2) * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(acc4[j].z));
+              st[(4 * j + 3) * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(acc4[j].w));
+            }
+            store_block(c);
+          }
+          if (threadIdx.x == 0) tile_count[wk.tile(u)] = 0;  // ready for the next call
+          if (threadIdx.x == 0) NF4_STAMP(6);
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm->acc_empty[acc]);
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) NF4_STAMP(7);
   if (warp == kMmaWarp) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
@@ -302,41 +463,122 @@ EncodeTiled get_encoder() {
   return fn;
 }
 
+// Splits of K: enough work units to cover the SMs when there are few output
+// tiles; the split count divides the number of k stages and leaves each split
+// at least 8 stages.
+int gemm_splits(int64_t rows, int64_t cols, int64_t m, int num_sms) {
+  if (m <= 64) return 1;
+  const int64_t ntiles = (rows / kTileN) * ((m + kTileM - 1) / kTileM);
+  const int64_t kst = cols / kTileK;
+  int best = 1;
+  for (int sp = 2; sp <= 8; ++sp)
+    if (kst % sp == 0 && kst / sp >= 8 && ntiles * sp <= num_sms) best = sp;
+  return best;
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
 }  // namespace
 
-size_t gemm_workspace_bytes(int64_t, int64_t, int64_t) { return 0; }
+size_t gemm_workspace_bytes(int64_t rows, int64_t cols, int64_t m) {
+  const int sp = gemm_splits(rows, cols, m, sm_count());
+  if (sp == 1) return 0;
+  const int64_t ntiles = (rows / kTileN) * ((m + kTileM - 1) / kTileM);
+  const size_t counters = ((size_t)ntiles * 4 + 255) & ~(size_t)255;
+  return counters + (size_t)ntiles * sp * kTileN * kTileM * sizeof(float);
+}
 
-cudaError_t launch_gemm(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x, int64_t m,
-                        void* y, void*, unsigned* err, cudaStream_t stream, int num_sms) {
-  auto* yb = static_cast<__nv_bfloat16*>(y);
-  if (m <= 64) return launch_gemv(packed, s, rows, cols, x, (int)m, y, stream, num_sms);
-  if (rows > INT32_MAX || cols > INT32_MAX || m > INT32_MAX) return cudaErrorInvalidValue;
+namespace {
+
+// 2-D tiled tensor map (no swizzle unless asked); false if the driver refuses it
+bool make_map(CUtensorMap* map, CUtensorMapDataType type, size_t esize, const void* base, uint64_t inner,
+              uint64_t outer, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
   EncodeTiled encode = get_encoder();
-  if (encode == nullptr) return cudaErrorNotSupported;
-  CUtensorMap xmap;
-  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)m};
-  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)kTileK, (cuuint32_t)kTileM};
+  if (encode == nullptr) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  const cuuint64_t strides[1] = {(cuuint64_t)(inner * esize)};
+  const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
-  if (encode(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
-  const int ntiles = (int)((rows / kTileN) * ((m + kTileM - 1) / kTileM));
-  const int grid = ntiles < num_sms ? ntiles : num_sms;
-  const bool dq = s.absmax == nullptr;
-  cudaError_t e;
-  if (dq) {
-    e = cudaFuncSetAttribute(gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  return encode(map, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool kDQ, bool kScaleTma>
+cudaError_t launch_variant(const Scales& s, int rows, int cols, int m, int splits, const CUtensorMap& xmap,
+                           const CUtensorMap& wmap, const CUtensorMap& smap, __nv_bfloat16* y, float* part,
+                           unsigned* counters, unsigned* err, int grid, cudaStream_t stream) {
+  // the shared-memory opt-in is a per-device function attribute: set it once
+  // per device (outside any stream capture that later calls may be part of)
+  static std::atomic<uint64_t> attr_done{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!(attr_done.load() & (1ull << dev))) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<kDQ, kScaleTma>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    gemm_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(packed, s, (int)rows, (int)cols, (int)m, xmap, yb, err);
-  } else {
-    e = cudaFuncSetAttribute(gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    gemm_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(packed, s, (int)rows, (int)cols, (int)m, xmap, yb, err);
+    attr_done.fetch_or(1ull << dev);
   }
+  gemm_kernel<kDQ, kScaleTma><<<grid, kThreads, kSmemBytes, stream>>>(s, rows, cols, m, splits, xmap, wmap, smap, y,
+                                                                      part, counters, err);
   count_launches(1);
   return cudaGetLastError();
 }
 
+}  // namespace
+
+cudaError_t launch_gemm(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x, int64_t m,
+                        void* y, void* workspace, unsigned* err, cudaStream_t stream, int num_sms) {
+  auto* yb = static_cast<__nv_bfloat16*>(y);
+  if (m <= 64) return launch_gemv(packed, s, rows, cols, x, (int)m, y, stream, num_sms);
+  if (rows > INT32_MAX || cols > INT32_MAX || m > INT32_MAX) return cudaErrorInvalidValue;
+  const bool dq = s.absmax == nullptr;
+  const int64_t rb = cols / kBlock;  // level-1 blocks per weight row
+  CUtensorMap xmap, wmap, smap;
+  if (!make_map(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, cols, m, kTileK, kTileM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, packed, cols / 2, rows, kTileK / 2, kTileN,
+                CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorNotSupported;
+  // scale chunks through TMA when each row of scales is a whole number of 16-byte units
+  const void* sbase = dq ? (const void*)s.q : (const void*)s.absmax;
+  const size_t srow = dq ? (size_t)rb : (size_t)rb * 4;
+  bool scale_tma = srow % 16 == 0 && reinterpret_cast<uintptr_t>(sbase) % 16 == 0;
+  if (scale_tma)
+    scale_tma = dq ? make_map(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, sbase, rb, rows, 16, kTileN,
+                              CU_TENSOR_MAP_SWIZZLE_NONE)
+                   : make_map(&smap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, sbase, rb, rows, 4, kTileN,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!scale_tma) smap = wmap;  // unused by the kernel variant
+  const int splits = gemm_splits(rows, cols, m, num_sms);
+  const int64_t ntiles = (rows / kTileN) * ((m + kTileM - 1) / kTileM);
+  const int64_t units = ntiles * splits;
+  const int grid = (int)(units < num_sms ? units : num_sms);
+  unsigned* counters = nullptr;
+  float* part = nullptr;
+  if (splits > 1) {
+    const size_t cbytes = ((size_t)ntiles * 4 + 255) & ~(size_t)255;
+    counters = static_cast<unsigned*>(workspace);
+    part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + cbytes);
+    cudaError_t e = cudaMemsetAsync(counters, 0, (size_t)ntiles * 4, stream);
+    if (e != cudaSuccess) return e;
+  }
+  const int R = (int)rows, C = (int)cols, M = (int)m;
+  if (dq && scale_tma)
+    return launch_variant<true, true>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream);
+  if (dq)
+    return launch_variant<true, false>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream);
+  if (scale_tma)
+    return launch_variant<false, true>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream);
+  return launch_variant<false, false>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream);
+}
+
 }  // namespace nf4
+
+#ifdef NF4_TRACE
+extern "C" __attribute__((visibility("default"))) int nf4_trace_read(unsigned long long* host) {
+  return (int)cudaMemcpyFromSymbol(host, nf4::g_trace, sizeof(nf4::g_trace));
+}
+#endif

@@ -33,20 +33,27 @@ __constant__ float c_threshold[15] = NF4_THRESHOLD_INIT;
 constexpr float kNearThreshold = 0x1p-19f;
 constexpr float kTinyScale = 0x1p-120f;  // below this 1/a may overflow: divide exactly
 
-// `entry` is this lane's bucket word; every lane of the warp must call this
-__device__ __forceinline__ int code_of(uint32_t entry, float w, float a, float r, bool exact) {
-  const float q = exact ? __fdiv_rn(w, a) : __fmul_rn(w, r);
-  const float v = __fmaf_rn(q, NF4_Q32_SCALE, 3.0f);
-  const int bk = (__float_as_int(v) >> 18) & 31;  // NaN/Inf inputs still land in 0..31
-  const uint32_t e = __shfl_sync(0xffffffffu, entry, bk);
-  const int base = (int)(e & 15u);
-  const float thr = __uint_as_float(e);
-  int code = base + (q > thr ? 1 : 0);
-  if (fabsf(q - thr) <= kNearThreshold) {
-    const float x = exact ? q : __fdiv_rn(w, a);
-    code = base + (x > c_threshold[base < 15 ? base : 14] ? 1 : 0);
-  }
+// Exact decision for the rare elements near a threshold (and for blocks whose
+// scale is too small for the reciprocal): the IEEE quotient counted against
+// the exact thresholds.
+__device__ __noinline__ int code_exact(float w, float a) {
+  const float x = __fdiv_rn(w, a);
+  int code = 0;
+#pragma unroll
+  for (int i = 0; i < 15; ++i) code += (x > c_threshold[i]) ? 1 : 0;
   return code;
+}
+
+// `entry` is this lane's bucket word; every lane of the warp must call this
+// (the lookup is a shuffle).  q estimates w / a within 3 * 2^-24.  `near`
+// records whether the estimate was too close to the entry to decide.
+__device__ __forceinline__ int code_fast(uint32_t entry, float q, bool& near) {
+  const float v = __fmaf_rn(q, NF4_Q32_SCALE, 3.0f);
+  // lane index wraps modulo 32, so the exponent bits above the bucket need no mask
+  const uint32_t e = __shfl_sync(0xffffffffu, entry, __float_as_int(v) >> 18);
+  const float thr = __uint_as_float(e);
+  near |= fabsf(q - thr) <= kNearThreshold;
+  return (int)(e & 15u) + (q > thr ? 1 : 0);
 }
 
 template <bool kBF16>
@@ -112,12 +119,16 @@ __global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ 
 
     // Step 3: nearest code of RN(w / a); an all-zero block takes the zero code (7)
     const bool zero = !(a > 0.0f);
-    const bool exact = a < kTinyScale;
-    const float r = exact ? 0.0f : __frcp_rn(a);
-    const float as = zero ? 1.0f : a;  // keeps the (discarded) zero-block arithmetic finite
+    const bool exact = !zero && a < kTinyScale;      // 1/a could overflow: divide exactly
+    const float r = __frcp_rn(zero ? 1.0f : a);
     int c[16];
+    bool near = exact;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) c[i] = code_of(entry, w[i], as, r, exact && !zero);
+    for (int i = 0; i < 16; ++i) c[i] = code_fast(entry, __fmul_rn(w[i], r), near);
+    if (near) {  // rare: redo this lane's 16 elements with exact quotients
+#pragma unroll
+      for (int i = 0; i < 16; ++i) c[i] = code_exact(w[i], a);
+    }
     // Step 4: element 2j -> high nibble of byte j
     uint32_t lo = 0, hi = 0;
 #pragma unroll

@@ -273,3 +273,44 @@ def test_gemm_config4_sampled(m):
     got = yh[bs, ns]
     assert np.all(np.abs(got - ref) <= REL_TOL * np.maximum(np.abs(ref), FLOOR * rms))
     check_matmul(y[:1], full_row, f"gemm m{m} row 0")
+
+
+@pytest.mark.parametrize("m", [65, 200, 256, 300])
+def test_gemm_split_k(m):
+    """few output tiles: K is split across CTAs and the fp32 partials are
+    added in split order"""
+    rows, cols = 256, 2048
+    qw, p_ref, a_ref = quantized_pair(rows, cols, 61 + m, True)
+    x = synth.activations((m, cols), 62 + m)
+    y = nf4.gemm(qw, dev_bf16(x))
+    check_matmul(y, oracle.matmul(p_ref, a_ref, rows, cols, x), f"gemm split m{m}")
+
+
+def test_gemm_deterministic_and_bench_shape():
+    """4096 x 4096 weight, M = 256 (split-K path): bit-identical across calls,
+    sampled outputs within tolerance"""
+    rows, cols, m = 4096, 4096, 256
+    qw, p_ref, a_ref = quantized_pair(rows, cols, 1002, True)
+    x = synth.activations((m, cols), 1277)
+    y1 = nf4.gemm(qw, dev_bf16(x))
+    y2 = nf4.gemm(qw, dev_bf16(x))
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    r = synth.rng(9)
+    bs, ns = r.integers(0, m, 4096), r.integers(0, rows, 4096)
+    ref = oracle.matmul_sampled(p_ref, a_ref, rows, cols, x, bs, ns)
+    full_row = oracle.matmul(p_ref, a_ref, rows, cols, x[:1])
+    rms = np.sqrt(np.mean(full_row ** 2))
+    got = y1.float().cpu().numpy().astype(np.float64)[bs, ns]
+    assert np.all(np.abs(got - ref) <= REL_TOL * np.maximum(np.abs(ref), FLOOR * rms))
+
+
+@pytest.mark.parametrize("cols", [320, 1024, 4096])
+@pytest.mark.parametrize("use_dq", [False, True])
+def test_gemm_scale_paths(cols, use_dq):
+    """plain fp32 and double-quantized scales, with scale rows that are (1024,
+    4096) and are not (320) whole 16-byte units"""
+    rows, m = 128, 160
+    qw, p_ref, a_ref = quantized_pair(rows, cols, 71 + cols, use_dq)
+    x = synth.activations((m, cols), 72 + cols)
+    y = nf4.gemm(qw, dev_bf16(x))
+    check_matmul(y, oracle.matmul(p_ref, a_ref, rows, cols, x), f"gemm cols{cols} dq{use_dq}")
