@@ -94,39 +94,66 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restri
 
 // bf16 output: one lane per 64-element block.  The lane builds the block's 16
 // bf16 values bf16_rn(RN(code[i] * a)) as byte-permute pools (the same decode
-// the matmuls use) and expands its 32 code bytes with byte permutes: eight
-// 16-byte stores of bf16 pairs, no shared-memory lookups.
+// the matmuls use) and expands its 32 code bytes with byte permutes.  The
+// warp's 32 consecutive blocks (4 KB of bf16) go through a swizzled shared
+// tile so the global stores are 512 contiguous bytes per instruction.
 template <bool kDQ>
 __global__ void __launch_bounds__(256) dequantize_bf16_kernel(const uint8_t* __restrict__ packed, Scales s,
                                                               int64_t n, __nv_bfloat16* __restrict__ out) {
   __shared__ float unit_lut[kDQ ? 256 : 1];
+  __shared__ __align__(16) uint4 stage[8][32 * 8];  // per warp: 32 blocks x 8 chunks of 16 bytes
   if (kDQ) unit_lut[threadIdx.x & 255] = dq_unit(threadIdx.x & 255, s.dq_code);
   __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint4* st = stage[warp];
   const int64_t nfull = n / kBlock;
   const int64_t nblocks = (n + kBlock - 1) / kBlock;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblocks; b += stride) {
-    const float a = block_scale<kDQ>(s, unit_lut, b);
-    const Table T = make_table(a);
-    if (b < nfull) {
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t b0 = ((int64_t)blockIdx.x * (blockDim.x >> 5) + warp) * 32; b0 < nblocks; b0 += nwarps * 32) {
+    const int64_t b = b0 + lane;
+    const bool full_warp = b0 + 32 <= nfull;  // all 32 blocks complete: the coalesced path
+    if (full_warp) {
       const uint4* src = reinterpret_cast<const uint4*>(packed + b * (kBlock / 2));
       const uint4 w0 = __ldcs(src), w1 = __ldcs(src + 1);
+      const Table T = make_table(block_scale<kDQ>(s, unit_lut, b));
       const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-      uint4* o = reinterpret_cast<uint4*>(out + b * kBlock);
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         uint32_t d[4];
         decode_word(words[c], T, d);
-        __stcs(o + c, make_uint4(d[0], d[1], d[2], d[3]));
+        st[lane * 8 + (c ^ (lane & 7))] = make_uint4(d[0], d[1], d[2], d[3]);  // XOR swizzle: no bank conflicts
       }
-    } else {
-      // short last block: element by element from the same table
-      for (int64_t e = b * kBlock; e < n; ++e) {
-        const uint8_t byte = packed[e / 2];
-        const uint32_t nib = (e & 1) ? (byte & 15u) : (byte >> 4);
-        uint32_t d[4];
-        decode_word(nib * 0x11111111u, T, d);  // every lane of the word holds this code
-        reinterpret_cast<uint16_t*>(out)[e] = (uint16_t)(d[0] & 0xffffu);
+      __syncwarp();
+      uint4* o = reinterpret_cast<uint4*>(out + b0 * kBlock);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int piece = i * 32 + lane;  // 16-byte piece of the warp's 4 KB
+        const int blk = piece >> 3, c = piece & 7;
+        __stcs(o + piece, st[blk * 8 + (c ^ (blk & 7))]);
+      }
+      __syncwarp();
+    } else if (b < nblocks) {
+      const Table T = make_table(block_scale<kDQ>(s, unit_lut, b));
+      if (b < nfull) {
+        const uint4* src = reinterpret_cast<const uint4*>(packed + b * (kBlock / 2));
+        const uint4 w0 = __ldcs(src), w1 = __ldcs(src + 1);
+        const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        uint4* o = reinterpret_cast<uint4*>(out + b * kBlock);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t d[4];
+          decode_word(words[c], T, d);
+          __stcs(o + c, make_uint4(d[0], d[1], d[2], d[3]));
+        }
+      } else {
+        // short last block: element by element from the same table
+        for (int64_t e = b * kBlock; e < n; ++e) {
+          const uint8_t byte = packed[e / 2];
+          const uint32_t nib = (e & 1) ? (byte & 15u) : (byte >> 4);
+          uint32_t d[4];
+          decode_word(nib * 0x11111111u, T, d);  // every nibble of the word holds this code
+          reinterpret_cast<uint16_t*>(out)[e] = (uint16_t)(d[0] & 0xffffu);
+        }
       }
     }
   }
@@ -143,7 +170,7 @@ cudaError_t launch_dequantize(const uint8_t* packed, const Scales& s, int64_t n,
   if (grid < 1) grid = 1;
   const bool dq = s.absmax == nullptr;
   if (out_bf16) {
-    int64_t g2 = (nblocks + 255) / 256;
+    int64_t g2 = (nblocks + 255) / 256;  // 8 warps x 32 blocks per CTA per pass
     if (g2 > cap) g2 = cap;
     if (g2 < 1) g2 = 1;
     auto* ob = static_cast<__nv_bfloat16*>(out);

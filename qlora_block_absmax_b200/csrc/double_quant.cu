@@ -127,6 +127,13 @@ __device__ float finish_mean(const long long (&limb_in)[kLimbs], int64_t nb) {
   return __double2float_rn(__ddiv_rn(s, (double)nb));
 }
 
+#ifdef NF4_TRACE  // diagnostics build only
+__device__ unsigned long long g_dq_trace[1024 * 8];
+#define DQ_STAMP(slot) (g_dq_trace[blockIdx.x * 8 + (slot)] = global_ns())
+#else
+#define DQ_STAMP(slot) ((void)0)
+#endif
+
 // One cooperative launch (every CTA resident): exact sum -> grid barrier ->
 // codes.  The barrier spins on a counter with a wall-clock bound; if it runs
 // out the error word is set and the codes are skipped.
@@ -135,6 +142,7 @@ __global__ void __launch_bounds__(256) dq_fused_kernel(const float* __restrict__
                                                        float* __restrict__ mean_out, SumWorkspace* __restrict__ ws,
                                                        unsigned* __restrict__ err) {
   // ---- phase 1: this thread's values into the integer limbs
+  if (threadIdx.x == 0) DQ_STAMP(0);
   long long acc[kLimbs];
 #pragma unroll
   for (int L = 0; L < kLimbs; ++L) acc[L] = 0;
@@ -171,10 +179,13 @@ __global__ void __launch_bounds__(256) dq_fused_kernel(const float* __restrict__
 
   // ---- grid barrier (bounded)
   if (threadIdx.x == 0) {
+    DQ_STAMP(1);
     atomicAdd(&ws->done, 1u);
     int ok = 1;
     const unsigned long long t0 = global_ns();
-    while (atomicAdd(&ws->done, 0u) < gridDim.x) {
+    // poll with plain loads (an atomic per poll would contend with the arrivals)
+    while (*reinterpret_cast<volatile unsigned*>(&ws->done) < gridDim.x) {
+      __nanosleep(64);
       if (global_ns() - t0 > kWaitLimitNs) {
         atomicOr(err, kErrTimeout);
         ok = 0;
@@ -182,6 +193,7 @@ __global__ void __launch_bounds__(256) dq_fused_kernel(const float* __restrict__
       }
     }
     __threadfence();
+    DQ_STAMP(2);
     if (ok) {
       long long l[kLimbs];
 #pragma unroll
@@ -190,6 +202,7 @@ __global__ void __launch_bounds__(256) dq_fused_kernel(const float* __restrict__
       if (blockIdx.x == 0) *mean_out = s_mu;
     }
     s_ok = ok;
+    DQ_STAMP(3);
   }
   __syncthreads();
   if (!s_ok) return;
@@ -276,3 +289,9 @@ cudaError_t launch_double_quant(const float* absmax, int64_t nb, int dq_code, ui
 }
 
 }  // namespace nf4
+
+#ifdef NF4_TRACE
+extern "C" __attribute__((visibility("default"))) int nf4_dq_trace_read(unsigned long long* host) {
+  return (int)cudaMemcpyFromSymbol(host, nf4::g_dq_trace, sizeof(nf4::g_dq_trace));
+}
+#endif

@@ -45,39 +45,22 @@ __device__ __noinline__ int code_exact(float w, float a) {
 }
 
 // `entry` is this lane's bucket word; every lane of the warp must call this
-// (the lookup is a shuffle).  q estimates w / a within 3 * 2^-24.  `near`
-// records whether the estimate was too close to the entry to decide.
-__device__ __forceinline__ int code_fast(uint32_t entry, float q, bool& near) {
+// (the lookup is a shuffle).  q estimates w / a within 3 * 2^-24.  `gap`
+// tracks the smallest distance between an estimate and its entry.
+__device__ __forceinline__ uint32_t code_fast(uint32_t entry, float q, float& gap) {
   const float v = __fmaf_rn(q, NF4_Q32_SCALE, 3.0f);
   // lane index wraps modulo 32, so the exponent bits above the bucket need no mask
   const uint32_t e = __shfl_sync(0xffffffffu, entry, __float_as_int(v) >> 18);
   const float thr = __uint_as_float(e);
-  near |= fabsf(q - thr) <= kNearThreshold;
-  return (int)(e & 15u) + (q > thr ? 1 : 0);
+  gap = fminf(gap, fabsf(q - thr));
+  return (e & 15u) + (q > thr ? 1u : 0u);
 }
 
-template <bool kBF16>
-__device__ __forceinline__ void load16(const void* src, int64_t first, float (&w)[16]) {
-  if (kBF16) {
-    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(src) + first);
-    uint4 v0 = __ldcs(p), v1 = __ldcs(p + 1);
-    uint32_t u[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      w[2 * i] = bf16_lo_to_f32(u[i]);
-      w[2 * i + 1] = bf16_hi_to_f32(u[i]);
-    }
-  } else {
-    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(src) + first);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float4 v = __ldcs(p + i);
-      w[4 * i] = v.x;
-      w[4 * i + 1] = v.y;
-      w[4 * i + 2] = v.z;
-      w[4 * i + 3] = v.w;
-    }
-  }
+// two codes -> one byte (first in the high nibble); four bytes -> one word
+__device__ __forceinline__ uint32_t pack8(const uint32_t (&c)[16], int o) {
+  const uint32_t b0 = c[o] * 16u + c[o + 1], b1 = c[o + 2] * 16u + c[o + 3];
+  const uint32_t b2 = c[o + 4] * 16u + c[o + 5], b3 = c[o + 6] * 16u + c[o + 7];
+  return prmt(prmt(b0, b1, 0x0040), prmt(b2, b3, 0x0040), 0x5410);
 }
 
 template <bool kBF16>
@@ -99,13 +82,45 @@ __global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ 
   const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
   const int64_t warp_id = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
 
-  for (int64_t wb = warp_id * 8; wb < nblocks; wb += warps_total * 8) {  // uniform per warp
+  // raw 16-element slices, one iteration ahead: the next slice's loads are in
+  // flight while this one is coded
+  using Raw = uint4[kBF16 ? 2 : 4];
+  auto fetch = [&](int64_t wb, Raw& raw) {
+    const int64_t b = wb + (lane >> 2);
+    if (b < nfull) {
+      const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(src) +
+                                                      (b * kBlock + sub * 16) * (kBF16 ? 2 : 4));
+#pragma unroll
+      for (int i = 0; i < (kBF16 ? 2 : 4); ++i) raw[i] = __ldcs(p + i);
+    }
+  };
+  Raw cur, nxt;
+  int64_t wb = warp_id * 8;
+  if (wb < nblocks) fetch(wb, cur);
+  for (; wb < nblocks; wb += warps_total * 8) {  // uniform per warp
+    if (wb + warps_total * 8 < nblocks) fetch(wb + warps_total * 8, nxt);
     const int64_t b = wb + (lane >> 2);
     const bool live = b < nblocks;
     const int64_t first = b * kBlock + sub * 16;
     float w[16];
     if (live && b < nfull) {
-      load16<kBF16>(src, first, w);
+      if (kBF16) {
+        const uint32_t u[8] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w, cur[1].x, cur[1].y, cur[1].z, cur[1].w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          w[2 * i] = bf16_lo_to_f32(u[i]);
+          w[2 * i + 1] = bf16_hi_to_f32(u[i]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 v = cur[(kBF16 ? 0 : i)];
+          w[4 * i] = __uint_as_float(v.x);
+          w[4 * i + 1] = __uint_as_float(v.y);
+          w[4 * i + 2] = __uint_as_float(v.z);
+          w[4 * i + 3] = __uint_as_float(v.w);
+        }
+      }
     } else {  // short last block (or no block): missing elements read as 0
 #pragma unroll
       for (int i = 0; i < 16; ++i) w[i] = (live && first + i < n) ? load1<kBF16>(src, first + i) : 0.0f;
@@ -121,22 +136,19 @@ __global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ 
     const bool zero = !(a > 0.0f);
     const bool exact = !zero && a < kTinyScale;      // 1/a could overflow: divide exactly
     const float r = __frcp_rn(zero ? 1.0f : a);
-    int c[16];
-    bool near = exact;
+    uint32_t c[16];
+    float gap = 1.0f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) c[i] = code_fast(entry, __fmul_rn(w[i], r), near);
-    if (near) {  // rare: redo this lane's 16 elements with exact quotients
+    for (int i = 0; i < 16; ++i) c[i] = code_fast(entry, __fmul_rn(w[i], r), gap);
+    if (exact || gap <= kNearThreshold) {  // rare: redo this lane's 16 elements with exact quotients
 #pragma unroll
-      for (int i = 0; i < 16; ++i) c[i] = code_exact(w[i], a);
+      for (int i = 0; i < 16; ++i) c[i] = (uint32_t)code_exact(w[i], a);
     }
     // Step 4: element 2j -> high nibble of byte j
-    uint32_t lo = 0, hi = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      lo |= (uint32_t)((c[2 * j] << 4) | c[2 * j + 1]) << (8 * j);
-      hi |= (uint32_t)((c[8 + 2 * j] << 4) | c[8 + 2 * j + 1]) << (8 * j);
-    }
+    uint32_t lo = pack8(c, 0), hi = pack8(c, 8);
     if (zero) lo = hi = 0x77777777u;
+#pragma unroll
+    for (int i = 0; i < (kBF16 ? 2 : 4); ++i) cur[i] = nxt[i];
     if (!live) continue;
     if (b < nfull) {
       *reinterpret_cast<uint2*>(packed + first / 2) = make_uint2(lo, hi);
@@ -165,7 +177,12 @@ cudaError_t launch_quantize(const void* src, bool bf16, int64_t n, uint8_t* pack
   const int64_t nblocks = (n + kBlock - 1) / kBlock;
   const int per_cta = 256 / 4;
   int64_t grid = (nblocks + per_cta - 1) / per_cta;
-  const int64_t cap = (int64_t)num_sms * 8;
+  int occ = 0;  // one wave: as many CTAs as fit on the SMs at once
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, bf16 ? (const void*)quantize_kernel<true>
+                                                                : (const void*)quantize_kernel<false>,
+                                                    256, 0) != cudaSuccess || occ < 1)
+    occ = 1;
+  const int64_t cap = (int64_t)num_sms * occ;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
   if (bf16)
