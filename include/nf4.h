@@ -115,6 +115,26 @@ NF4_API nf4_status nf4_double_quant(const float *absmax, int64_t nb, int32_t dq_
                             size_t workspace_bytes, nf4_stream_t stream);
 NF4_API size_t nf4_double_quant_workspace_bytes(int64_t nb);
 
+/* nf4_double_quant without a caller-provided workspace, for callers that
+ * cannot allocate device memory: code that runs under a fixed memory budget
+ * set at start-up, or inside a host framework that owns the device allocator
+ * and hands out no scratch.  (The pages have no counterpart to this call; it
+ * only changes where the scratch lives.)
+ *   Same arguments and results as nf4_double_quant, minus the workspace.  The
+ *   scratch is a 256-byte static array inside the library: every GPU that
+ *   loads the library holds it until the process exits.  The function itself
+ *   allocates nothing (no cudaMalloc, no cudaFree).
+ *   The first call on a device looks up the array's device address with that
+ *   device current; make that first call before any stream capture.
+ *   Every call clears the array on `stream` before using it, and all calls
+ *   share it: calls that can run on the GPU at the same time (different
+ *   streams, other host threads) race and must be ordered by the caller.
+ *   Limit: nb <= NF4_DQ_NOALLOC_MAX_NB (the exact-sum digits in the array
+ *   stay exact up to this count); larger nb returns NF4_ERR_INVALID_ARG. */
+#define NF4_DQ_NOALLOC_MAX_NB 2147483647LL
+NF4_API nf4_status nf4_double_quant_noalloc(const float *absmax, int64_t nb, int32_t dq_blocksize, int32_t dq_code,
+                                            uint8_t *q_out, float *scale_out, float *mean_out, nf4_stream_t stream);
+
 /* Dequantization, [bnb-tools] Step 5 ("Dequantization": expand back to a higher
  * precision with the scale and the code book).  With double quantization the
  * scale is first reconstructed: a^ = fp32(fp32(fp32(dec(q)/Q) * m) + mu).

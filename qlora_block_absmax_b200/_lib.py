@@ -34,6 +34,7 @@ SIGNATURES = {
     "nf4_quantize": (ctypes.c_int, [P, I32, I64, I32, P, P, P]),
     "nf4_double_quant": (ctypes.c_int, [P, I64, I32, I32, P, P, P, P, SZ, P]),
     "nf4_double_quant_workspace_bytes": (SZ, [I64]),
+    "nf4_double_quant_noalloc": (ctypes.c_int, [P, I64, I32, I32, P, P, P, P]),
     "nf4_dequantize": (ctypes.c_int, [ctypes.POINTER(NF4Weight), P, I32, P]),
     "nf4_gemv": (ctypes.c_int, [ctypes.POINTER(NF4Weight), P, I32, P, P]),
     "nf4_gemm": (ctypes.c_int, [ctypes.POINTER(NF4Weight), P, I64, P, P, SZ, P]),

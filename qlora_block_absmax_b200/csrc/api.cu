@@ -152,6 +152,61 @@ nf4_status nf4_double_quant(const float* absmax, int64_t nb, int32_t dq_blocksiz
                                             d.error_word, reinterpret_cast<cudaStream_t>(stream), d.num_sms));
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Double quantization with library-owned scratch (no caller workspace).
+// The scratch is a file-scope device array; host code only ever uses the
+// device address looked up below, never the symbol itself (in host code the
+// symbol's name is a host-side stand-in, not a device address).
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 256;  // one exact-sum record (limbs + barrier count)
+static_assert(kNoAllocScratchBytes >= nf4::kDoubleQuantWorkspace, "scratch too small");
+__device__ __align__(256) unsigned char g_dq_scratch[kNoAllocScratchBytes];
+
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kMaxDevices];  // device address of g_dq_scratch, per device
+
+// Device address of the scratch on the current device, looked up once per
+// device (with that device current) and cached.
+nf4_status scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NF4_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_dq_scratch) != cudaSuccess || p == nullptr) return NF4_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return NF4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+nf4_status nf4_double_quant_noalloc(const float* absmax, int64_t nb, int32_t dq_blocksize, int32_t dq_code,
+                                    uint8_t* q_out, float* scale_out, float* mean_out, nf4_stream_t stream) {
+  if (nb < 0 || nb > NF4_DQ_NOALLOC_MAX_NB) return NF4_ERR_INVALID_ARG;
+  if (dq_code != NF4_DQ_E4M3 && dq_code != NF4_DQ_INT8) return NF4_ERR_INVALID_ARG;
+  if (dq_blocksize != nf4::kDqBlock) return NF4_ERR_UNSUPPORTED;
+  if (nb == 0) return NF4_OK;
+  if (absmax == nullptr || q_out == nullptr || scale_out == nullptr || mean_out == nullptr)
+    return NF4_ERR_INVALID_ARG;
+  if (!aligned(absmax, 16) || !aligned(q_out, 16) || !aligned(scale_out, 4) || !aligned(mean_out, 4))
+    return NF4_ERR_MISALIGNED;
+  DeviceInfo d;
+  nf4_status st = device_info(&d);
+  if (st != NF4_OK) return st;
+  void* scratch = nullptr;
+  if ((st = scratch_address(&scratch)) != NF4_OK) return st;
+  // the launcher clears the scratch on `stream` before the kernel reads it
+  return from_cuda(nf4::launch_double_quant(absmax, nb, dq_code, q_out, scale_out, mean_out, scratch,
+                                            d.error_word, reinterpret_cast<cudaStream_t>(stream), d.num_sms));
+}
+
 nf4_status nf4_dequantize(const nf4_weight* w, void* out, int32_t out_dtype, nf4_stream_t stream) {
   nf4::Scales s;
   nf4_status st = check_weight(w, &s);
