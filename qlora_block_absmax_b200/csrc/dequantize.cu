@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(256) dequantize_bf16_kernel(const uint8_t* __r
   if (kDQ) unit_lut[threadIdx.x & 255] = dq_unit(threadIdx.x & 255, s.dq_code);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const DecodeMul dm = decode_mul();
   uint4* st = stage[warp];
   const int64_t nfull = n / kBlock;
   const int64_t nblocks = (n + kBlock - 1) / kBlock;
@@ -120,7 +121,7 @@ __global__ void __launch_bounds__(256) dequantize_bf16_kernel(const uint8_t* __r
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         uint32_t d[4];
-        decode_word(words[c], T, d);
+        decode_word(words[c], T, d, dm);
         st[lane * 8 + (c ^ (lane & 7))] = make_uint4(d[0], d[1], d[2], d[3]);  // XOR swizzle: no bank conflicts
       }
       __syncwarp();
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(256) dequantize_bf16_kernel(const uint8_t* __r
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint32_t d[4];
-          decode_word(words[c], T, d);
+          decode_word(words[c], T, d, dm);
           __stcs(o + c, make_uint4(d[0], d[1], d[2], d[3]));
         }
       } else {

@@ -111,17 +111,20 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// 32 lanes x 32 consecutive fp32 columns (one register per column) of this warp's subpartition
+// 32 lanes x 32 consecutive fp32 columns (one register per column) of this warp's subpartition.
+// The load and its wait are one asm statement: the registers are defined only once the wait has
+// returned, so no use of them can be scheduled in between.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
-      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+      "tcgen05.wait::ld.sync.aligned;"
       : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
         "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
         "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
         "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+      : "r"(taddr)
+      : "memory");
 }
 
 __device__ __forceinline__ bool aborted(Smem* sm) { return *(volatile int*)&sm->abort != 0; }
@@ -221,6 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int p = ((warp - kProdWarp0) & 3) * 32 + lane;  // weight row within the tile
     const float mu = kDQ ? *s.mean : 0.0f;
     const int64_t rb = cols / kBlock;
+    const DecodeMul dm = decode_mul();
     uint32_t it = 0;
     for (int u = blockIdx.x; u < wk.units; u += gridDim.x) {
       const int64_t row = (int64_t)wk.n0(u) + p;
@@ -236,6 +240,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t b = row * rb + ks;  // level-1 block of this row and stage
         const uint32_t qcode = kDQ && kScaleTma ? sc[ks & 15] : 0u;
         const float plain = !kDQ && kScaleTma ? reinterpret_cast<const float*>(sc)[ks & 3] : 0.0f;
+        // the slot is refilled by TMA (async proxy) after these generic-proxy reads: order them first
+        fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm->wempty[ws]);  // the code slot may be refilled
         float a;
@@ -250,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint32_t d[4];
-          decode_word(words[c], T, d);
+          decode_word(words[c], T, d, dm);
           *reinterpret_cast<uint4*>(dst + ((c ^ (p & 7)) << 4)) = make_uint4(d[0], d[1], d[2], d[3]);
         }
         fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core

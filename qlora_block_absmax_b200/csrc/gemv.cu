@@ -102,6 +102,7 @@ __global__ void __launch_bounds__(kWarps * 32, NT >= 4 ? 1 : 2)
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) xrow[nt] = (8 * nt + g < batch) ? x + (int64_t)(8 * nt + g) * cols : nullptr;
 
+  const DecodeMul dm = decode_mul();
   StepData cur, nxt;
   int64_t st = warp;
   if (st < nsteps) load_step<kDQ>(cur, packed, s, row0, cols, st * 4 + t, st * 4 + t < nblk);
@@ -123,8 +124,8 @@ __global__ void __launch_bounds__(kWarps * 32, NT >= 4 ? 1 : 2)
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       uint32_t d0[4], d1[4];
-      decode_word(w0[j], T0, d0);
-      decode_word(w1[j], T1, d1);
+      decode_word(w0[j], T0, d0, dm);
+      decode_word(w1[j], T1, d1, dm);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         uint4 xv = make_uint4(0, 0, 0, 0);

@@ -35,19 +35,32 @@ __device__ __forceinline__ Table make_table(float a) {
   return T;
 }
 
+// Multipliers the decode reads at run time (65536 and 255).  Because the
+// compiler cannot see their values, `q * 65536 >> 32` and `m * 255` stay
+// integer multiplies, which run on the FMA pipe; the shift and the logic op
+// they replace would compete with the byte permutes for the ALU pipe.
+namespace {
+__constant__ uint32_t c_decode_mul[2] = {65536u, 255u};
+}
+struct DecodeMul {
+  uint32_t hi16, ff;
+};
+__device__ __forceinline__ DecodeMul decode_mul() { return DecodeMul{c_decode_mul[0], c_decode_mul[1]}; }
+
 // Decode 8 codes (one packed word) into 4 bf16x2 registers:
 // out[0] = (e0, e1), out[1] = (e2, e3), out[2] = (e4, e5), out[3] = (e6, e7),
 // element e_j being the j-th code in memory order (high nibble first).
-__device__ __forceinline__ void decode_word(uint32_t q, const Table& T, uint32_t (&out)[4]) {
+__device__ __forceinline__ void decode_word(uint32_t q, const Table& T, uint32_t (&out)[4], const DecodeMul& k) {
   const uint32_t qx = q ^ 0x88888888u;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const uint32_t s = h ? (q >> 16) : q;    // 4 selector nibbles
-    const uint32_t sx = h ? (qx >> 16) : qx; // same, pool-B view (bit 3 flipped)
+    const uint32_t s = h ? __umulhi(q, k.hi16) : q;    // 4 selector nibbles
+    const uint32_t sx = h ? __umulhi(qx, k.hi16) : qx; // same, pool-B view (bit 3 flipped)
     const uint32_t la = prmt(T.la0, T.la1, s), lb = prmt(T.lb0, T.lb1, sx);
     const uint32_t ha = prmt(T.ha0, T.ha1, s), hb = prmt(T.hb0, T.hb1, sx);
-    const uint32_t m1 = prmt(0x7f7f7f7fu, 0x7f7f7f7fu, sx);  // 0x7f where code >= 8, else 0
-    const uint32_t M = m1 | (m1 + m1);                          // 0xff where code >= 8
+    // 0x01 where code >= 8 (plain selector), 0x00 where code < 8 (sign mode of a byte whose top bit is 0)
+    const uint32_t m1 = prmt(0x01010101u, 0x01010101u, sx);
+    const uint32_t M = m1 * k.ff;                               // 0xff where code >= 8
     const uint32_t L = (la & ~M) | (lb & M);
     const uint32_t H = (ha & ~M) | (hb & M);
     out[2 * h] = prmt(L, H, 0x4051);      // selector nibble k -> element: 1,0,3,2
@@ -55,5 +68,9 @@ __device__ __forceinline__ void decode_word(uint32_t q, const Table& T, uint32_t
   }
 }
 
+// Same with compile-time constants (the compiler picks shifts and logic ops).
+__device__ __forceinline__ void decode_word(uint32_t q, const Table& T, uint32_t (&out)[4]) {
+  decode_word(q, T, out, DecodeMul{65536u, 255u});
+}
 
 }  // namespace nf4

@@ -227,13 +227,47 @@ def test_gemv_config3_shapes(shape, batch):
 
 
 def test_gemv_one_hot_pins_bit_exact():
-    rows, cols = 64, 256
+    """one-hot activations read single weights back: the decode GEMV (batch <= 8) and the skinny
+    tensor-core path (9 <= m <= 64) both return the dequantized bf16 weight bf16_rn(code * a^) bit for bit"""
+    rows, cols = 128, 256
     qw, p_ref, a_ref = quantized_pair(rows, cols, 3, True)
     wc = oracle.dequantize(p_ref, a_ref, rows * cols, 64, "bf16").reshape(rows, cols)
-    ks = [0, 1, 63, 64, 130, 255, 7, 200]
+    ks = [0, 1, 63, 64, 130, 255, 7, 200, 31, 32, 127, 128, 191, 192, 254, 100]
     x = synth.f32_to_bf16_bits(np.eye(cols, dtype=np.float32)[ks])
-    y = nf4.gemv(qw, dev_bf16(x))
-    assert np.array_equal(host_bf16_bits(y), wc[:, ks].T)
+    y16 = nf4.gemm(qw, dev_bf16(x))
+    assert np.array_equal(host_bf16_bits(y16), wc[:, ks].T)
+    y8 = nf4.gemv(qw, dev_bf16(x[:8]))
+    assert np.array_equal(host_bf16_bits(y8), wc[:, ks[:8]].T)
+
+
+# GEMV shapes around the grid's edges: a single 16-row tile; tiles fewer than the SMs; many thin tiles
+# (64 or 128 columns); tiles that leave a partial wave; long rows with a ragged last step (cols = 4160).
+@pytest.mark.parametrize("rows,cols", [(16, 64), (32, 1024), (65536, 64), (80000, 128), (4096, 4096),
+                                       (14336, 4096), (2048, 4160)])
+@pytest.mark.parametrize("batch,use_dq,code", [(1, True, "e4m3"), (8, True, "int8"), (5, False, "e4m3")])
+def test_gemv_grid_shapes(rows, cols, batch, use_dq, code):
+    qw, p_ref, a_ref = quantized_pair(rows, cols, 7 + rows // 16 + cols, use_dq, code)
+    x = synth.activations((batch, cols), 77 + batch)
+    y1 = nf4.gemv(qw, dev_bf16(x))
+    y2 = nf4.gemv(qw, dev_bf16(x))  # same call again: same bits
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    check_matmul(y1, oracle.matmul(p_ref, a_ref, rows, cols, x), f"gemv {rows}x{cols} b{batch}")
+    nf4.check_device_error()
+
+
+def test_gemv_unaligned_scale_codes():
+    """double-quant codes starting at an odd address (the record's q array is not 4-byte aligned)"""
+    rows, cols = 512, 1536
+    qw, p_ref, a_ref = quantized_pair(rows, cols, 21, True)
+    q_off = torch.zeros(qw.absmax_q.numel() + 3, dtype=torch.uint8, device="cuda")
+    q_off[1:1 + qw.absmax_q.numel()] = qw.absmax_q
+    qw2 = nf4.QuantizedWeight(packed=qw.packed, rows=rows, cols=cols, absmax_q=q_off[1:1 + qw.absmax_q.numel()],
+                              absmax_scale=qw.absmax_scale, absmax_mean=qw.absmax_mean, dq_code=qw.dq_code)
+    assert qw2.absmax_q.data_ptr() % 4 == 1
+    x = synth.activations((3, cols), 5)
+    y = nf4.gemv(qw2, dev_bf16(x))
+    assert torch.equal(y.view(torch.int16), nf4.gemv(qw, dev_bf16(x)).view(torch.int16))
+    check_matmul(y, oracle.matmul(p_ref, a_ref, rows, cols, x), "gemv unaligned q")
 
 
 def test_gemv_zero_codes_give_zero():
@@ -302,6 +336,22 @@ def test_gemm_deterministic_and_bench_shape():
     rms = np.sqrt(np.mean(full_row ** 2))
     got = y1.float().cpu().numpy().astype(np.float64)[bs, ns]
     assert np.all(np.abs(got - ref) <= REL_TOL * np.maximum(np.abs(ref), FLOOR * rms))
+
+
+@pytest.mark.parametrize("rows,m", [(14336, 1024), (4096, 4096), (14336, 256)])
+def test_gemm_repeatable_many_tiles(rows, m):
+    """Several output tiles per CTA (the persistent grid cycles its rings many times): ten identical calls
+    give identical bits.  A slot refilled by TMA before the producer warps' reads of it were ordered, or a
+    TMEM read used before it landed, shows up here as a few weight rows differing between calls."""
+    cols = 4096
+    w = synth.normal_weights((rows, cols), 2024)
+    qw = nf4.quantize_weight(dev(w))
+    x = dev_bf16(synth.activations((m, cols), 2025))
+    ws = torch.empty(max(nf4.gemm_workspace_bytes(qw, m), 16), dtype=torch.uint8, device="cuda")
+    ref = nf4.gemm(qw, x, workspace=ws).view(torch.int16).clone()
+    for _ in range(10):
+        assert torch.equal(nf4.gemm(qw, x, workspace=ws).view(torch.int16), ref)
+    nf4.check_device_error()
 
 
 @pytest.mark.parametrize("cols", [320, 1024, 4096])
