@@ -371,8 +371,7 @@ def run_ours(args):
 # ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of each kernel at this workload, from the
 # --set full capture in profiles/kernels_nf4_path_bf16_4096x4096.md; an entry is removed whenever its kernel
 # changes after the capture
-TRAFFIC = {"quantize": 33576192, "double_quant": 1084416, "dequantize": 8683776, "gemv": 8680960,
-           "gemm": 10810624}
+TRAFFIC = {"quantize": 33576192, "double_quant": 1084416}
 
 
 def run_reference(args):
