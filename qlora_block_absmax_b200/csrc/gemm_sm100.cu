@@ -65,7 +65,6 @@ struct Smem {  // placed after the 1024-aligned stage buffers
   uint64_t acc_empty[2];
   uint32_t tmem_base;
   int abort;
-  int last;
   float unit_lut[256];
 };
 
@@ -148,8 +147,10 @@ __device__ unsigned long long g_trace[1024 * 16];
 
 // Work unit u = tile * splits + split: the split takes k stages
 // [split * kps, (split + 1) * kps).  With splits > 1 the epilogue writes an
-// fp32 partial tile to the workspace and the last split to finish a tile adds
-// the partials in split order (deterministic) and writes bf16 Y.
+// fp32 partial tile to the workspace; once every split of the tile has written
+// its partial (a counter per tile; the launch holds all units at once), split s
+// adds the partials of 32-row chunks s, s + splits, ... in split order
+// (deterministic) and writes those bf16 rows of Y.
 struct Work {
   int ntiles_m, units, splits, kps;
   __device__ int tile(int u) const { return u / splits; }
@@ -400,14 +401,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&sm->acc_empty[acc]);  // TMEM no longer needed
         __threadfence();
         epi_bar();
-        if (threadIdx.x == 0) sm->last = atomicAdd(&tile_count[wk.tile(u)], 1u) == (unsigned)(wk.splits - 1);
+        // every split of the tile waits for all partials (the splits of a tile are co-resident: the
+        // grid holds every unit at once), then finishes its share of the 32-row chunks
+        if (threadIdx.x == 0) {
+          atomicAdd(&tile_count[wk.tile(u)], 1u);
+          const unsigned long long t0 = global_ns();
+          while (*(volatile unsigned*)&tile_count[wk.tile(u)] < (unsigned)wk.splits) {
+            if (global_ns() - t0 > kWaitLimitNs) {
+              atomicOr(err, kErrTimeout);
+              *(volatile int*)&sm->abort = 1;
+              break;
+            }
+            __nanosleep(64);
+          }
+        }
         epi_bar();
         if (threadIdx.x == 0) NF4_STAMP(5);
-        if (sm->last) {
+        if (!aborted(sm)) {
           __threadfence();
           const float* tp = part + (size_t)wk.tile(u) * wk.splits * (kTileN * kTileM);
 #pragma unroll 1
-          for (int c = 0; c < kTileM / 32; ++c) {
+          for (int c = wk.split(u); c < kTileM / 32; c += wk.splits) {
             float4 acc4[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j)
@@ -435,7 +449,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             store_block(c);
           }
-          if (threadIdx.x == 0) tile_count[wk.tile(u)] = 0;  // ready for the next call
           if (threadIdx.x == 0) NF4_STAMP(6);
         }
       }
