@@ -9,15 +9,18 @@
 //
 // Tile: 128 weight rows (UMMA M, operand A) x 256 activation rows (UMMA N,
 // operand B) x 64 k per pipeline stage (one level-1 block per weight row).
-// D[n, m] lives in TMEM (lane = weight row, column = activation row); two
-// accumulators (2 x 256 columns) let the MMA run one tile ahead of the
-// epilogue.  One persistent CTA per SM walks the tiles; warp roles:
+// D[n, m] lives in TMEM (lane = weight row, column = activation row, 256
+// columns); the decoded weight tile goes straight into TMEM too (a 3-stage
+// ring of 32 columns: lane = weight row, column j = codes 2j, 2j+1 as bf16x2),
+// so the MMA reads only the activation tile from shared memory.  One
+// persistent CTA per SM walks the tiles; warp roles:
 //   warps 0-3   epilogue: tcgen05.ld -> bf16 -> Y (warp w reads TMEM lanes 32w..)
 //   warps 4-11  dequant producers, two groups of four taking alternate stages:
 //               thread p decodes weight row p of the stage (64 codes) with the
-//               byte-permute tables and writes the 128B-swizzled K-major tile
+//               byte-permute tables and stores it to its TMEM lane (tcgen05.st)
 //   warp 12     TMA producer: activation tile (256 x 64 bf16, 128B swizzle)
 //   warp 13     TMEM allocator and MMA issuer (one elected thread)
+//   warp 14     TMA producer: packed codes and 16-byte scale chunks
 // Every mbarrier wait is bounded; on timeout the device error word is set and
 // the roles leave their loops, so a fault cannot hang the GPU.
 #include <cuda.h>
@@ -34,16 +37,15 @@ namespace {
 constexpr int kTileN = 128;       // weight rows per tile (UMMA M)
 constexpr int kTileM = 256;       // activation rows per tile (UMMA N)
 constexpr int kTileK = 64;        // k per stage (128 bytes of bf16: one swizzle atom)
-constexpr int kXStages = 4;  // activation-tile ring (TMA from L2/HBM)
-constexpr int kAStages = 3;  // decoded weight-tile ring (written by the producer warps)
+constexpr int kXStages = 5;  // activation-tile ring (TMA from L2/HBM)
+constexpr int kAStages = 3;  // decoded weight-tile ring in TMEM (written by the producer warps)
 constexpr int kWStages = 6;  // packed-code + scale ring (TMA from HBM), deeper to hide its latency
-constexpr int kABytes = kTileN * kTileK * 2;  // 16 KB: decoded bf16 weight tile (operand A)
 constexpr int kBBytes = kTileM * kTileK * 2;  // 32 KB: activation tile (operand B)
 constexpr int kWBytes = kTileN * kTileK / 2;  // 4 KB: packed codes of the weight tile
 constexpr int kSBytes = kTileN * 16;          // 2 KB: 16-byte scale chunk per weight row
-constexpr int kRingBytes = kAStages * kABytes + kXStages * kBBytes + kWStages * (kWBytes + kSBytes);
+constexpr int kRingBytes = kXStages * kBBytes + kWStages * (kWBytes + kSBytes);  // A lives in TMEM
 constexpr int kAccCols = kTileM;              // fp32 columns per accumulator
-constexpr int kTmemCols = 2 * kAccCols;       // 512
+constexpr int kTmemCols = 512;               // accumulator (256 columns) + 3 A stages of 32 columns
 constexpr int kThreads = 15 * 32;
 constexpr int kEpiWarps = 4;
 constexpr int kProdWarp0 = 4;                 // producers: warps 4..11
@@ -89,11 +91,12 @@ __host__ __device__ constexpr uint32_t instr_desc(int m, int n) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t acc) {
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(acc)
       : "memory");
 }
 
@@ -171,9 +174,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;  // 1024-aligned stage buffers (swizzle atoms)
   uint8_t* gbase = smem_raw + (base - raw);
-  const uint32_t a_smem0 = base, b_smem0 = base + kAStages * kABytes;
+  const uint32_t b_smem0 = base;
   const uint32_t w_smem0 = b_smem0 + kXStages * kBBytes, s_smem0 = w_smem0 + kWStages * kWBytes;
-  uint8_t* a_gen0 = gbase;
   const uint8_t* w_gen0 = gbase + (w_smem0 - base);
   const uint8_t* s_gen0 = gbase + (s_smem0 - base);
   uint16_t* out_stage = reinterpret_cast<uint16_t*>(gbase + kRingBytes);  // epilogue transpose
@@ -251,16 +253,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         else
           a = kScaleTma ? plain : __ldg(s.absmax + b);
         const Table T = make_table(a);
-        if (!wait_or_abort(&sm->aempty[as], aph ^ 1, sm, err)) break;  // the MMAs left this slot
-        uint8_t* dst = a_gen0 + as * kABytes + p * 128;
         const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        uint32_t r[32];  // column j of the row: codes 2j, 2j+1 as bf16x2
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint32_t d[4];
           decode_word(words[c], T, d, dm);
-          *reinterpret_cast<uint4*>(dst + ((c ^ (p & 7)) << 4)) = make_uint4(d[0], d[1], d[2], d[3]);
+          r[4 * c] = d[0];
+          r[4 * c + 1] = d[1];
+          r[4 * c + 2] = d[2];
+          r[4 * c + 3] = d[3];
         }
-        fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+        if (!wait_or_abort(&sm->aempty[as], aph ^ 1, sm, err)) break;  // the MMAs left this slot
+        {
+          const uint32_t ta = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(kAccCols + as * 32);
+          asm volatile(
+              "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+              "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n"
+              "tcgen05.wait::st.sync.aligned;" ::"r"(ta),
+              "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+              "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+              "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+              "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+              : "memory");
+        }
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm->afull[as]);
       }
@@ -315,8 +332,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc = instr_desc(kTileN, kTileM);
       uint32_t it = 0, ucount = 0;
       for (int u = blockIdx.x; u < wk.units && !aborted(sm); u += gridDim.x, ++ucount) {
-        const int acc = ucount & 1;
-        if (!wait_or_abort(&sm->acc_empty[acc], ((ucount >> 1) & 1) ^ 1, sm, err)) break;
+        const int acc = 0;  // one accumulator: the A ring takes the other TMEM columns
+        if (!wait_or_abort(&sm->acc_empty[acc], (ucount & 1) ^ 1, sm, err)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + acc * kAccCols;
         bool ok = true;
@@ -329,11 +346,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           if (it == 0) NF4_STAMP(2);
-          const uint32_t a_addr = a_smem0 + as * kABytes, b_addr = b_smem0 + xs * kBBytes;
+          const uint32_t a_tm = tmem + (uint32_t)(kAccCols + as * 32), b_addr = b_smem0 + xs * kBBytes;
 #pragma unroll
-          for (int kk = 0; kk < kTileK / 16; ++kk)  // 16 bf16 = 32 bytes per MMA along k
-            tc_mma(d_tmem, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32), idesc,
-                   (j | kk) != 0);
+          for (int kk = 0; kk < kTileK / 16; ++kk)  // 16 bf16 per MMA along k: 8 TMEM columns, 32 smem bytes
+            tc_mma_ts(d_tmem, a_tm + kk * 8, smem_desc_sw128(b_addr + kk * 32), idesc, (j | kk) != 0);
           tc_commit(&sm->aempty[as]);  // slots free once these MMAs have read them
           tc_commit(&sm->xempty[xs]);
         }
@@ -346,8 +362,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------ epilogue: TMEM -> Y (or fp32 partials)
     uint32_t ucount = 0;
     for (int u = blockIdx.x; u < wk.units; u += gridDim.x, ++ucount) {
-      const int acc = ucount & 1;
-      if (!wait_or_abort(&sm->acc_full[acc], (ucount >> 1) & 1, sm, err)) break;
+      const int acc = 0;
+      if (!wait_or_abort(&sm->acc_full[acc], ucount & 1, sm, err)) break;
       tc_fence_after();
       if (threadIdx.x == 0) NF4_STAMP(4);
       const int nl = warp * 32 + lane;  // weight row within the tile
