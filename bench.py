@@ -189,7 +189,7 @@ def run_ours(args):
         c.q = torch.empty(nb, dtype=torch.uint8, device=dev)
         c.scale = torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev)
         c.mean = torch.empty(1, dtype=torch.float32, device=dev)
-        c.ws = torch.empty(256, dtype=torch.uint8, device=dev)
+        c.ws = torch.zeros(256, dtype=torch.uint8, device=dev)  # double-quant workspace: zeroed once
         c.deq = torch.empty(ROWS, COLS, dtype=torch.bfloat16, device=dev)
         c.y = torch.empty(GEMV_B, ROWS, dtype=torch.bfloat16, device=dev)
         c.Y = torch.empty(GEMM_M, ROWS, dtype=torch.bfloat16, device=dev)

@@ -108,7 +108,11 @@ NF4_API nf4_status nf4_quantize(const void *src, int32_t src_dtype, int64_t n, i
  *   scale_out   device, ceil(nb/dq_blocksize) fp32
  *   mean_out    device, 1 fp32 (4-byte aligned)
  *   workspace   device scratch of nf4_double_quant_workspace_bytes(nb) bytes,
- *               16-byte aligned; its contents on entry are ignored
+ *               16-byte aligned, owned by the caller.  Zero-fill it before its
+ *               first use; every call that completes leaves it ready for the
+ *               next one (no clearing between calls).  Calls that may run at
+ *               the same time need separate buffers; after
+ *               nf4_check_device_error reports an error, zero it again.
  * dq_blocksize must be 256.  nb == 0 launches nothing and leaves mean_out unset. */
 NF4_API nf4_status nf4_double_quant(const float *absmax, int64_t nb, int32_t dq_blocksize, int32_t dq_code,
                             uint8_t *q_out, float *scale_out, float *mean_out, void *workspace,

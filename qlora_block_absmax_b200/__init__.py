@@ -112,8 +112,8 @@ def double_quant(absmax: torch.Tensor, code: str = "e4m3", dq_blocksize: int = D
     else:
         q, scale, mean = out
     ws_bytes = lib.nf4_double_quant_workspace_bytes(nb)
-    if workspace is None:
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=absmax.device)
+    if workspace is None:  # a fresh zeroed buffer (a caller's own buffer is zeroed once and reused)
+        workspace = torch.zeros(ws_bytes, dtype=torch.uint8, device=absmax.device)
     st = lib.nf4_double_quant(_ptr(absmax), nb, dq_blocksize, _DQ_CODES[code], _ptr(q), _ptr(scale), _ptr(mean),
                               _ptr(workspace), workspace.numel(), _stream(stream))
     _lib.check(st, "nf4_double_quant")

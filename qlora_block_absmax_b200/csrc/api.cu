@@ -148,7 +148,7 @@ nf4_status nf4_double_quant(const float* absmax, int64_t nb, int32_t dq_blocksiz
   DeviceInfo d;
   nf4_status st = device_info(&d);
   if (st != NF4_OK) return st;
-  return from_cuda(nf4::launch_double_quant(absmax, nb, dq_code, q_out, scale_out, mean_out, workspace,
+  return from_cuda(nf4::launch_double_quant(absmax, nb, dq_code, q_out, scale_out, mean_out, workspace, false,
                                             d.error_word, reinterpret_cast<cudaStream_t>(stream), d.num_sms));
 }
 
@@ -203,7 +203,7 @@ nf4_status nf4_double_quant_noalloc(const float* absmax, int64_t nb, int32_t dq_
   void* scratch = nullptr;
   if ((st = scratch_address(&scratch)) != NF4_OK) return st;
   // the launcher clears the scratch on `stream` before the kernel reads it
-  return from_cuda(nf4::launch_double_quant(absmax, nb, dq_code, q_out, scale_out, mean_out, scratch,
+  return from_cuda(nf4::launch_double_quant(absmax, nb, dq_code, q_out, scale_out, mean_out, scratch, true,
                                             d.error_word, reinterpret_cast<cudaStream_t>(stream), d.num_sms));
 }
 

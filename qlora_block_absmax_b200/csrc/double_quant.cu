@@ -15,6 +15,12 @@
 // of order.  Warp shuffles and shared memory combine threads, 64-bit atomics
 // combine CTAs.  After a grid barrier every CTA normalises the same limbs,
 // rounds the sum once to fp64 and derives mu.
+//
+// The workspace keeps itself ready for the next call: the barrier is a
+// counter the last arriving CTA resets before it advances an epoch word (the
+// others wait for the epoch to change), and the limbs are double-buffered by
+// epoch parity -- a call adds into limbs[e & 1] and clears limbs[(e + 1) & 1],
+// which the previous call used.  Only the first call needs a zeroed buffer.
 // Codes: one warp per 256-value block.
 #include "nf4_common.cuh"
 #include "internal.h"
@@ -25,8 +31,9 @@ namespace {
 constexpr int kLimbs = 10;
 
 struct SumWorkspace {
-  unsigned long long limb[kLimbs];  // two's-complement running sums of 32-bit digits
-  unsigned int done;                // CTAs finished
+  unsigned long long limb[2][kLimbs];  // two's-complement running sums of 32-bit digits, by epoch parity
+  unsigned int count;                  // CTAs arrived at the barrier of the current epoch
+  unsigned int epoch;                  // barrier generation
 };
 static_assert(sizeof(SumWorkspace) <= kDoubleQuantWorkspace, "workspace");
 
@@ -141,8 +148,13 @@ __global__ void __launch_bounds__(256) dq_fused_kernel(const float* __restrict__
                                                        uint8_t* __restrict__ q, float* __restrict__ scale,
                                                        float* __restrict__ mean_out, SumWorkspace* __restrict__ ws,
                                                        unsigned* __restrict__ err) {
-  // ---- phase 1: this thread's values into the integer limbs
-  if (threadIdx.x == 0) DQ_STAMP(0);
+  // ---- phase 1: this thread's values into the integer limbs of this call's epoch (the epoch
+  // cannot advance before every CTA, this one included, has arrived at the barrier)
+  __shared__ unsigned s_epoch;
+  if (threadIdx.x == 0) {
+    DQ_STAMP(0);
+    s_epoch = *reinterpret_cast<volatile unsigned*>(&ws->epoch);
+  }
   long long acc[kLimbs];
 #pragma unroll
   for (int L = 0; L < kLimbs; ++L) acc[L] = 0;
@@ -169,27 +181,36 @@ __global__ void __launch_bounds__(256) dq_fused_kernel(const float* __restrict__
 #pragma unroll
     for (int L = 0; L < kLimbs; ++L) red[warp][L] = acc[L];
   __syncthreads();
+  const unsigned epoch = s_epoch;
+  unsigned long long* limb = ws->limb[epoch & 1];
   if (threadIdx.x < kLimbs) {
     long long t = 0;
     for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w][threadIdx.x];
-    atomicAdd(&ws->limb[threadIdx.x], (unsigned long long)t);  // wraps mod 2^64 = signed add
+    atomicAdd(&limb[threadIdx.x], (unsigned long long)t);  // wraps mod 2^64 = signed add
+  } else if (blockIdx.x == 0 && threadIdx.x < 2 * kLimbs) {
+    ws->limb[(epoch + 1) & 1][threadIdx.x - kLimbs] = 0ull;  // ready for the next call
   }
   __threadfence();
   __syncthreads();
 
-  // ---- grid barrier (bounded)
+  // ---- grid barrier (bounded): the last CTA to arrive resets the count and advances the epoch
   if (threadIdx.x == 0) {
     DQ_STAMP(1);
-    atomicAdd(&ws->done, 1u);
     int ok = 1;
-    const unsigned long long t0 = global_ns();
-    // poll with plain loads (an atomic per poll would contend with the arrivals)
-    while (*reinterpret_cast<volatile unsigned*>(&ws->done) < gridDim.x) {
-      __nanosleep(64);
-      if (global_ns() - t0 > kWaitLimitNs) {
-        atomicOr(err, kErrTimeout);
-        ok = 0;
-        break;
+    if (atomicAdd(&ws->count, 1u) == gridDim.x - 1) {
+      ws->count = 0;
+      __threadfence();
+      atomicExch(&ws->epoch, epoch + 1);
+    } else {
+      const unsigned long long t0 = global_ns();
+      // poll with plain loads (an atomic per poll would contend with the arrivals)
+      while (*reinterpret_cast<volatile unsigned*>(&ws->epoch) == epoch) {
+        __nanosleep(64);
+        if (global_ns() - t0 > kWaitLimitNs) {
+          atomicOr(err, kErrTimeout);
+          ok = 0;
+          break;
+        }
       }
     }
     __threadfence();
@@ -197,7 +218,7 @@ __global__ void __launch_bounds__(256) dq_fused_kernel(const float* __restrict__
     if (ok) {
       long long l[kLimbs];
 #pragma unroll
-      for (int L = 0; L < kLimbs; ++L) l[L] = (long long)atomicAdd(&ws->limb[L], 0ull);
+      for (int L = 0; L < kLimbs; ++L) l[L] = (long long)atomicAdd(&limb[L], 0ull);
       s_mu = finish_mean(l, nb);  // the same integers in every CTA: the same mu
       if (blockIdx.x == 0) *mean_out = s_mu;
     }
@@ -264,9 +285,10 @@ __global__ void __launch_bounds__(256) dq_fused_kernel(const float* __restrict__
 }  // namespace
 
 cudaError_t launch_double_quant(const float* absmax, int64_t nb, int dq_code, uint8_t* q, float* scale,
-                                float* mean, void* workspace, unsigned* err, cudaStream_t stream, int num_sms) {
-  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(SumWorkspace), stream);
-  if (e != cudaSuccess) return e;
+                                float* mean, void* workspace, bool clear, unsigned* err, cudaStream_t stream,
+                                int num_sms) {
+  cudaError_t e = cudaSuccess;
+  if (clear && (e = cudaMemsetAsync(workspace, 0, sizeof(SumWorkspace), stream)) != cudaSuccess) return e;
   // one CTA per SM: 256 threads and ~1 KB of shared memory, so all are resident
   int64_t grid = (nb + 256 * 4 - 1) / (256 * 4);
   if (grid > num_sms) grid = num_sms;

@@ -25,8 +25,10 @@ struct Scales {
 cudaError_t launch_quantize(const void* src, bool bf16, int64_t n, uint8_t* packed, float* absmax,
                             cudaStream_t stream, int num_sms);
 
+// workspace: zero before its first use, left ready by every completed call; `clear` zeroes it first
 cudaError_t launch_double_quant(const float* absmax, int64_t nb, int dq_code, uint8_t* q, float* scale,
-                                float* mean, void* workspace, unsigned* err, cudaStream_t stream, int num_sms);
+                                float* mean, void* workspace, bool clear, unsigned* err, cudaStream_t stream,
+                                int num_sms);
 constexpr size_t kDoubleQuantWorkspace = 256;
 
 cudaError_t launch_dequantize(const uint8_t* packed, const Scales& s, int64_t n, void* out, bool out_bf16,

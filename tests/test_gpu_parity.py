@@ -160,6 +160,23 @@ def test_double_quant_bit_exact(case, code):
     assert np.array_equal(q.cpu().numpy(), q_ref)
 
 
+def test_double_quant_workspace_reused():
+    """one workspace, zeroed once, across calls of different sizes (different grids) and both codes:
+    every call leaves its barrier and exact-sum buffers ready for the next, so each result is exact"""
+    cases = dq_cases()
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    for name, code in [("config2", "e4m3"), ("one", "int8"), ("wide", "e4m3"), ("257", "int8"),
+                       ("config2", "int8"), ("signed", "e4m3"), ("zeros_and_tiny", "e4m3"), ("config2", "e4m3")]:
+        a = cases[name]
+        c = oracle.DQ_E4M3 if code == "e4m3" else oracle.DQ_INT8
+        q_ref, s_ref, m_ref = oracle.double_quant(a, 256, c)
+        q, s, m = nf4.double_quant(dev(a), code, workspace=ws)
+        assert np.float32(m.item()).view(np.uint32) == np.float32(m_ref).view(np.uint32), name
+        assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32)), name
+        assert np.array_equal(q.cpu().numpy(), q_ref), name
+    nf4.check_device_error()
+
+
 # --------------------------------------------------------------------------- dequantize
 
 @pytest.mark.parametrize("use_dq,code", [(False, "e4m3"), (True, "e4m3"), (True, "int8")])

@@ -30,7 +30,7 @@ def run(lib, absmax, code, noalloc):
     if noalloc:
         st = lib.nf4_double_quant_noalloc(ptr(absmax), nb, 256, code, ptr(q), ptr(scale), ptr(mean), stream)
     else:
-        ws = torch.empty(lib.nf4_double_quant_workspace_bytes(nb), dtype=torch.uint8, device="cuda")
+        ws = torch.zeros(lib.nf4_double_quant_workspace_bytes(nb), dtype=torch.uint8, device="cuda")
         st = lib.nf4_double_quant(ptr(absmax), nb, 256, code, ptr(q), ptr(scale), ptr(mean), ptr(ws),
                                   ws.numel(), stream)
     assert st == 0, _lib.STATUS_NAMES.get(st, st)
