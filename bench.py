@@ -195,7 +195,7 @@ def run_ours(args):
         c.Y = torch.empty(GEMM_M, ROWS, dtype=torch.bfloat16, device=dev)
         c.qw = nf4.QuantizedWeight(packed=c.packed, rows=ROWS, cols=COLS, absmax_q=c.q, absmax_scale=c.scale,
                                    absmax_mean=c.mean, dq_code=nf4.NF4_DQ_E4M3)
-        c.gws = torch.empty(max(nf4.gemm_workspace_bytes(c.qw, GEMM_M), 16), dtype=torch.uint8, device=dev)
+        c.gws = torch.zeros(max(nf4.gemm_workspace_bytes(c.qw, GEMM_M), 16), dtype=torch.uint8, device=dev)
         cs.append(c)
     stream = torch.cuda.current_stream()
 

@@ -162,7 +162,12 @@ NF4_API nf4_status nf4_gemv(const nf4_weight *w, const void *x, int32_t batch, v
  *   x  device bf16 [m, cols];  y  device bf16 [m, rows];  m >= 1
  *   cols % 64 == 0; rows % 128 == 0.
  *   workspace  device scratch of nf4_gemm_workspace_bytes(w, m) bytes (may be
- *              NULL when that size is 0), 16-byte aligned. */
+ *              NULL when that size is 0), 16-byte aligned, owned by the
+ *              caller.  Zero-fill it before its first use; every call that
+ *              completes leaves it ready for the next (no clearing between
+ *              calls).  Calls that may run at the same time need separate
+ *              buffers; after nf4_check_device_error reports an error, zero it
+ *              again. */
 NF4_API nf4_status nf4_gemm(const nf4_weight *w, const void *x, int64_t m, void *y, void *workspace,
                     size_t workspace_bytes, nf4_stream_t stream);
 NF4_API size_t nf4_gemm_workspace_bytes(const nf4_weight *w, int64_t m);

@@ -175,7 +175,7 @@ def gemm(qw: QuantizedWeight, x: torch.Tensor, out=None, workspace: Optional[tor
         out = torch.empty(m, qw.rows, dtype=torch.bfloat16, device=x.device)
     ws_bytes = lib.nf4_gemm_workspace_bytes(ctypes.byref(d), m)
     if workspace is None and ws_bytes:
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=x.device)
+        workspace = torch.zeros(ws_bytes, dtype=torch.uint8, device=x.device)  # zeroed once, then reusable
     st = lib.nf4_gemm(ctypes.byref(d), _ptr(x2), m, _ptr(out), _ptr(workspace),
                       workspace.numel() if workspace is not None else 0, _stream(stream))
     _lib.check(st, "nf4_gemm")

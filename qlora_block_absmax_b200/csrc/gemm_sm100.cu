@@ -153,7 +153,9 @@ __device__ unsigned long long g_trace[1024 * 16];
 // fp32 partial tile to the workspace; once every split of the tile has written
 // its partial (a counter per tile; the launch holds all units at once), split s
 // adds the partials of 32-row chunks s, s + splits, ... in split order
-// (deterministic) and writes those bf16 rows of Y.
+// (deterministic) and writes those bf16 rows of Y.  Each split then arrives a
+// second time; the last of those resets the counter, so the workspace is left
+// ready for the next call.
 struct Work {
   int ntiles_m, units, splits, kps;
   __device__ int tile(int u) const { return u / splits; }
@@ -430,6 +432,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             __nanosleep(64);
           }
+          // second arrival: the split that completes 2 * splits has seen every split pass the wait
+          // above, so it can reset the counter for the next call
+          if (!aborted(sm) && atomicAdd(&tile_count[wk.tile(u)], 1u) == 2u * (unsigned)wk.splits - 1u)
+            tile_count[wk.tile(u)] = 0;
         }
         epi_bar();
         if (threadIdx.x == 0) NF4_STAMP(5);
@@ -597,8 +603,6 @@ cudaError_t launch_gemm(const uint8_t* packed, const Scales& s, int64_t rows, in
     const size_t cbytes = ((size_t)ntiles * 4 + 255) & ~(size_t)255;
     counters = static_cast<unsigned*>(workspace);
     part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + cbytes);
-    cudaError_t e = cudaMemsetAsync(counters, 0, (size_t)ntiles * 4, stream);
-    if (e != cudaSuccess) return e;
   }
   const int R = (int)rows, C = (int)cols, M = (int)m;
   if (dq && scale_tma)

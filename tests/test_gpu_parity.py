@@ -364,7 +364,7 @@ def test_gemm_repeatable_many_tiles(rows, m):
     w = synth.normal_weights((rows, cols), 2024)
     qw = nf4.quantize_weight(dev(w))
     x = dev_bf16(synth.activations((m, cols), 2025))
-    ws = torch.empty(max(nf4.gemm_workspace_bytes(qw, m), 16), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(max(nf4.gemm_workspace_bytes(qw, m), 16), dtype=torch.uint8, device="cuda")
     ref = nf4.gemm(qw, x, workspace=ws).view(torch.int16).clone()
     for _ in range(10):
         assert torch.equal(nf4.gemm(qw, x, workspace=ws).view(torch.int16), ref)
