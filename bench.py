@@ -231,30 +231,30 @@ def run_ours(args):
     l0 = nf4.kernel_launches()
     step(cs[0])
     launches_per_step = nf4.kernel_launches() - l0
-    # The device-timed region is one CUDA graph holding the K steps, with an
-    # event-record node before and after every library call, so host-side
+    # The device-timed region is one CUDA graph holding the K steps (the library
+    # launches are chained with programmatic dependent launch), so host-side
     # marshalling cannot gap the GPU timeline.
-    def capture(nsteps, with_events):
-        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)]
-               for _ in range(nsteps)] if with_events else None
+    def capture(nsteps, only=None):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             for i in range(nsteps):
-                for j, f in enumerate(calls(cs[i % copies])):
-                    if with_events:
-                        evs[i][j].record()
+                fs = calls(cs[i % copies])
+                for f in (fs if only is None else (fs[only],)):
                     f()
-                if with_events:
-                    evs[i][5].record()
-        return g, evs
+        return g
 
-    g_warm, _ = capture(args.warmup, False)
-    g_timed, events = capture(args.steps, True)
+    g_warm = capture(args.warmup)
+    g_timed = capture(args.steps)
+    # per-kernel times: one graph per library call holding its K launches on the
+    # same rotating inputs, timed as a whole (no event nodes between launches)
+    g_kernel = [capture(args.steps, j) for j in range(len(KERNELS))]
     g_warm.replay()
+    for g in g_kernel:
+        g.replay()
     nf4.check_device_error()
     barrier()
 
-    # ---- device-timed region: K steps (one graph replay), per-kernel events inside
+    # ---- device-timed region: K steps (one graph replay)
     sampler = ClockSampler(local)
     sampler.start()
     barrier()
@@ -265,14 +265,19 @@ def run_ours(args):
     t_end.record(stream)
     barrier()
     launches = launches_per_step * args.steps
-    clocks = sampler.stop()
     elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end))
-    per_kernel_ms = {k: 0.0 for k in KERNELS}
-    for ev in events:
-        for j, k in enumerate(KERNELS):
-            per_kernel_ms[k] += ev[j].elapsed_time(ev[j + 1])
+    per_kernel_ms = {}
+    for j, k in enumerate(KERNELS):
+        k0 = torch.cuda.Event(enable_timing=True)
+        k1 = torch.cuda.Event(enable_timing=True)
+        k0.record(stream)
+        g_kernel[j].replay()
+        k1.record(stream)
+        barrier()
+        per_kernel_ms[k] = max_over_ranks(k0.elapsed_time(k1))
+    clocks = sampler.stop()
     nf4.check_device_error()
-    del g_warm, g_timed
+    del g_warm, g_timed, g_kernel
 
     # ---- end to end through the public API with host buffers
     host_out = {"packed": torch.empty(n // 2, dtype=torch.uint8).pin_memory(),
@@ -354,7 +359,8 @@ def run_ours(args):
         "breakdown": breakdown,
         "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": int(launches),
-        "launch": "the K timed steps captured in one CUDA graph; e2e leg launches eagerly",
+        "launch": ("the K timed steps captured in one CUDA graph, launches chained with programmatic dependent "
+                   "launch; per-kernel times from one graph of K launches of that kernel; e2e leg launches eagerly"),
         "clocks": clocks,
         "impl": "ours",
     }

@@ -26,11 +26,13 @@ __device__ __forceinline__ float block_scale(const Scales& s, const float* unit_
 template <bool kDQ, bool kBF16>
 __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restrict__ packed, Scales s, int64_t n,
                                                          void* __restrict__ out) {
+  pdl_launch_dependents();
   __shared__ float code[16];
   __shared__ float unit_lut[kDQ ? 256 : 1];
   if (threadIdx.x < 16) code[threadIdx.x] = c_code[threadIdx.x];
   if (kDQ) unit_lut[threadIdx.x & 255] = dq_unit(threadIdx.x & 255, s.dq_code);
   __syncthreads();
+  pdl_wait();
 
   const int sub = threadIdx.x & 3;
   const int64_t nfull = n / kBlock;
@@ -102,8 +104,10 @@ __global__ void __launch_bounds__(256) dequantize_bf16_kernel(const uint8_t* __r
                                                               int64_t n, __nv_bfloat16* __restrict__ out) {
   __shared__ float unit_lut[kDQ ? 256 : 1];
   __shared__ __align__(16) uint4 stage[8][32 * 8];  // per warp: 32 blocks x 8 chunks of 16 bytes
+  pdl_launch_dependents();
   if (kDQ) unit_lut[threadIdx.x & 255] = dq_unit(threadIdx.x & 255, s.dq_code);
   __syncthreads();
+  pdl_wait();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const DecodeMul dm = decode_mul();
   uint4* st = stage[warp];
@@ -175,19 +179,23 @@ cudaError_t launch_dequantize(const uint8_t* packed, const Scales& s, int64_t n,
     if (g2 > cap) g2 = cap;
     if (g2 < 1) g2 = 1;
     auto* ob = static_cast<__nv_bfloat16*>(out);
-    if (dq)
-      dequantize_bf16_kernel<true><<<(unsigned)g2, 256, 0, stream>>>(packed, s, n, ob);
-    else
-      dequantize_bf16_kernel<false><<<(unsigned)g2, 256, 0, stream>>>(packed, s, n, ob);
+    const cudaError_t e = dq ? launch_pdl(dequantize_bf16_kernel<true>, dim3((unsigned)g2), dim3(256), 0, stream,
+                                          packed, s, n, ob)
+                             : launch_pdl(dequantize_bf16_kernel<false>, dim3((unsigned)g2), dim3(256), 0, stream,
+                                          packed, s, n, ob);
     count_launches(1);
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
   }
-  if (dq && out_bf16) dequantize_kernel<true, true><<<(unsigned)grid, 256, 0, stream>>>(packed, s, n, out);
-  if (dq && !out_bf16) dequantize_kernel<true, false><<<(unsigned)grid, 256, 0, stream>>>(packed, s, n, out);
-  if (!dq && out_bf16) dequantize_kernel<false, true><<<(unsigned)grid, 256, 0, stream>>>(packed, s, n, out);
-  if (!dq && !out_bf16) dequantize_kernel<false, false><<<(unsigned)grid, 256, 0, stream>>>(packed, s, n, out);
+  const dim3 g((unsigned)grid), b(256);
+  cudaError_t e;
+  if (dq)
+    e = out_bf16 ? launch_pdl(dequantize_kernel<true, true>, g, b, 0, stream, packed, s, n, out)
+                 : launch_pdl(dequantize_kernel<true, false>, g, b, 0, stream, packed, s, n, out);
+  else
+    e = out_bf16 ? launch_pdl(dequantize_kernel<false, true>, g, b, 0, stream, packed, s, n, out)
+                 : launch_pdl(dequantize_kernel<false, false>, g, b, 0, stream, packed, s, n, out);
   count_launches(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace nf4

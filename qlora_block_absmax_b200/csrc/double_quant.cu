@@ -148,6 +148,7 @@ __global__ void __launch_bounds__(256) dq_fused_kernel(const float* __restrict__
                                                        uint8_t* __restrict__ q, float* __restrict__ scale,
                                                        float* __restrict__ mean_out, SumWorkspace* __restrict__ ws,
                                                        unsigned* __restrict__ err) {
+  pdl_launch_dependents();  // the next kernel may set itself up; it still waits for this one to finish
   // ---- phase 1: this thread's values into the integer limbs of this call's epoch (the epoch
   // cannot advance before every CTA, this one included, has arrived at the barrier)
   __shared__ unsigned s_epoch;

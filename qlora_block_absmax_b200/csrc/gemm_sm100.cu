@@ -173,6 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __nv_bfloat16* __restrict__ y, float* __restrict__ part, unsigned* __restrict__ tile_count,
                 unsigned* err) {
   extern __shared__ uint8_t smem_raw[];
+  pdl_launch_dependents();
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;  // 1024-aligned stage buffers (swizzle atoms)
   uint8_t* gbase = smem_raw + (base - raw);
@@ -220,6 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();  // everything above is on-chip set-up; from here on global memory is read and written
   const uint32_t tmem = sm->tmem_base;
   if (threadIdx.x == 0) NF4_STAMP(0);
 
@@ -563,10 +565,10 @@ cudaError_t launch_variant(const Scales& s, int rows, int cols, int m, int split
     if (e != cudaSuccess) return e;
     attr_done.fetch_or(1ull << dev);
   }
-  gemm_kernel<kDQ, kScaleTma><<<grid, kThreads, kSmemBytes, stream>>>(s, rows, cols, m, splits, xmap, wmap, smap, y,
-                                                                      part, counters, err);
+  const cudaError_t e = launch_pdl(gemm_kernel<kDQ, kScaleTma>, dim3(grid), dim3(kThreads), kSmemBytes, stream, s,
+                                   rows, cols, m, splits, xmap, wmap, smap, y, part, counters, err);
   count_launches(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace

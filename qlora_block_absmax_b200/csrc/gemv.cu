@@ -81,8 +81,10 @@ __global__ void __launch_bounds__(kWarps * 32, NT >= 4 ? 1 : 2)
                 const __nv_bfloat16* __restrict__ x, int batch, __nv_bfloat16* __restrict__ y) {
   __shared__ float unit_lut[kDQ ? 256 : 1];
   __shared__ float red[kWarps][16][8 * NT];
+  pdl_launch_dependents();
   if (kDQ) unit_lut[threadIdx.x & 255] = dq_unit(threadIdx.x & 255, s.dq_code);
   __syncthreads();
+  pdl_wait();
   const float mu = kDQ ? *s.mean : 0.0f;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -164,12 +166,14 @@ cudaError_t launch_nt(const uint8_t* packed, const Scales& s, int64_t rows, int6
   const unsigned grid = (unsigned)(rows / 16);
   const auto* xb = static_cast<const __nv_bfloat16*>(x);
   auto* yb = static_cast<__nv_bfloat16*>(y);
-  if (s.absmax == nullptr)
-    gemv_kernel<NT, true><<<grid, kWarps * 32, 0, stream>>>(packed, s, rows, cols, xb, batch, yb);
-  else
-    gemv_kernel<NT, false><<<grid, kWarps * 32, 0, stream>>>(packed, s, rows, cols, xb, batch, yb);
+  const cudaError_t e =
+      s.absmax == nullptr
+          ? launch_pdl(gemv_kernel<NT, true>, dim3(grid), dim3(kWarps * 32), 0, stream, packed, s, rows, cols, xb,
+                       batch, yb)
+          : launch_pdl(gemv_kernel<NT, false>, dim3(grid), dim3(kWarps * 32), 0, stream, packed, s, rows, cols, xb,
+                       batch, yb);
   count_launches(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace

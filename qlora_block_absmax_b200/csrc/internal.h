@@ -6,6 +6,25 @@
 
 namespace nf4 {
 
+// Launch with programmatic stream serialization: the kernel may start while the
+// previous kernel in the stream finishes; it waits for it (griddepcontrol.wait)
+// before touching global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 constexpr int kBlock = 64;      // level-1 block (elements per absmax)
 constexpr int kDqBlock = 256;   // level-2 block (absmax values per second-level scale)
 

@@ -73,6 +73,7 @@ template <bool kBF16>
 __global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ src, int64_t n,
                                                        uint8_t* __restrict__ packed,
                                                        float* __restrict__ absmax) {
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const uint32_t entry = c_q32[lane];
   const int sub = lane & 3;                                  // which 16 of the block's 64
@@ -96,6 +97,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ 
   };
   Raw cur, nxt;
   int64_t wb = warp_id * 8;
+  pdl_wait();
   if (wb < nblocks) fetch(wb, cur);
   for (; wb < nblocks; wb += warps_total * 8) {  // uniform per warp
     if (wb + warps_total * 8 < nblocks) fetch(wb + warps_total * 8, nxt);
@@ -185,12 +187,12 @@ cudaError_t launch_quantize(const void* src, bool bf16, int64_t n, uint8_t* pack
   const int64_t cap = (int64_t)num_sms * occ;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
-  if (bf16)
-    quantize_kernel<true><<<(unsigned)grid, 256, 0, stream>>>(src, n, packed, absmax);
-  else
-    quantize_kernel<false><<<(unsigned)grid, 256, 0, stream>>>(src, n, packed, absmax);
+  const cudaError_t e = bf16 ? launch_pdl(quantize_kernel<true>, dim3((unsigned)grid), dim3(256), 0, stream, src, n,
+                                           packed, absmax)
+                              : launch_pdl(quantize_kernel<false>, dim3((unsigned)grid), dim3(256), 0, stream, src, n,
+                                           packed, absmax);
   count_launches(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace nf4
