@@ -15,8 +15,9 @@
 // midpoints rounded down to fp32) below x.  A 32-bucket table covers [-1, 1];
 // lane j of every warp holds bucket j: the one threshold inside it (2.0 if
 // none) with the count of thresholds below the bucket in its low 4 mantissa
-// bits.  x is first estimated as q = w * RN(1/a) (within 3 * 2^-24 of x); q
-// picks the bucket, a shuffle fetches the entry, and code = base + (q > entry).
+// bits.  x is first estimated as q = w * RN(1/a) (within 3 * 2^-24 of x); one
+// fused multiply-add rounded down puts q's bucket in the low 5 mantissa bits
+// of its result, a shuffle fetches the entry, and code = base + (q > entry).
 // When q lies within 2^-19 of the entry -- where the estimate, or the 4 bits
 // stored in the entry, could change the decision -- the exact quotient
 // __fdiv_rn(w, a) is compared with the exact threshold instead.  Every code is
@@ -48,9 +49,10 @@ __device__ __noinline__ int code_exact(float w, float a) {
 // (the lookup is a shuffle).  q estimates w / a within 3 * 2^-24.  `gap`
 // tracks the smallest distance between an estimate and its entry.
 __device__ __forceinline__ uint32_t code_fast(uint32_t entry, float q, float& gap) {
-  const float v = __fmaf_rn(q, NF4_Q32_SCALE, 3.0f);
-  // lane index wraps modulo 32, so the exponent bits above the bucket need no mask
-  const uint32_t e = __shfl_sync(0xffffffffu, entry, __float_as_int(v) >> 18);
+  // v = 2^23 + 16 + floor(16 S q) lies in [2^23, 2^23 + 32): the bucket is its low 5 mantissa bits,
+  // and a shuffle takes its source lane modulo 32
+  const float v = __fmaf_rd(q, 16.0f * NF4_Q32_SCALE, 0x1p23f + 16.0f);
+  const uint32_t e = __shfl_sync(0xffffffffu, entry, __float_as_int(v));
   const float thr = __uint_as_float(e);
   gap = fminf(gap, fabsf(q - thr));
   return (e & 15u) + (q > thr ? 1u : 0u);
