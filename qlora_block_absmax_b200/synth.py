@@ -79,3 +79,22 @@ def config2_weight() -> np.ndarray:
 def layer_seed(layer: int, proj: int) -> int:
     """seed of projection `proj` (index into LLAMA8B_LAYER) of decoder layer `layer`"""
     return 2000 + 7 * layer + proj
+
+
+def normal_weights_device(shape, seed: int, std: float = WEIGHT_STD, device: str = "cuda"):
+    """bf16 ~N(0, std^2) generated on the device, for the whole-model workload (7e9 weights are too many to draw
+    on the host): torch's seeded device generator, fp32 draws scaled and cast once to bf16 (nearest even).  The
+    values are fixed by the seed; checks copy the tensors they need back to the host as the oracle's input."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return (torch.randn(shape, generator=g, device=device, dtype=torch.float32) * std).to(torch.bfloat16)
+
+
+def activations_device(shape, seed: int, device: str = "cuda"):
+    """bf16 ~N(0, 1) activations from torch's seeded device generator (see normal_weights_device)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+

@@ -381,3 +381,63 @@ def test_gemm_scale_paths(cols, use_dq):
     x = synth.activations((m, cols), 72 + cols)
     y = nf4.gemm(qw, dev_bf16(x))
     check_matmul(y, oracle.matmul(p_ref, a_ref, rows, cols, x), f"gemm cols{cols} dq{use_dq}")
+
+
+# --------------------------------------------------------------------------- whole model (config 5)
+
+def test_whole_model_8b_config5():
+    """An 8B-shaped decoder stack: 32 layers x (q, k, v, o, gate, up, down), 6.98e9 bf16 weights ~N(0, 0.02), each
+    matrix from its own seed, quantized to NF4 with E4M3 double quant on the GPU, then a GEMV pass over all 224
+    matrices in layer order at batch 1, 4 and 8.  One matrix of each projection type (from different layers) is
+    checked in full against the oracle: packed codes, 8-bit absmax codes, second-level scales and mean bit for bit,
+    and 512 sampled outputs of every batch within the matmul tolerance.  Storage matches the 4.127 bits/param
+    figure (3.60 GB for the stack)."""
+    torch.cuda.empty_cache()
+    shapes = synth.LLAMA8B_LAYER
+    checked = {(3 + 5 * p) % synth.LLAMA8B_LAYERS: p for p in range(len(shapes))}  # layer -> projection
+    records, sources, total_params, stored = [], {}, 0, 0
+    for layer in range(synth.LLAMA8B_LAYERS):
+        for p, (name, rows, cols) in enumerate(shapes):
+            w = synth.normal_weights_device((rows, cols), synth.layer_seed(layer, p))
+            qw = nf4.quantize_weight(w, use_double_quant=True, code="e4m3")
+            if checked.get(layer) == p:
+                sources[(layer, p)] = w.view(torch.int16).cpu().numpy().view(np.uint16)
+            del w
+            records.append((layer, p, qw))
+            total_params += rows * cols
+            stored += qw.storage_bytes()
+    assert total_params == 6_979_321_856
+    assert abs(stored * 8 / total_params - (4 + 8 / 64 + 32 / (64 * 256))) < 1e-3
+    xs = {b: (synth.activations_device((b, 4096), 3000 + b), synth.activations_device((b, 14336), 3100 + b))
+          for b in (1, 4, 8)}
+    outs = {}
+    for b, (x_model, x_ffn) in xs.items():  # one pass over the stack, layer order
+        for layer, p, qw in records:
+            y = nf4.gemv(qw, x_ffn if shapes[p][0] == "down" else x_model)
+            if (layer, p) in sources:
+                outs[(layer, p, b)] = y
+    nf4.check_device_error()
+    r = synth.rng(77)
+    for (layer, p), src in sources.items():
+        name, rows, cols = shapes[p]
+        qw = records[layer * len(shapes) + p][2]
+        w32 = synth.bf16_bits_to_f32(src.reshape(-1))
+        p_ref, a_ref = oracle.quantize(w32)
+        q_ref, s_ref, m_ref = oracle.double_quant(a_ref, 256, oracle.DQ_E4M3)
+        assert np.array_equal(qw.packed.cpu().numpy(), p_ref), (layer, name)
+        assert np.array_equal(qw.absmax_q.cpu().numpy(), q_ref), (layer, name)
+        assert np.array_equal(qw.absmax_scale.cpu().numpy().view(np.uint32), s_ref.view(np.uint32)), (layer, name)
+        assert np.float32(qw.absmax_mean.item()).view(np.uint32) == np.float32(m_ref).view(np.uint32)
+        a_hat = oracle.absmax_reconstruct(q_ref, s_ref, m_ref, 256, oracle.DQ_E4M3)
+        for b, (x_model, x_ffn) in xs.items():
+            x = (x_ffn if name == "down" else x_model).view(torch.int16).cpu().numpy().view(np.uint16)
+            bs, ns = r.integers(0, b, 512), r.integers(0, rows, 512)
+            ref = oracle.matmul_sampled(p_ref, a_hat, rows, cols, x, bs, ns)
+            full_row = oracle.matmul(p_ref, a_hat, rows, cols, x[:1])
+            rms = np.sqrt(np.mean(full_row ** 2))
+            got = outs[(layer, p, b)].float().cpu().numpy().astype(np.float64)[bs, ns]
+            bad = np.abs(got - ref) > REL_TOL * np.maximum(np.abs(ref), FLOOR * rms)
+            assert not bad.any(), (layer, name, b, int(bad.sum()))
+    del records, outs
+    torch.cuda.empty_cache()
+
