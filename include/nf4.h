@@ -196,6 +196,14 @@ NF4_API int32_t nf4_device_supported(void);
  * library so far (all devices, all threads).  Host only. */
 NF4_API uint64_t nf4_kernel_launches(void);
 
+/* Self-test of the failure path shared by every bounded device-side wait:
+ * launches one CTA that waits on an mbarrier nothing completes.  After the
+ * library's wall-clock bound (2 s) the wait gives up, records a timeout in the
+ * device error word and the kernel returns, so the context stays usable; the
+ * next nf4_check_device_error(stream) reports NF4_ERR_TIMEOUT (and clears it).
+ * Returns the launch status. */
+NF4_API nf4_status nf4_selftest_wait_timeout(nf4_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

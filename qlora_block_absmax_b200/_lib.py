@@ -45,6 +45,7 @@ SIGNATURES = {
     "nf4_code_table": (None, [ctypes.POINTER(ctypes.c_float)]),
     "nf4_device_supported": (I32, []),
     "nf4_kernel_launches": (ctypes.c_uint64, []),
+    "nf4_selftest_wait_timeout": (ctypes.c_int, [P]),
 }
 
 _lib = None

@@ -271,4 +271,11 @@ nf4_status nf4_check_device_error(nf4_stream_t stream) {
   return NF4_OK;
 }
 
+nf4_status nf4_selftest_wait_timeout(nf4_stream_t stream) {
+  DeviceInfo d;
+  nf4_status st = device_info(&d);
+  if (st != NF4_OK) return st;
+  return from_cuda(nf4::launch_wait_timeout(d.error_word, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -441,3 +441,24 @@ def test_whole_model_8b_config5():
     del records, outs
     torch.cuda.empty_cache()
 
+
+# --------------------------------------------------------------------------- failure path
+
+def test_bounded_wait_times_out_and_context_survives():
+    """A device-side wait that nothing completes gives up after the library's bound, reports NF4_ERR_TIMEOUT
+    through nf4_check_device_error, and leaves the context usable (a quantization afterwards is exact)."""
+    from qlora_block_absmax_b200 import _lib
+    lib = _lib.load()
+    stream = torch.cuda.current_stream().cuda_stream
+    assert lib.nf4_selftest_wait_timeout(stream) == 0
+    with pytest.raises(_lib.NF4Error) as e:
+        nf4.check_device_error()
+    assert "TIMEOUT" in str(e.value)
+    nf4.check_device_error()  # the word was cleared
+    w = synth.normal_weights((4096,), 5)
+    p_ref, a_ref = oracle.quantize(w)
+    p, a = nf4.quantize(dev(w))
+    assert np.array_equal(p.cpu().numpy(), p_ref)
+    assert np.array_equal(a.cpu().numpy().view(np.uint32), a_ref.view(np.uint32))
+    nf4.check_device_error()
+
