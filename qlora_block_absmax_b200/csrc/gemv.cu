@@ -21,8 +21,17 @@
 //   decode feeds up to 8 activation rows per n-tile.  Lanes with the same t
 //   use the same four k positions per MMA, which keeps the B fragment a
 //   contiguous 8-byte slice of x.
+// At batch 1 the decode, not HBM, bounds the kernel, so half of it leaves
+// the ALU pipe: rows g+8 are expanded through a 64 KB shared table of fp32
+// code pairs instead (one copy per bank; a byte permute of the packed word
+// with the lane's offset is the address, then two multiplies by a and one
+// bf16x2 convert) -- the same bf16_rn(RN(code * a)) values.  With more
+// activation rows the lookups would compete with the activation loads, so
+// larger batches decode both rows with byte permutes.
 // Partial sums of the 8 warps are added in a fixed order through shared
 // memory, so results are deterministic.
+#include <atomic>
+
 #include "nf4_common.cuh"
 #include "nf4_decode.cuh"
 #include "internal.h"
@@ -32,6 +41,9 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kStepK = 256;  // k per warp step (4 level-1 blocks)
+constexpr int kPairTableBytes = 256 * 32 * 8;  // fp32 code pairs, one copy per bank
+
+__constant__ float c_code_gemv[16] = NF4_CODE_INIT;
 
 __device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -75,14 +87,23 @@ __device__ __forceinline__ void load_step(StepData& d, const uint8_t* __restrict
   }
 }
 
-template <int NT, bool kDQ>
+template <int NT, bool kDQ, bool kTable>
 __global__ void __launch_bounds__(kWarps * 32, NT >= 4 ? 1 : 2)
     gemv_kernel(const uint8_t* __restrict__ packed, Scales s, int64_t rows, int64_t cols,
                 const __nv_bfloat16* __restrict__ x, int batch, __nv_bfloat16* __restrict__ y) {
   __shared__ float unit_lut[kDQ ? 256 : 1];
   __shared__ float red[kWarps][16][8 * NT];
+  extern __shared__ __align__(16) uint8_t pair_table[];  // entry v of lane l at 256 v + 8 l
   pdl_launch_dependents();
   if (kDQ) unit_lut[threadIdx.x & 255] = dq_unit(threadIdx.x & 255, s.dq_code);
+  if (kTable) {
+#pragma unroll
+    for (int k = 0; k < kPairTableBytes / 16 / (kWarps * 32); ++k) {
+      const int idx = threadIdx.x + k * kWarps * 32;  // 16-byte pieces: two lanes' copies of one entry
+      const float hi = c_code_gemv[(idx >> 4) >> 4], lo = c_code_gemv[(idx >> 4) & 15];
+      *reinterpret_cast<float4*>(pair_table + idx * 16) = make_float4(hi, lo, hi, lo);
+    }
+  }
   __syncthreads();
   pdl_wait();
   const float mu = kDQ ? *s.mean : 0.0f;
@@ -105,6 +126,7 @@ __global__ void __launch_bounds__(kWarps * 32, NT >= 4 ? 1 : 2)
   for (int nt = 0; nt < NT; ++nt) xrow[nt] = (8 * nt + g < batch) ? x + (int64_t)(8 * nt + g) * cols : nullptr;
 
   const DecodeMul dm = decode_mul();
+  const uint32_t lane8 = (uint32_t)(lane * 8);
   StepData cur, nxt;
   int64_t st = warp;
   if (st < nsteps) load_step<kDQ>(cur, packed, s, row0, cols, st * 4 + t, st * 4 + t < nblk);
@@ -117,7 +139,9 @@ __global__ void __launch_bounds__(kWarps * 32, NT >= 4 ? 1 : 2)
       a0 = dq_absmax(unit_lut[cur.q0], cur.s0, mu);
       a1 = dq_absmax(unit_lut[cur.q1], cur.s1, mu);
     }
-    const Table T0 = make_table(a0), T1 = make_table(a1);
+    const Table T0 = make_table(a0);
+    Table T1;
+    if (!kTable) T1 = make_table(a1);
     const uint32_t w0[8] = {cur.w0[0].x, cur.w0[0].y, cur.w0[0].z, cur.w0[0].w,
                             cur.w0[1].x, cur.w0[1].y, cur.w0[1].z, cur.w0[1].w};
     const uint32_t w1[8] = {cur.w1[0].x, cur.w1[0].y, cur.w1[0].z, cur.w1[0].w,
@@ -125,9 +149,20 @@ __global__ void __launch_bounds__(kWarps * 32, NT >= 4 ? 1 : 2)
     const int64_t kbase = blk * kBlock;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
+      // row g with byte-permute pools (ALU pipe); row g+8 the same, or (kTable) through the shared pair
+      // table: a byte permute forms the address of this lane's copy, two multiplies and one convert give the
+      // pair -- moving part of the decode off the ALU pipe
       uint32_t d0[4], d1[4];
       decode_word(w0[j], T0, d0, dm);
-      decode_word(w1[j], T1, d1, dm);
+      if (kTable) {
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const float2 c = *reinterpret_cast<const float2*>(pair_table + prmt(w1[j], lane8, 0x5504u | (b << 4)));
+          d1[b] = pack_bf16x2(__fmul_rn(c.x, a1), __fmul_rn(c.y, a1));
+        }
+      } else {
+        decode_word(w1[j], T1, d1, dm);
+      }
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         uint4 xv = make_uint4(0, 0, 0, 0);
@@ -166,12 +201,29 @@ cudaError_t launch_nt(const uint8_t* packed, const Scales& s, int64_t rows, int6
   const unsigned grid = (unsigned)(rows / 16);
   const auto* xb = static_cast<const __nv_bfloat16*>(x);
   auto* yb = static_cast<__nv_bfloat16*>(y);
-  const cudaError_t e =
-      s.absmax == nullptr
-          ? launch_pdl(gemv_kernel<NT, true>, dim3(grid), dim3(kWarps * 32), 0, stream, packed, s, rows, cols, xb,
-                       batch, yb)
-          : launch_pdl(gemv_kernel<NT, false>, dim3(grid), dim3(kWarps * 32), 0, stream, packed, s, rows, cols, xb,
-                       batch, yb);
+  const bool dq = s.absmax == nullptr;
+  cudaError_t e;
+  if (NT == 1 && batch == 1) {  // decode at batch 1: the mixed decode with the 64 KB pair table
+    // the table needs the shared-memory opt-in: set it once per device and variant
+    static std::atomic<uint64_t> attr_done[2];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!(attr_done[dq].load() & (1ull << dev))) {
+      e = cudaFuncSetAttribute(dq ? (const void*)gemv_kernel<NT, true, true> : (const void*)gemv_kernel<NT, false, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, kPairTableBytes);
+      if (e != cudaSuccess) return e;
+      attr_done[dq].fetch_or(1ull << dev);
+    }
+    e = dq ? launch_pdl(gemv_kernel<NT, true, true>, dim3(grid), dim3(kWarps * 32), kPairTableBytes, stream, packed,
+                        s, rows, cols, xb, batch, yb)
+           : launch_pdl(gemv_kernel<NT, false, true>, dim3(grid), dim3(kWarps * 32), kPairTableBytes, stream, packed,
+                        s, rows, cols, xb, batch, yb);
+  } else {
+    e = dq ? launch_pdl(gemv_kernel<NT, true, false>, dim3(grid), dim3(kWarps * 32), 0, stream, packed, s, rows, cols,
+                        xb, batch, yb)
+           : launch_pdl(gemv_kernel<NT, false, false>, dim3(grid), dim3(kWarps * 32), 0, stream, packed, s, rows, cols,
+                        xb, batch, yb);
+  }
   count_launches(1);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
