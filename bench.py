@@ -377,8 +377,7 @@ def run_ours(args):
 # ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of each kernel at this workload, from the
 # --set full capture in profiles/kernels_nf4_path_bf16_4096x4096.md; an entry is removed whenever its kernel
 # changes after the capture
-TRAFFIC = {"quantize": 33576192, "double_quant": 1084928, "dequantize": 8679680, "gemv": 8681216,
-           "gemm": 10812672}
+TRAFFIC = {"quantize": 33576192, "double_quant": 1084928, "dequantize": 8679680, "gemm": 10812672}
 
 
 def run_reference(args):

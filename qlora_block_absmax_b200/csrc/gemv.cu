@@ -21,11 +21,12 @@
 //   decode feeds up to 8 activation rows per n-tile.  Lanes with the same t
 //   use the same four k positions per MMA, which keeps the B fragment a
 //   contiguous 8-byte slice of x.
-// At batch 1 the decode, not HBM, bounds the kernel, so half of it leaves
-// the ALU pipe: rows g+8 are expanded through a 64 KB shared table of fp32
-// code pairs instead (one copy per bank; a byte permute of the packed word
-// with the lane's offset is the address, then two multiplies by a and one
-// bf16x2 convert) -- the same bf16_rn(RN(code * a)) values.  With more
+// At batch 1 the decode, not HBM, bounds the kernel, so three quarters of it
+// leave the ALU pipe: row g+8 and the second half of row g's step are
+// expanded through a 64 KB shared table of fp32 code pairs instead (one copy
+// per bank; a byte permute of the packed word with the lane's offset is the
+// address, then two multiplies by a and one bf16x2 convert) -- the same
+// bf16_rn(RN(code * a)) values.  With more
 // activation rows the lookups would compete with the activation loads, so
 // larger batches decode both rows with byte permutes.
 // Partial sums of the 8 warps are added in a fixed order through shared
@@ -149,11 +150,18 @@ __global__ void __launch_bounds__(kWarps * 32, NT >= 4 ? 1 : 2)
     const int64_t kbase = blk * kBlock;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      // row g with byte-permute pools (ALU pipe); row g+8 the same, or (kTable) through the shared pair
-      // table: a byte permute forms the address of this lane's copy, two multiplies and one convert give the
-      // pair -- moving part of the decode off the ALU pipe
+      // byte-permute pools (ALU pipe), or (kTable) the shared pair table: a byte permute forms the address of
+      // this lane's copy, two multiplies and one convert give the pair -- moving decode work off the ALU pipe
       uint32_t d0[4], d1[4];
-      decode_word(w0[j], T0, d0, dm);
+      if (kTable && j >= 4) {  // (kTable) row g's second half through the table as well
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const float2 c = *reinterpret_cast<const float2*>(pair_table + prmt(w0[j], lane8, 0x5504u | (b << 4)));
+          d0[b] = pack_bf16x2(__fmul_rn(c.x, a0), __fmul_rn(c.y, a0));
+        }
+      } else {
+        decode_word(w0[j], T0, d0, dm);
+      }
       if (kTable) {
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
