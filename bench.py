@@ -145,6 +145,22 @@ def cpu_baseline(sample_rows: int, reps: int = 1):
 
 # ---------------------------------------------------------------------------- our arm
 
+def max_over_ranks(v: float, world: int, device) -> float:
+    """The largest of the ranks' values (every rank gets it); the value itself with one rank."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(step_bytes: float, steps: int, elapsed_ms_max: float, world: int) -> float:
+    """Whole-job GB/s of `world` replicas: every rank's bytes over the slowest rank's device time."""
+    return world * step_bytes / (elapsed_ms_max / steps * 1e-3) / 1e9
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -216,12 +232,8 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def max_ms(v: float) -> float:
+        return max_over_ranks(v, world, dev)
 
     for i in range(args.warmup):
         step(cs[i % copies])
@@ -265,7 +277,7 @@ def run_ours(args):
     t_end.record(stream)
     barrier()
     launches = launches_per_step * args.steps
-    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    elapsed_ms = max_ms(t_start.elapsed_time(t_end))
     per_kernel_ms = {}
     for j, k in enumerate(KERNELS):
         k0 = torch.cuda.Event(enable_timing=True)
@@ -274,7 +286,7 @@ def run_ours(args):
         g_kernel[j].replay()
         k1.record(stream)
         barrier()
-        per_kernel_ms[k] = max_over_ranks(k0.elapsed_time(k1))
+        per_kernel_ms[k] = max_ms(k0.elapsed_time(k1))
     clocks = sampler.stop()
     nf4.check_device_error()
     del g_warm, g_timed, g_kernel
@@ -333,13 +345,13 @@ def run_ours(args):
         e2e_step(i)
     e1.record(s_out)
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_ms = max_ms(e0.elapsed_time(e1))
 
     work = work_per_step()
     step_bytes = sum(v["bytes"] for v in work.values())
     ms_per_step = elapsed_ms / args.steps
-    value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
-    e2e_value = world * step_bytes / (e2e_ms / args.steps * 1e-3) / 1e9
+    value = replica_throughput(step_bytes, args.steps, elapsed_ms, world)
+    e2e_value = replica_throughput(step_bytes, args.steps, e2e_ms, world)
 
     peaks, peak_src = load_peaks()
     breakdown = {}
