@@ -69,6 +69,8 @@ def _load():
         "oracle_nf4_dequantize_bf16": (None, [P, P, I64, I32, P]),
         "oracle_nf4_matmul": (None, [P, P, I64, I64, I32, P, I64, P]),
         "oracle_nf4_matmul_sampled": (None, [P, P, I64, I64, I32, P, I64, P, P, I64, P]),
+        "oracle_nf4_matmul_dx": (None, [P, P, I64, I64, I32, P, I64, P]),
+        "oracle_nf4_matmul_dx_sampled": (None, [P, P, I64, I64, I32, P, I64, P, P, I64, P]),
         "oracle_set_threads": (None, [ctypes.c_int]),
         "oracle_get_threads": (ctypes.c_int, []),
     }
@@ -209,3 +211,29 @@ def matmul_sampled(packed: np.ndarray, absmax: np.ndarray, N: int, K: int, x_bf1
                                       _p(np.ascontiguousarray(absmax, dtype=np.float32)),
                                       N, K, blocksize, _p(x), x.shape[0], _p(bs), _p(ns), bs.size, _p(y))
     return y
+
+
+def matmul_dx(packed: np.ndarray, absmax: np.ndarray, N: int, K: int, dy_bf16: np.ndarray,
+              blocksize: int = 64) -> np.ndarray:
+    """Input gradient of ``matmul``: dy_bf16 uint16 [B, N] -> fp64 dx [B, K] = dy . Wc,
+    fp64 accumulation over n."""
+    dy = np.ascontiguousarray(dy_bf16, dtype=np.uint16).reshape(-1, N)
+    B = dy.shape[0]
+    dx = np.zeros((B, K), np.float64)
+    _load().oracle_nf4_matmul_dx(_p(np.ascontiguousarray(packed, dtype=np.uint8)),
+                                 _p(np.ascontiguousarray(absmax, dtype=np.float32)),
+                                 N, K, blocksize, _p(dy), B, _p(dx))
+    return dx
+
+
+def matmul_dx_sampled(packed: np.ndarray, absmax: np.ndarray, N: int, K: int, dy_bf16: np.ndarray,
+                      bs: np.ndarray, ks: np.ndarray, blocksize: int = 64) -> np.ndarray:
+    """fp64 dx at the given (b, k) coordinates only."""
+    dy = np.ascontiguousarray(dy_bf16, dtype=np.uint16).reshape(-1, N)
+    bs = np.ascontiguousarray(bs, dtype=np.int64)
+    ks = np.ascontiguousarray(ks, dtype=np.int64)
+    dx = np.zeros(bs.size, np.float64)
+    _load().oracle_nf4_matmul_dx_sampled(_p(np.ascontiguousarray(packed, dtype=np.uint8)),
+                                         _p(np.ascontiguousarray(absmax, dtype=np.float32)),
+                                         N, K, blocksize, _p(dy), dy.shape[0], _p(bs), _p(ks), bs.size, _p(dx))
+    return dx

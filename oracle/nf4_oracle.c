@@ -415,3 +415,40 @@ void oracle_nf4_matmul_sampled(const uint8_t *packed, const float *absmax, int64
 #pragma omp parallel for schedule(static)
   for (int64_t t = 0; t < count; ++t) y[t] = dot_row(packed, absmax, K, blocksize, ns[t], x + bs[t] * K);
 }
+
+/* ------------------------------------------------------------------------- */
+/* Input gradient of the same matmul.  [bnb-tools] "Strengths and            */
+/* limitations" (Limitations) and [bnb-tut] "QLoRA: Fine-Tuning a 4-bit       */
+/* Model": the 4-bit base weight stays frozen and receives no gradient of its */
+/* own, but the gradient passes through it to the adapters and layers below: */
+/* dx[b,k] = sum_n dy[b,n] * Wc[n,k], with Wc the same 16-bit expanded weight */
+/* as above.  Products of two bf16 values are exact in fp64; summed in fp64   */
+/* over n in ascending order.                                                 */
+/* ------------------------------------------------------------------------- */
+
+static double dot_col(const uint8_t *packed, const float *absmax, int64_t N, int64_t K,
+                      int32_t blocksize, int64_t k, const uint16_t *dyrow) {
+  const float *c = codebook32();
+  double acc = 0.0;
+  for (int64_t n = 0; n < N; ++n) {
+    int64_t i = n * K + k;
+    float wc = oracle_bf16_to_f32(oracle_bf16_rn(c[code_at(packed, i)] * absmax[i / blocksize]));
+    acc += (double)oracle_bf16_to_f32(dyrow[n]) * (double)wc;
+  }
+  return acc;
+}
+
+void oracle_nf4_matmul_dx(const uint8_t *packed, const float *absmax, int64_t N, int64_t K,
+                          int32_t blocksize, const uint16_t *dy, int64_t B, double *dx) {
+#pragma omp parallel for schedule(static)
+  for (int64_t k = 0; k < K; ++k)
+    for (int64_t b = 0; b < B; ++b) dx[b * K + k] = dot_col(packed, absmax, N, K, blocksize, k, dy + b * N);
+}
+
+void oracle_nf4_matmul_dx_sampled(const uint8_t *packed, const float *absmax, int64_t N, int64_t K,
+                                  int32_t blocksize, const uint16_t *dy, int64_t B,
+                                  const int64_t *bs, const int64_t *ks, int64_t count, double *dx) {
+  (void)B;
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < count; ++t) dx[t] = dot_col(packed, absmax, N, K, blocksize, ks[t], dy + bs[t] * N);
+}

@@ -88,6 +88,16 @@ void oracle_nf4_matmul_sampled(const uint8_t *packed, const float *absmax, int64
                                int32_t blocksize, const uint16_t *x, int64_t B,
                                const int64_t *bs, const int64_t *ns, int64_t count, double *y);
 
+/* Input gradient of that matmul (the frozen weight passes the loss gradient
+ * to the layers below): dy is bf16 [B,N]; dx[b,k] = sum_n dy[b,n]*Wc[n,k]
+ * accumulated in fp64 over n in ascending order. */
+void oracle_nf4_matmul_dx(const uint8_t *packed, const float *absmax, int64_t N, int64_t K,
+                          int32_t blocksize, const uint16_t *dy, int64_t B, double *dx);
+/* Same arithmetic for a list of (b, k) output coordinates only. */
+void oracle_nf4_matmul_dx_sampled(const uint8_t *packed, const float *absmax, int64_t N, int64_t K,
+                                  int32_t blocksize, const uint16_t *dy, int64_t B,
+                                  const int64_t *bs, const int64_t *ks, int64_t count, double *dx);
+
 /* Worker threads used by the loops marked parallel (0 = OpenMP default). */
 void oracle_set_threads(int n);
 int oracle_get_threads(void);

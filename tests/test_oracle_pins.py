@@ -359,3 +359,57 @@ def test_matmul_zero_codes_give_zero():
     a = np.ones(N * K // 64, np.float32)
     x = synth.activations((2, K), 3)
     assert np.all(oracle.matmul(p, a, N, K, x) == 0)
+
+
+
+# ---------------------------------------------------------------- input gradient (dx = dy . Wc)
+
+def test_matmul_dx_one_hot_rows_are_weight_rows():
+    """dy = e_n picks row n of the 16-bit expanded weight, exactly (catches a
+    transposed operand or a wrong row index)."""
+    N, K = 80, 192
+    w = synth.normal_weights((N, K), 61)
+    p, a = oracle.quantize(w, 64)
+    wc = synth.bf16_bits_to_f32(oracle.dequantize(p, a, N * K, 64, "bf16")).reshape(N, K)
+    rows = [0, 1, 63, 64, 79]
+    eye = synth.f32_to_bf16_bits(np.eye(N, dtype=np.float32)[rows])
+    dx = oracle.matmul_dx(p, a, N, K, eye)
+    assert np.array_equal(dx, wc[rows].astype(np.float64))
+
+
+def test_matmul_dx_adjoint_of_forward():
+    """<dy, x . Wc^T> = <dy . Wc, x> for every x, dy: the gradient is the
+    adjoint of the forward map (pinned on its own), on a non-square weight so a
+    transposed weight cannot pass."""
+    N, K = 128, 320
+    w = synth.normal_weights((N, K), 62)
+    p, a = oracle.quantize(w, 64)
+    x = synth.activations((5, K), 63)
+    dy = synth.activations((5, N), 64)
+    y = oracle.matmul(p, a, N, K, x)
+    dx = oracle.matmul_dx(p, a, N, K, dy)
+    lhs = np.sum(synth.bf16_bits_to_f32(dy).astype(np.float64) * y)
+    rhs = np.sum(dx * synth.bf16_bits_to_f32(x).astype(np.float64))
+    assert abs(lhs - rhs) <= 1e-12 * max(abs(lhs), 1.0)
+    # the same identity fails for the transpose-free mistake dx = dy . Wc[:, reversed k]
+    assert abs(lhs - np.sum(dx[:, ::-1] * synth.bf16_bits_to_f32(x).astype(np.float64))) > 1e-6
+
+
+def test_matmul_dx_numpy_product_and_sampled():
+    N, K = 96, 256
+    w = synth.normal_weights((N, K), 65)
+    p, a = oracle.quantize(w, 64)
+    wc = synth.bf16_bits_to_f32(oracle.dequantize(p, a, N * K, 64, "bf16")).reshape(N, K)
+    dy = synth.activations((4, N), 66)
+    dx = oracle.matmul_dx(p, a, N, K, dy)
+    ref = synth.bf16_bits_to_f32(dy).astype(np.float64) @ wc.astype(np.float64)
+    assert np.allclose(dx, ref, rtol=1e-12, atol=1e-15)
+    bs, ks = np.array([0, 3, 2, 1]), np.array([0, 255, 64, 129])
+    assert np.array_equal(oracle.matmul_dx_sampled(p, a, N, K, dy, bs, ks), dx[bs, ks])
+
+
+def test_matmul_dx_zero_codes_give_zero():
+    N, K = 64, 128
+    p = np.full(N * K // 2, 0x77, np.uint8)
+    a = np.ones(N * K // 64, np.float32)
+    assert np.all(oracle.matmul_dx(p, a, N, K, synth.activations((2, N), 4)) == 0)
