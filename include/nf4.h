@@ -172,6 +172,24 @@ NF4_API nf4_status nf4_gemm(const nf4_weight *w, const void *x, int64_t m, void 
                     size_t workspace_bytes, nf4_stream_t stream);
 NF4_API size_t nf4_gemm_workspace_bytes(const nf4_weight *w, int64_t m);
 
+/* Input gradient of nf4_gemm, for training adapters on a frozen 4-bit base
+ * ([bnb-tools] "Strengths and limitations": the quantized weights receive no
+ * gradient, but the gradient flows through them to the adapters; [bnb-tut]
+ * "QLoRA: Fine-Tuning a 4-bit Model": the 4-bit base stays frozen):
+ *   dX[m, k] = bf16_rn( sum_n dY[m, n] * Wc[n, k] ),  Wc as in nf4_gemv,
+ * on tcgen05 tensor cores, accumulated in fp32 (order unspecified).  The
+ * packed weight is read in its stored [rows, cols] layout; no transposed copy
+ * is made.
+ *   dy  device bf16 [m, rows] (the gradient of Y);  dx  device bf16 [m, cols]
+ *   m >= 1; rows % 64 == 0; cols % 128 == 0 (else NF4_ERR_UNSUPPORTED).
+ *   workspace  device scratch of nf4_gemm_dx_workspace_bytes(w, m) bytes, with
+ *              the same contract as nf4_gemm's workspace (zero-fill before its
+ *              first use; left ready by every completed call; separate
+ *              buffers for calls that may overlap). */
+NF4_API nf4_status nf4_gemm_dx(const nf4_weight *w, const void *dy, int64_t m, void *dx, void *workspace,
+                       size_t workspace_bytes, nf4_stream_t stream);
+NF4_API size_t nf4_gemm_dx_workspace_bytes(const nf4_weight *w, int64_t m);
+
 /* Bytes of a quantized tensor of n elements: ceil(n/2) codes + either
  * 4*ceil(n/blocksize) (fp32 absmax) or ceil(n/blocksize) 8-bit codes +
  * 4*ceil(nb/dq_blocksize) + 4 (double quant).  Host only. */

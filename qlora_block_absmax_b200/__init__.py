@@ -23,7 +23,7 @@ from . import _lib
 from ._lib import NF4_BF16, NF4_DQ_E4M3, NF4_DQ_INT8, NF4_F32, NF4Error
 
 __all__ = ["QuantizedWeight", "quantize", "double_quant", "quantize_weight", "dequantize", "gemv", "gemm",
-           "storage_bytes", "gemm_workspace_bytes", "code_table", "check_device_error", "kernel_launches", "NF4Error", "library_path"]
+           "storage_bytes", "gemm_workspace_bytes", "gemm_dx", "gemm_dx_workspace_bytes", "code_table", "check_device_error", "kernel_launches", "NF4Error", "library_path"]
 
 BLOCKSIZE = 64
 DQ_BLOCKSIZE = 256
@@ -186,6 +186,33 @@ def gemm_workspace_bytes(qw: QuantizedWeight, m: int) -> int:
     """Scratch bytes nf4_gemm needs for `m` activation rows (0 when none)."""
     d = qw.descriptor()
     return int(_lib.load().nf4_gemm_workspace_bytes(ctypes.byref(d), m))
+
+
+def gemm_dx(qw: QuantizedWeight, dy: torch.Tensor, out=None, workspace: Optional[torch.Tensor] = None,
+            stream=None) -> torch.Tensor:
+    """Input gradient of ``gemm``: dX[m, k] = bf16(sum_n dY[m, n] Wc[n, k]) for dY bf16 [M, rows]."""
+    _need_cuda(dy, "dy")
+    if dy.dtype != torch.bfloat16:
+        raise TypeError("dy must be bfloat16")
+    dy2 = dy.reshape(-1, qw.rows)
+    m = dy2.shape[0]
+    lib = _lib.load()
+    d = qw.descriptor()
+    if out is None:
+        out = torch.empty(m, qw.cols, dtype=torch.bfloat16, device=dy.device)
+    ws_bytes = lib.nf4_gemm_dx_workspace_bytes(ctypes.byref(d), m)
+    if workspace is None and ws_bytes:
+        workspace = torch.zeros(ws_bytes, dtype=torch.uint8, device=dy.device)  # zeroed once, then reusable
+    st = lib.nf4_gemm_dx(ctypes.byref(d), _ptr(dy2), m, _ptr(out), _ptr(workspace),
+                         workspace.numel() if workspace is not None else 0, _stream(stream))
+    _lib.check(st, "nf4_gemm_dx")
+    return out
+
+
+def gemm_dx_workspace_bytes(qw: QuantizedWeight, m: int) -> int:
+    """Scratch bytes nf4_gemm_dx needs for `m` gradient rows (0 when none)."""
+    d = qw.descriptor()
+    return int(_lib.load().nf4_gemm_dx_workspace_bytes(ctypes.byref(d), m))
 
 
 def storage_bytes(n: int, use_double_quant: bool = True) -> int:

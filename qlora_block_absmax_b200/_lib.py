@@ -39,6 +39,8 @@ SIGNATURES = {
     "nf4_gemv": (ctypes.c_int, [ctypes.POINTER(NF4Weight), P, I32, P, P]),
     "nf4_gemm": (ctypes.c_int, [ctypes.POINTER(NF4Weight), P, I64, P, P, SZ, P]),
     "nf4_gemm_workspace_bytes": (SZ, [ctypes.POINTER(NF4Weight), I64]),
+    "nf4_gemm_dx": (ctypes.c_int, [ctypes.POINTER(NF4Weight), P, I64, P, P, SZ, P]),
+    "nf4_gemm_dx_workspace_bytes": (SZ, [ctypes.POINTER(NF4Weight), I64]),
     "nf4_storage_bytes": (SZ, [I64, I32, I32, I32]),
     "nf4_check_device_error": (ctypes.c_int, [P]),
     "nf4_status_string": (ctypes.c_char_p, [ctypes.c_int]),

@@ -112,6 +112,12 @@ size_t nf4_gemm_workspace_bytes(const nf4_weight* w, int64_t m) {
   return nf4::gemm_workspace_bytes(w->rows, w->cols, m);
 }
 
+size_t nf4_gemm_dx_workspace_bytes(const nf4_weight* w, int64_t m) {
+  if (w == nullptr || w->rows <= 0 || w->cols <= 0 || m <= 0) return 0;
+  if (w->rows % 64 != 0 || w->cols % 128 != 0) return 0;
+  return nf4::gemm_dx_workspace_bytes(w->rows, w->cols, m);
+}
+
 int32_t nf4_device_supported(void) {
   DeviceInfo d;
   return device_info(&d) == NF4_OK ? 1 : 0;
@@ -254,6 +260,25 @@ nf4_status nf4_gemm(const nf4_weight* w, const void* x, int64_t m, void* y, void
   if ((st = device_info(&d)) != NF4_OK) return st;
   return from_cuda(nf4::launch_gemm(w->packed, s, w->rows, w->cols, x, m, y, workspace, d.error_word,
                                     reinterpret_cast<cudaStream_t>(stream), d.num_sms));
+}
+
+nf4_status nf4_gemm_dx(const nf4_weight* w, const void* dy, int64_t m, void* dx, void* workspace,
+                       size_t workspace_bytes, nf4_stream_t stream) {
+  nf4::Scales s;
+  nf4_status st = check_weight(w, &s);
+  if (st != NF4_OK) return st;
+  if (m < 0) return NF4_ERR_INVALID_ARG;
+  if (w->rows % 64 != 0 || w->cols % 128 != 0) return NF4_ERR_UNSUPPORTED;
+  if (m == 0 || w->rows == 0 || w->cols == 0) return NF4_OK;
+  if (dy == nullptr || dx == nullptr) return NF4_ERR_INVALID_ARG;
+  if (!aligned(dy, 16) || !aligned(dx, 16)) return NF4_ERR_MISALIGNED;
+  const size_t need = nf4::gemm_dx_workspace_bytes(w->rows, w->cols, m);
+  if (workspace_bytes < need || (need > 0 && workspace == nullptr)) return NF4_ERR_INVALID_ARG;
+  if (need > 0 && !aligned(workspace, 16)) return NF4_ERR_MISALIGNED;
+  DeviceInfo d;
+  if ((st = device_info(&d)) != NF4_OK) return st;
+  return from_cuda(nf4::launch_gemm_dx(w->packed, s, w->rows, w->cols, dy, m, dx, workspace, d.error_word,
+                                       reinterpret_cast<cudaStream_t>(stream), d.num_sms));
 }
 
 nf4_status nf4_check_device_error(nf4_stream_t stream) {

@@ -30,12 +30,13 @@
 #include "nf4_common.cuh"
 #include "nf4_decode.cuh"
 #include "internal.h"
+#include "umma.cuh"
 
 namespace nf4 {
 namespace {
 
-constexpr int kTileN = 128;       // weight rows per tile (UMMA M)
-constexpr int kTileM = 256;       // activation rows per tile (UMMA N)
+using namespace umma;
+
 constexpr int kTileK = 64;        // k per stage (128 bytes of bf16: one swizzle atom)
 constexpr int kXStages = 5;  // activation-tile ring (TMA from L2/HBM)
 constexpr int kAStages = 3;  // decoded weight-tile ring in TMEM (written by the producer warps)
@@ -44,15 +45,12 @@ constexpr int kBBytes = kTileM * kTileK * 2;  // 32 KB: activation tile (operand
 constexpr int kWBytes = kTileN * kTileK / 2;  // 4 KB: packed codes of the weight tile
 constexpr int kSBytes = kTileN * 16;          // 2 KB: 16-byte scale chunk per weight row
 constexpr int kRingBytes = kXStages * kBBytes + kWStages * (kWBytes + kSBytes);  // A lives in TMEM
-constexpr int kAccCols = kTileM;              // fp32 columns per accumulator
 constexpr int kTmemCols = 512;               // accumulator (256 columns) + 3 A stages of 32 columns
 constexpr int kThreads = 15 * 32;
-constexpr int kEpiWarps = 4;
 constexpr int kProdWarp0 = 4;                 // producers: warps 4..11
 constexpr int kTmaWarp = 12;                  // activation tiles
 constexpr int kMmaWarp = 13;
 constexpr int kTmaWWarp = 14;                 // packed codes and scales
-constexpr int kStageOutBytes = 32 * 32 * 2;    // per epilogue warp: 32 rows x 32 columns of bf16
 constexpr size_t kSmemBytes = (size_t)kRingBytes + kEpiWarps * kStageOutBytes + 1024 /*align*/ +
                               2048 /*barriers, lut*/;
 
@@ -70,75 +68,6 @@ struct Smem {  // placed after the 1024-aligned stage buffers
   float unit_lut[256];
 };
 
-// ------------------------------------------------------------------ tcgen05 / TMA wrappers
-
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
-  // K-major, 128-byte swizzle: rows of 128 B, 8-row groups 1024 B apart
-  uint64_t d = 0;
-  d |= (uint64_t)((addr >> 4) & 0x3fffu);          // start address
-  d |= (uint64_t)1 << 16;                          // leading byte offset (unused for swizzled K-major)
-  d |= (uint64_t)(1024 >> 4) << 32;                // stride byte offset: next 8-row group
-  d |= (uint64_t)1 << 46;                          // descriptor version (Blackwell)
-  d |= (uint64_t)2 << 61;                          // layout: SWIZZLE_128B
-  return d;
-}
-
-// kind::f16 instruction descriptor: bf16 A and B, fp32 D, both K-major
-__host__ __device__ constexpr uint32_t instr_desc(int m, int n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
-                                          uint32_t acc) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(acc)
-      : "memory");
-}
-
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
-          "r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// 32 lanes x 32 consecutive fp32 columns (one register per column) of this warp's subpartition.
-// The load and its wait are one asm statement: the registers are defined only once the wait has
-// returned, so no use of them can be scheduled in between.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
-      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
-        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
-        "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
-        "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-      : "r"(taddr)
-      : "memory");
-}
-
-__device__ __forceinline__ bool aborted(Smem* sm) { return *(volatile int*)&sm->abort != 0; }
-
-// bounded wait; on failure mark the CTA aborted so every role leaves its loop
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Smem* sm, unsigned* err) {
-  if (aborted(sm)) return false;
-  if (mbar_wait_bounded(bar, parity, err)) return true;
-  *(volatile int*)&sm->abort = 1;
-  return false;
-}
-
 // ------------------------------------------------------------------ kernel
 
 #ifdef NF4_TRACE  // diagnostics build only: per-CTA wall-clock stamps of pipeline milestones
@@ -147,24 +76,6 @@ __device__ unsigned long long g_trace[1024 * 16];
 #else
 #define NF4_STAMP(slot) ((void)0)
 #endif
-
-// Work unit u = tile * splits + split: the split takes k stages
-// [split * kps, (split + 1) * kps).  With splits > 1 the epilogue writes an
-// fp32 partial tile to the workspace; once every split of the tile has written
-// its partial (a counter per tile; the launch holds all units at once), split s
-// adds the partials of 32-row chunks s, s + splits, ... in split order
-// (deterministic) and writes those bf16 rows of Y.  Each split then arrives a
-// second time; the last of those resets the counter, so the workspace is left
-// ready for the next call.
-struct Work {
-  int ntiles_m, units, splits, kps;
-  __device__ int tile(int u) const { return u / splits; }
-  __device__ int split(int u) const { return u % splits; }
-  __device__ int n0(int u) const { return (tile(u) / ntiles_m) * kTileN; }
-  __device__ int m0(int u) const { return (tile(u) % ntiles_m) * kTileM; }
-};
-
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory"); }
 
 template <bool kDQ, bool kScaleTma>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -364,118 +275,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < kEpiWarps) {
     // ------------------------------------------------ epilogue: TMEM -> Y (or fp32 partials)
+    const EpiOut o{y, rows, m_total, part, tile_count, err};
     uint32_t ucount = 0;
     for (int u = blockIdx.x; u < wk.units; u += gridDim.x, ++ucount) {
       const int acc = 0;
       if (!wait_or_abort(&sm->acc_full[acc], ucount & 1, sm, err)) break;
       tc_fence_after();
       if (threadIdx.x == 0) NF4_STAMP(4);
-      const int nl = warp * 32 + lane;  // weight row within the tile
-      const int64_t n = (int64_t)wk.n0(u) + nl;
-      const int m0 = wk.m0(u);
       const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + acc * kAccCols;
-      uint16_t* st = out_stage + warp * (32 * 32);  // this warp's [32 m][32 n] bf16 tile
-      // Y rows m0 + c*32 + r, columns n0 + warp*32 .. +31: the warp's 32x32 block goes
-      // through shared memory so each lane stores 16 contiguous bytes of a Y row
-      auto store_block = [&](int c) {
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int piece = lane + 32 * i;  // 128 pieces of 8 bf16
-          const int r = piece >> 2, q = piece & 3;
-          const int m = m0 + c * 32 + r;
-          const uint4 v = *reinterpret_cast<const uint4*>(st + r * 32 + q * 8);
-          if (m < m_total)
-            *reinterpret_cast<uint4*>(y + (int64_t)m * rows + (n - lane) + q * 8) = v;
-        }
-        __syncwarp();
-      };
-      if (wk.splits == 1) {
-#pragma unroll 1
-        for (int c = 0; c < kTileM / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(taddr + c * 32, v);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) st[j * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
-          store_block(c);
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm->acc_empty[acc]);
-      } else {
-        // fp32 partial tile of this unit, laid out [m/4][n_local][4]: each 16-byte
-        // access of a warp covers 32 consecutive n (512 contiguous bytes)
-        float* mine = part + (size_t)u * (kTileN * kTileM);
-#pragma unroll 1
-        for (int c = 0; c < kTileM / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(taddr + c * 32, v);
-#pragma unroll
-          for (int j = 0; j < 32; j += 4)
-            __stcg(reinterpret_cast<float4*>(mine + ((size_t)((c * 32 + j) / 4) * kTileN + nl) * 4),
-                   make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
-                               __uint_as_float(v[j + 3])));
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm->acc_empty[acc]);  // TMEM no longer needed
-        __threadfence();
-        epi_bar();
-        // every split of the tile waits for all partials (the splits of a tile are co-resident: the
-        // grid holds every unit at once), then finishes its share of the 32-row chunks
-        if (threadIdx.x == 0) {
-          atomicAdd(&tile_count[wk.tile(u)], 1u);
-          const unsigned long long t0 = global_ns();
-          while (*(volatile unsigned*)&tile_count[wk.tile(u)] < (unsigned)wk.splits) {
-            if (global_ns() - t0 > kWaitLimitNs) {
-              atomicOr(err, kErrTimeout);
-              *(volatile int*)&sm->abort = 1;
-              break;
-            }
-            __nanosleep(64);
-          }
-          // second arrival: the split that completes 2 * splits has seen every split pass the wait
-          // above, so it can reset the counter for the next call
-          if (!aborted(sm) && atomicAdd(&tile_count[wk.tile(u)], 1u) == 2u * (unsigned)wk.splits - 1u)
-            tile_count[wk.tile(u)] = 0;
-        }
-        epi_bar();
-        if (threadIdx.x == 0) NF4_STAMP(5);
-        if (!aborted(sm)) {
-          __threadfence();
-          const float* tp = part + (size_t)wk.tile(u) * wk.splits * (kTileN * kTileM);
-#pragma unroll 1
-          for (int c = wk.split(u); c < kTileM / 32; c += wk.splits) {
-            float4 acc4[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              acc4[j] = __ldcg(reinterpret_cast<const float4*>(tp + ((size_t)(c * 8 + j) * kTileN + nl) * 4));
-            for (int sp = 1; sp < wk.splits; ++sp) {  // partials added in split order
-              const float* q = tp + (size_t)sp * (kTileN * kTileM);
-              float4 t[8];
-#pragma unroll
-              for (int j = 0; j < 8; ++j)
-                t[j] = __ldcg(reinterpret_cast<const float4*>(q + ((size_t)(c * 8 + j) * kTileN + nl) * 4));
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                acc4[j].x += t[j].x;
-                acc4[j].y += t[j].y;
-                acc4[j].z += t[j].z;
-                acc4[j].w += t[j].w;
-              }
-            }
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              st[(4 * j + 0) * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(acc4[j].x));
-              st[(4 * j + 1) * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(acc4[j].y));
-              st[(4 * j + 2) * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(acc4[j].z));
-              st[(4 * j + 3) * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(acc4[j].w));
-            }
-            store_block(c);
-          }
-          if (threadIdx.x == 0) NF4_STAMP(6);
-        }
-      }
+      epilogue_unit(wk, u, taddr, out_stage, sm, &sm->acc_empty[acc], o);
+      if (threadIdx.x == 0) NF4_STAMP(6);
     }
   }
 
@@ -506,38 +315,15 @@ EncodeTiled get_encoder() {
   return fn;
 }
 
-// Splits of K: enough work units to cover the SMs when there are few output
-// tiles; the split count divides the number of k stages and leaves each split
-// at least 8 stages.
 int gemm_splits(int64_t rows, int64_t cols, int64_t m, int num_sms) {
-  if (m <= 64) return 1;
-  const int64_t ntiles = (rows / kTileN) * ((m + kTileM - 1) / kTileM);
-  const int64_t kst = cols / kTileK;
-  int best = 1;
-  for (int sp = 2; sp <= 8; ++sp)
-    if (kst % sp == 0 && kst / sp >= 8 && ntiles * sp <= num_sms) best = sp;
-  return best;
-}
-
-int sm_count() {
-  int dev = 0, n = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n;
+  if (m <= 64) return 1;  // served by the GEMV
+  return reduction_splits((rows / kTileN) * ((m + kTileM - 1) / kTileM), cols / kTileK, num_sms);
 }
 
 }  // namespace
 
-size_t gemm_workspace_bytes(int64_t rows, int64_t cols, int64_t m) {
-  const int sp = gemm_splits(rows, cols, m, sm_count());
-  if (sp == 1) return 0;
-  const int64_t ntiles = (rows / kTileN) * ((m + kTileM - 1) / kTileM);
-  const size_t counters = ((size_t)ntiles * 4 + 255) & ~(size_t)255;
-  return counters + (size_t)ntiles * sp * kTileN * kTileM * sizeof(float);
-}
+namespace umma {
 
-namespace {
-
-// 2-D tiled tensor map (no swizzle unless asked); false if the driver refuses it
 bool make_map(CUtensorMap* map, CUtensorMapDataType type, size_t esize, const void* base, uint64_t inner,
               uint64_t outer, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
   EncodeTiled encode = get_encoder();
@@ -549,6 +335,34 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType type, size_t esize, const vo
   return encode(map, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+int reduction_splits(int64_t ntiles, int64_t stages, int num_sms) {
+  int best = 1;
+  for (int sp = 2; sp <= 8; ++sp)
+    if (stages % sp == 0 && stages / sp >= 8 && ntiles * sp <= num_sms) best = sp;
+  return best;
+}
+
+size_t split_workspace_bytes(int64_t ntiles, int splits) {
+  if (splits == 1) return 0;
+  const size_t counters = ((size_t)ntiles * 4 + 255) & ~(size_t)255;
+  return counters + (size_t)ntiles * splits * kTileN * kTileM * sizeof(float);
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+}  // namespace umma
+
+size_t gemm_workspace_bytes(int64_t rows, int64_t cols, int64_t m) {
+  const int sp = gemm_splits(rows, cols, m, sm_count());
+  return split_workspace_bytes((rows / kTileN) * ((m + kTileM - 1) / kTileM), sp);
+}
+
+namespace {
 
 template <bool kDQ, bool kScaleTma>
 cudaError_t launch_variant(const Scales& s, int rows, int cols, int m, int splits, const CUtensorMap& xmap,

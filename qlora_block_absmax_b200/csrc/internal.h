@@ -60,6 +60,11 @@ size_t gemm_workspace_bytes(int64_t rows, int64_t cols, int64_t m);
 cudaError_t launch_gemm(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x,
                         int64_t m, void* y, void* workspace, unsigned* err, cudaStream_t stream, int num_sms);
 
+// input gradient dX = dY . Wc (rows % 64 == 0, cols % 128 == 0)
+size_t gemm_dx_workspace_bytes(int64_t rows, int64_t cols, int64_t m);
+cudaError_t launch_gemm_dx(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* dy,
+                           int64_t m, void* dx, void* workspace, unsigned* err, cudaStream_t stream, int num_sms);
+
 // failure-path self-test: a bounded wait that runs out (see selftest.cu)
 cudaError_t launch_wait_timeout(unsigned* err, cudaStream_t stream);
 

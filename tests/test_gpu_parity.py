@@ -383,6 +383,111 @@ def test_gemm_scale_paths(cols, use_dq):
     check_matmul(y, oracle.matmul(p_ref, a_ref, rows, cols, x), f"gemm cols{cols} dq{use_dq}")
 
 
+# --------------------------------------------------------------------------- input gradient dX = dY . Wc
+
+def check_dx_sampled(dx: torch.Tensor, p_ref, a_ref, rows, cols, dy, seed, count=2048):
+    """`count` sampled outputs against the oracle (rms floor from the first full row), plus row 0 in full"""
+    m = dy.shape[0]
+    r = synth.rng(seed)
+    bs, ks = r.integers(0, m, count), r.integers(0, cols, count)
+    ref = oracle.matmul_dx_sampled(p_ref, a_ref, rows, cols, dy, bs, ks)
+    full_row = oracle.matmul_dx(p_ref, a_ref, rows, cols, dy[:1])
+    rms = np.sqrt(np.mean(full_row ** 2))
+    got = dx.float().cpu().numpy().astype(np.float64)[bs, ks]
+    bad = np.abs(got - ref) > REL_TOL * np.maximum(np.abs(ref), FLOOR * rms)
+    assert not bad.any(), f"{bad.sum()} of {count} sampled dx outputs beyond tolerance"
+    check_matmul(dx[:1], full_row, "dx row 0")
+
+
+@pytest.mark.parametrize("m", [1, 16, 100, 256, 300])
+def test_gemm_dx_small(m):
+    rows, cols = 256, 512
+    qw, p_ref, a_ref = quantized_pair(rows, cols, 81 + m, True)
+    dy = synth.activations((m, rows), 82 + m)
+    dx = nf4.gemm_dx(qw, dev_bf16(dy))
+    assert dx.shape == (m, cols)
+    check_matmul(dx, oracle.matmul_dx(p_ref, a_ref, rows, cols, dy), f"gemm_dx m{m}")
+
+
+def test_gemm_dx_one_hot_rows_bit_exact():
+    """one-hot gradient rows read weight rows back: dX = bf16_rn(code * a^) of that row, bit for bit
+    (a single nonzero product per output, so the fp32 sum and the bf16 rounding are exact); covers
+    weight rows in every 16-row MMA step and 8-row swizzle group of a stage, and both column halves"""
+    rows, cols = 192, 384
+    qw, p_ref, a_ref = quantized_pair(rows, cols, 5, True)
+    wc = oracle.dequantize(p_ref, a_ref, rows * cols, 64, "bf16").reshape(rows, cols)
+    ns = [0, 1, 7, 8, 15, 16, 31, 47, 63, 64, 100, 127, 128, 150, 190, 191]
+    dy = synth.f32_to_bf16_bits(np.eye(rows, dtype=np.float32)[ns])
+    dx = nf4.gemm_dx(qw, dev_bf16(dy))
+    assert np.array_equal(host_bf16_bits(dx), wc[ns])
+
+
+@pytest.mark.parametrize("cols", [384, 1024, 4096])
+@pytest.mark.parametrize("use_dq,code", [(False, "e4m3"), (True, "e4m3"), (True, "int8")])
+def test_gemm_dx_scale_paths(cols, use_dq, code):
+    """plain fp32 and double-quantized scales; scale rows that are (1024, 4096) and are not (384) whole
+    16-byte units (TMA chunks vs per-block loads)"""
+    rows, m = 128, 160
+    qw, p_ref, a_ref = quantized_pair(rows, cols, 91 + cols, use_dq, code)
+    dy = synth.activations((m, rows), 92 + cols)
+    dx = nf4.gemm_dx(qw, dev_bf16(dy))
+    check_matmul(dx, oracle.matmul_dx(p_ref, a_ref, rows, cols, dy), f"gemm_dx cols{cols} dq{use_dq} {code}")
+
+
+@pytest.mark.parametrize("m", [65, 256, 300])
+def test_gemm_dx_split_k(m):
+    """few output tiles: the reduction over weight rows is split across CTAs"""
+    rows, cols = 2048, 256
+    qw, p_ref, a_ref = quantized_pair(rows, cols, 95 + m, True)
+    assert nf4.gemm_dx_workspace_bytes(qw, m) > 0
+    dy = synth.activations((m, rows), 96 + m)
+    dx = nf4.gemm_dx(qw, dev_bf16(dy))
+    check_matmul(dx, oracle.matmul_dx(p_ref, a_ref, rows, cols, dy), f"gemm_dx split m{m}")
+
+
+@pytest.mark.parametrize("shape", [(14336, 4096), (4096, 14336), (4096, 4096)])
+@pytest.mark.parametrize("m", [256, 1024, 4096])
+def test_gemm_dx_llama_shapes_sampled(shape, m):
+    """dX for the 8B-shaped projections (gate/up 14336x4096, down 4096x14336, 4096^2) at the prefill
+    token counts: 2048 sampled outputs and all of row 0 against the oracle"""
+    rows, cols = shape
+    qw, p_ref, a_ref = quantized_pair(rows, cols, 1030 + rows // 1024, True)
+    dy = synth.activations((m, rows), 1031 + m)
+    dx = nf4.gemm_dx(qw, dev_bf16(dy))
+    check_dx_sampled(dx, p_ref, a_ref, rows, cols, dy, 11 + m)
+    nf4.check_device_error()
+
+
+@pytest.mark.parametrize("rows,cols,m", [(14336, 4096, 1024), (4096, 4096, 256), (4096, 14336, 4096)])
+def test_gemm_dx_repeatable(rows, cols, m):
+    """ten identical calls (persistent CTAs cycling their rings, both accumulators; split path at m=256)
+    give identical bits"""
+    w = synth.normal_weights((rows, cols), 2030)
+    qw = nf4.quantize_weight(dev(w))
+    dy = dev_bf16(synth.activations((m, rows), 2031))
+    ws = torch.zeros(max(nf4.gemm_dx_workspace_bytes(qw, m), 16), dtype=torch.uint8, device="cuda")
+    ref = nf4.gemm_dx(qw, dy, workspace=ws).view(torch.int16).clone()
+    for _ in range(10):
+        assert torch.equal(nf4.gemm_dx(qw, dy, workspace=ws).view(torch.int16), ref)
+    nf4.check_device_error()
+
+
+def test_gemm_dx_adjoint_of_gemm():
+    """<dY, X . Wc^T> = <dY . Wc, X> between the library's own forward and gradient products at a full
+    prefill size (only bf16 output rounding separates the two sides)"""
+    rows, cols, m = 4096, 4096, 512
+    w = synth.normal_weights((rows, cols), 2040)
+    qw = nf4.quantize_weight(dev(w))
+    x = dev_bf16(synth.activations((m, cols), 2041))
+    dy = dev_bf16(synth.activations((m, rows), 2042))
+    t1 = dy.double() * nf4.gemm(qw, x).double()
+    t2 = nf4.gemm_dx(qw, dy).double() * x.double()
+    # each output carries at most half a bf16 ulp (2^-9 relative) of independent rounding: the sums differ
+    # by a random walk of those, bounded here at 8 standard deviations
+    scale = float(torch.sqrt((t1 ** 2).sum() + (t2 ** 2).sum()))
+    assert abs(float(t1.sum()) - float(t2.sum())) <= 2.0 ** -6 * scale
+
+
 # --------------------------------------------------------------------------- whole model (config 5)
 
 def test_whole_model_8b_config5():
