@@ -34,6 +34,7 @@ ROWS, COLS, GEMV_B, GEMM_M = 4096, 4096, 1, 256
 WORKLOAD = "nf4_path_bf16_4096x4096_outliers_gemv1_gemm256"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNELS = ("quantize", "double_quant", "dequantize", "gemv", "gemm")
+NEXT_KERNELS = ("gemm_dx",)  # timed beside the step, not part of it
 
 
 def work_per_step(rows=ROWS, cols=COLS, b=GEMV_B, m=GEMM_M):
@@ -49,6 +50,8 @@ def work_per_step(rows=ROWS, cols=COLS, b=GEMV_B, m=GEMM_M):
         "dequantize": {"bytes": w4 + 2 * n},
         "gemv": {"bytes": w4 + 2 * b * cols + 2 * b * rows, "flops": 2 * b * n},
         "gemm": {"bytes": w4 + 2 * m * cols + 2 * m * rows, "flops": 2 * m * n},
+        "gemm_dx": {"bytes": w4 + 2 * m * rows + 2 * m * cols, "flops": 2 * m * n,
+                    "what": f"dX[{m},{cols}] = dY[{m},{rows}] . Wc (input gradient)"},
     }
 
 
@@ -121,7 +124,7 @@ def oracle_sample_step(sample_rows: int, w_bits, x_bits, X_bits):
     oracle.matmul(p, ah, sample_rows, COLS, X_bits)
     dt = time.perf_counter() - t0
     work = work_per_step(rows=sample_rows)
-    return dt, sum(v["bytes"] for v in work.values())
+    return dt, sum(work[k]["bytes"] for k in KERNELS)
 
 
 def cpu_baseline(sample_rows: int, reps: int = 1):
@@ -182,9 +185,11 @@ def run_ours(args):
     w_bits = synth.config2_weight()
     x_bits = synth.activations((GEMV_B, COLS), 1013)
     X_bits = synth.activations((GEMM_M, COLS), 1277)
+    dY_bits = synth.activations((GEMM_M, ROWS), 1279)  # gradient of Y for the input-gradient product
     host_w = torch.from_numpy(w_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
     host_x = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
     host_X = torch.from_numpy(X_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    host_dY = torch.from_numpy(dY_bits.view(np.int16)).view(torch.bfloat16)
     n = ROWS * COLS
     nb = n // 64
     per_copy = 2 * n + n // 2 + 4 * nb + nb + 2 * n + 2 * GEMM_M * (ROWS + COLS)
@@ -212,6 +217,9 @@ def run_ours(args):
         c.qw = nf4.QuantizedWeight(packed=c.packed, rows=ROWS, cols=COLS, absmax_q=c.q, absmax_scale=c.scale,
                                    absmax_mean=c.mean, dq_code=nf4.NF4_DQ_E4M3)
         c.gws = torch.zeros(max(nf4.gemm_workspace_bytes(c.qw, GEMM_M), 16), dtype=torch.uint8, device=dev)
+        c.dY = host_dY.to(dev)
+        c.dX = torch.empty(GEMM_M, COLS, dtype=torch.bfloat16, device=dev)
+        c.dws = torch.zeros(max(nf4.gemm_dx_workspace_bytes(c.qw, GEMM_M), 16), dtype=torch.uint8, device=dev)
         cs.append(c)
     stream = torch.cuda.current_stream()
 
@@ -222,6 +230,10 @@ def run_ours(args):
                 lambda: nf4.dequantize(c.qw, torch.bfloat16, out=c.deq),
                 lambda: nf4.gemv(c.qw, c.x, out=c.y),
                 lambda: nf4.gemm(c.qw, c.X, out=c.Y, workspace=c.gws))
+
+    def next_calls(c):
+        """products beyond the step's five calls, timed on their own: the input gradient dX = dY . Wc"""
+        return (lambda: nf4.gemm_dx(c.qw, c.dY, out=c.dX, workspace=c.dws),)
 
     def step(c):
         for f in calls(c):
@@ -246,11 +258,11 @@ def run_ours(args):
     # The device-timed region is one CUDA graph holding the K steps (the library
     # launches are chained with programmatic dependent launch), so host-side
     # marshalling cannot gap the GPU timeline.
-    def capture(nsteps, only=None):
+    def capture(nsteps, only=None, fn=calls):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             for i in range(nsteps):
-                fs = calls(cs[i % copies])
+                fs = fn(cs[i % copies])
                 for f in (fs if only is None else (fs[only],)):
                     f()
         return g
@@ -260,8 +272,9 @@ def run_ours(args):
     # per-kernel times: one graph per library call holding its K launches on the
     # same rotating inputs, timed as a whole (no event nodes between launches)
     g_kernel = [capture(args.steps, j) for j in range(len(KERNELS))]
+    g_next = [capture(args.steps, j, next_calls) for j in range(len(NEXT_KERNELS))]
     g_warm.replay()
-    for g in g_kernel:
+    for g in g_kernel + g_next:
         g.replay()
     nf4.check_device_error()
     barrier()
@@ -287,9 +300,18 @@ def run_ours(args):
         k1.record(stream)
         barrier()
         per_kernel_ms[k] = max_ms(k0.elapsed_time(k1))
+    next_ms = {}
+    for j, k in enumerate(NEXT_KERNELS):
+        k0 = torch.cuda.Event(enable_timing=True)
+        k1 = torch.cuda.Event(enable_timing=True)
+        k0.record(stream)
+        g_next[j].replay()
+        k1.record(stream)
+        barrier()
+        next_ms[k] = max_ms(k0.elapsed_time(k1))
     clocks = sampler.stop()
     nf4.check_device_error()
-    del g_warm, g_timed, g_kernel
+    del g_warm, g_timed, g_kernel, g_next
 
     # ---- end to end through the public API with host buffers
     host_out = {"packed": torch.empty(n // 2, dtype=torch.uint8).pin_memory(),
@@ -348,7 +370,7 @@ def run_ours(args):
     e2e_ms = max_ms(e0.elapsed_time(e1))
 
     work = work_per_step()
-    step_bytes = sum(v["bytes"] for v in work.values())
+    step_bytes = sum(work[k]["bytes"] for k in KERNELS)
     ms_per_step = elapsed_ms / args.steps
     value = replica_throughput(step_bytes, args.steps, elapsed_ms, world)
     e2e_value = replica_throughput(step_bytes, args.steps, e2e_ms, world)
@@ -366,6 +388,15 @@ def run_ours(args):
         if "elems" in work[k]:
             d["gelem_s"] = round(work[k]["elems"] / t / 1e9, 2)
         breakdown[k] = d
+    nexts = {}
+    for k in NEXT_KERNELS:
+        t = next_ms[k] / args.steps * 1e-3
+        ach = work[k]["flops"] / t / 1e12
+        nexts[k] = {"what": work[k]["what"], "ms": round(t * 1e3, 5), "gbs": round(work[k]["bytes"] / t / 1e9, 1),
+                    "tflops": round(ach, 2), "roofline": {"bound": "tensor", "achieved": round(ach, 2),
+                                                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                                          "frac": round(ach / peaks["bf16_tflops"], 4),
+                                                          "traffic": TRAFFIC.get(k)}}
     dom = max(KERNELS, key=lambda k: per_kernel_ms[k])
     t_dom = per_kernel_ms[dom] / args.steps * 1e-3
     if dom == "gemm":
@@ -391,6 +422,7 @@ def run_ours(args):
                    "parallelism": "replicas" if world > 1 else "single"},
         "roofline": roof,
         "breakdown": breakdown,
+        "next": nexts,
         "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": int(launches),
         "launch": ("the K timed steps captured in one CUDA graph, launches chained with programmatic dependent "
@@ -410,9 +442,11 @@ def run_ours(args):
 
 
 # ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of each kernel at this workload, from the
-# --set full capture in profiles/kernels_nf4_path_bf16_4096x4096.md; an entry is removed whenever its kernel
-# changes after the capture
-TRAFFIC = {"quantize": 33576192, "double_quant": 1084928, "dequantize": 8679680, "gemm": 10812672}
+# --set full captures in profiles/kernels_nf4_path_bf16_4096x4096.md (quantize, double quant, dequantize) and
+# profiles/kernels_gemm_dx_and_gemm_bf16_4096x4096_m256.md (gemm, gemm_dx); an entry is removed whenever its
+# kernel changes after the capture
+TRAFFIC = {"quantize": 33576192, "double_quant": 1084928, "dequantize": 8679680, "gemm": 10811904,
+           "gemm_dx": 10812672}
 
 
 def run_reference(args):
