@@ -338,7 +338,7 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType type, size_t esize, const vo
 
 int reduction_splits(int64_t ntiles, int64_t stages, int num_sms) {
   int best = 1;
-  for (int sp = 2; sp <= 8; ++sp)
+  for (int sp = 2; sp <= kMaxSplits; ++sp)
     if (stages % sp == 0 && stages / sp >= 8 && ntiles * sp <= num_sms) best = sp;
   return best;
 }

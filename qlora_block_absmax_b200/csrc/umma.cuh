@@ -20,6 +20,7 @@ constexpr int kTileM = 256;  // activation rows per tile (UMMA N, fp32 TMEM colu
 constexpr int kAccCols = kTileM;
 constexpr int kEpiWarps = 4;                  // warps 0..3 read TMEM lanes 32w..32w+31
 constexpr int kStageOutBytes = 32 * 32 * 2;   // per epilogue warp: 32 rows x 32 columns of bf16
+constexpr int kMaxSplits = 4;                 // reduction splits of one output tile (reduction_splits)
 
 // ------------------------------------------------------------------ descriptors
 
@@ -194,11 +195,14 @@ __device__ __forceinline__ void epilogue_unit(const Work& wk, int u, uint32_t ta
     if (lane == 0) mbar_arrive(acc_empty);
     return;
   }
-  // fp32 partial tile of this unit, laid out [m/4][n_local][4]: each 16-byte
-  // access of a warp covers 32 consecutive n (512 contiguous bytes)
+  // Split reduction.  The fp32 partial of this unit goes to the workspace laid out [m/4][n_local][4] (each
+  // 16-byte access of a warp covers 32 consecutive n, 512 contiguous bytes), except the 32-row chunks this
+  // split reduces itself (c = split, split + splits, ...): those stay in TMEM until the reduction.
+  const int my = wk.split(u);
   float* mine = o.part + (size_t)u * (kTileN * kTileM);
 #pragma unroll 1
   for (int c = 0; c < kTileM / 32; ++c) {
+    if (c % wk.splits == my) continue;
     uint32_t v[32];
     tmem_ld32(taddr + c * 32, v);
 #pragma unroll
@@ -207,9 +211,6 @@ __device__ __forceinline__ void epilogue_unit(const Work& wk, int u, uint32_t ta
              make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
                          __uint_as_float(v[j + 3])));
   }
-  tc_fence_before();
-  __syncwarp();
-  if (lane == 0) mbar_arrive(acc_empty);  // TMEM no longer needed
   __threadfence();
   epi_bar();
   // every split of the tile waits for all partials (the splits of a tile are co-resident: the
@@ -231,38 +232,67 @@ __device__ __forceinline__ void epilogue_unit(const Work& wk, int u, uint32_t ta
       o.tile_count[wk.tile(u)] = 0;
   }
   epi_bar();
-  if (aborted(sm)) return;
-  __threadfence();
-  const float* tp = o.part + (size_t)wk.tile(u) * wk.splits * (kTileN * kTileM);
+  if (!aborted(sm)) {
+    __threadfence();
+    const float* tp = o.part + (size_t)wk.tile(u) * wk.splits * (kTileN * kTileM);
 #pragma unroll 1
-  for (int c = wk.split(u); c < kTileM / 32; c += wk.splits) {
-    float4 acc4[8];
+    for (int c = my; c < kTileM / 32; c += wk.splits) {
+      uint32_t v[32];
+      tmem_ld32(taddr + c * 32, v);  // this split's own partial of the chunk
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      acc4[j] = __ldcg(reinterpret_cast<const float4*>(tp + ((size_t)(c * 8 + j) * kTileN + nl) * 4));
-    for (int sp = 1; sp < wk.splits; ++sp) {  // partials added in split order
-      const float* q = tp + (size_t)sp * (kTileN * kTileM);
-      float4 t[8];
+      for (int h = 0; h < 2; ++h) {  // 16 rows at a time: every other split's loads in flight together
+        float4 t[kMaxSplits - 1][4];
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        t[j] = __ldcg(reinterpret_cast<const float4*>(q + ((size_t)(c * 8 + j) * kTileN + nl) * 4));
+        for (int q = 0; q < kMaxSplits - 1; ++q) {
+          const int sp = q + (q >= my);
+          if (sp < wk.splits) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        acc4[j].x += t[j].x;
-        acc4[j].y += t[j].y;
-        acc4[j].z += t[j].z;
-        acc4[j].w += t[j].w;
+            for (int j = 0; j < 4; ++j)
+              t[q][j] = __ldcg(reinterpret_cast<const float4*>(
+                  tp + (size_t)sp * (kTileN * kTileM) + ((size_t)(c * 8 + h * 4 + j) * kTileN + nl) * 4));
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          // partials added in split order 0, 1, ..., splits - 1
+          float4 acc4 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int sp = 0; sp < kMaxSplits; ++sp) {
+            if (sp >= wk.splits) break;
+            // split sp's partial: this split's own (TMEM) or the loads of slot sp (sp < my) / sp - 1 (sp > my);
+            // every array index below is a compile-time constant
+            float4 val;
+            if (sp == my) {
+              const int r = (h * 4 + j) * 4;
+              val = make_float4(__uint_as_float(v[r]), __uint_as_float(v[r + 1]), __uint_as_float(v[r + 2]),
+                                __uint_as_float(v[r + 3]));
+            } else if (sp < my) {
+              val = t[sp < kMaxSplits - 1 ? sp : kMaxSplits - 2][j];
+            } else {
+              val = t[sp > 0 ? sp - 1 : 0][j];
+            }
+            if (sp == 0) {
+              acc4 = val;
+            } else {
+              acc4.x += val.x;
+              acc4.y += val.y;
+              acc4.z += val.z;
+              acc4.w += val.w;
+            }
+          }
+          const int r = (h * 4 + j) * 4;  // row within the chunk
+          st[(r + 0) * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(acc4.x));
+          st[(r + 1) * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(acc4.y));
+          st[(r + 2) * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(acc4.z));
+          st[(r + 3) * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(acc4.w));
+        }
       }
+      store_block(c);
     }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      st[(4 * j + 0) * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(acc4[j].x));
-      st[(4 * j + 1) * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(acc4[j].y));
-      st[(4 * j + 2) * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(acc4[j].z));
-      st[(4 * j + 3) * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(acc4[j].w));
-    }
-    store_block(c);
   }
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(acc_empty);  // TMEM no longer needed
 }
 
 // ------------------------------------------------------------------ host side
