@@ -71,6 +71,8 @@ def _load():
         "oracle_nf4_matmul_sampled": (None, [P, P, I64, I64, I32, P, I64, P, P, I64, P]),
         "oracle_nf4_matmul_dx": (None, [P, P, I64, I64, I32, P, I64, P]),
         "oracle_nf4_matmul_dx_sampled": (None, [P, P, I64, I64, I32, P, I64, P, P, I64, P]),
+        "oracle_lora_down": (None, [P, I64, I64, P, I32, ctypes.c_float, P]),
+        "oracle_nf4_matmul_lora": (None, [P, P, I64, I64, I32, P, I64, P, P, I32, ctypes.c_float, P]),
         "oracle_set_threads": (None, [ctypes.c_int]),
         "oracle_get_threads": (ctypes.c_int, []),
     }
@@ -237,3 +239,25 @@ def matmul_dx_sampled(packed: np.ndarray, absmax: np.ndarray, N: int, K: int, dy
                                          _p(np.ascontiguousarray(absmax, dtype=np.float32)),
                                          N, K, blocksize, _p(dy), dy.shape[0], _p(bs), _p(ks), bs.size, _p(dx))
     return dx
+
+
+def lora_down(x_bf16: np.ndarray, K: int, A_bf16: np.ndarray, r: int, scale: float) -> np.ndarray:
+    """bf16 bits t [B, r] = bf16_rn(fp32(scale * x . A^T)) (fp64 sums)."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16).reshape(-1, K)
+    A = np.ascontiguousarray(A_bf16, dtype=np.uint16).reshape(r, K)
+    t = np.zeros((x.shape[0], r), np.uint16)
+    _load().oracle_lora_down(_p(x), x.shape[0], K, _p(A), r, float(scale), _p(t))
+    return t
+
+
+def matmul_lora(packed: np.ndarray, absmax: np.ndarray, N: int, K: int, x_bf16: np.ndarray, A_bf16: np.ndarray,
+                B_bf16: np.ndarray, r: int, scale: float, blocksize: int = 64) -> np.ndarray:
+    """fp64 y [B, N] = x . Wc^T + t . B^T with t = lora_down(x)."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16).reshape(-1, K)
+    A = np.ascontiguousarray(A_bf16, dtype=np.uint16).reshape(r, K)
+    Bu = np.ascontiguousarray(B_bf16, dtype=np.uint16).reshape(N, r)
+    y = np.zeros((x.shape[0], N), np.float64)
+    _load().oracle_nf4_matmul_lora(_p(np.ascontiguousarray(packed, dtype=np.uint8)),
+                                   _p(np.ascontiguousarray(absmax, dtype=np.float32)), N, K, blocksize, _p(x),
+                                   x.shape[0], _p(A), _p(Bu), r, float(scale), _p(y))
+    return y

@@ -413,3 +413,63 @@ def test_matmul_dx_zero_codes_give_zero():
     p = np.full(N * K // 2, 0x77, np.uint8)
     a = np.ones(N * K // 64, np.float32)
     assert np.all(oracle.matmul_dx(p, a, N, K, synth.activations((2, N), 4)) == 0)
+
+
+# ---------------------------------------------------------------- low-rank adapter on the 4-bit matmul
+
+def _bf16(a):
+    return synth.f32_to_bf16_bits(np.asarray(a, dtype=np.float32))
+
+
+def test_lora_zero_adapter_is_the_plain_matmul():
+    """an all-zero up map, or scale 0, leaves exactly the 4-bit product"""
+    N, K, r = 64, 192, 16
+    p, a = oracle.quantize(synth.normal_weights((N, K), 71), 64)
+    x = synth.activations((3, K), 72)
+    A = synth.activations((r, K), 73)
+    B = synth.activations((N, r), 74)
+    base = oracle.matmul(p, a, N, K, x)
+    assert np.array_equal(oracle.matmul_lora(p, a, N, K, x, A, np.zeros((N, r), np.uint16), r, 2.0), base)
+    assert np.array_equal(oracle.matmul_lora(p, a, N, K, x, A, B, r, 0.0), base)
+
+
+def test_lora_one_hot_down_map_on_zero_weight():
+    """zero-code weight (Wc = 0) and one-hot down-map rows A[j] = e_{k_j}: t = bf16(s * x[:, k_j]) (exact for
+    s = 2) and y = t . B^T, checked against a numpy product"""
+    N, K, r = 48, 128, 16
+    p = np.full(N * K // 2, 0x77, np.uint8)
+    a = np.ones(N * K // 64, np.float32)
+    ks = np.array([0, 1, 5, 63, 64, 65, 100, 127, 2, 3, 4, 6, 7, 8, 9, 10])
+    A = _bf16(np.eye(K, dtype=np.float32)[ks])
+    x = synth.activations((5, K), 75)
+    B = synth.activations((N, r), 76)
+    t = oracle.lora_down(x, K, A, r, 2.0)
+    xf = synth.bf16_bits_to_f32(x)
+    assert np.array_equal(synth.bf16_bits_to_f32(t), 2.0 * xf[:, ks])
+    y = oracle.matmul_lora(p, a, N, K, x, A, B, r, 2.0)
+    ref = (2.0 * xf[:, ks]).astype(np.float64) @ synth.bf16_bits_to_f32(B).astype(np.float64).T
+    assert np.allclose(y, ref, rtol=1e-13, atol=1e-13)
+
+
+def test_lora_down_matches_numpy_and_torch_rounding():
+    """t = bf16_rn(fp32(s * x . A^T)) against a numpy fp64 product and torch's bf16 cast"""
+    K, r = 320, 16
+    x = synth.activations((7, K), 77)
+    A = synth.activations((r, K), 78)
+    t = oracle.lora_down(x, K, A, r, 2.0)
+    prod = synth.bf16_bits_to_f32(x).astype(np.float64) @ synth.bf16_bits_to_f32(A).astype(np.float64).T
+    ref = torch.from_numpy((2.0 * prod).astype(np.float32)).bfloat16().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(t, ref)
+
+
+def test_lora_sum_of_parts():
+    """y = x . Wc^T + t . B^T term by term: the adapter part equals the zero-weight case"""
+    N, K, r = 64, 256, 16
+    p, a = oracle.quantize(synth.normal_weights((N, K), 79), 64)
+    x = synth.activations((4, K), 80)
+    A = synth.activations((r, K), 81)
+    B = synth.activations((N, r), 82)
+    y = oracle.matmul_lora(p, a, N, K, x, A, B, r, 2.0)
+    zero = np.full(N * K // 2, 0x77, np.uint8)
+    adapter = oracle.matmul_lora(zero, a, N, K, x, A, B, r, 2.0)
+    assert np.allclose(y, oracle.matmul(p, a, N, K, x) + adapter, rtol=1e-13, atol=1e-12)
