@@ -34,7 +34,8 @@ ROWS, COLS, GEMV_B, GEMM_M = 4096, 4096, 1, 256
 WORKLOAD = "nf4_path_bf16_4096x4096_outliers_gemv1_gemm256"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNELS = ("quantize", "double_quant", "dequantize", "gemv", "gemm")
-NEXT_KERNELS = ("gemm_dx",)  # timed beside the step, not part of it
+NEXT_KERNELS = ("gemm_dx", "gemm_lora")  # timed beside the step, not part of it
+LORA_R, LORA_ALPHA = 16, 32.0
 
 
 def work_per_step(rows=ROWS, cols=COLS, b=GEMV_B, m=GEMM_M):
@@ -52,6 +53,9 @@ def work_per_step(rows=ROWS, cols=COLS, b=GEMV_B, m=GEMM_M):
         "gemm": {"bytes": w4 + 2 * m * cols + 2 * m * rows, "flops": 2 * m * n},
         "gemm_dx": {"bytes": w4 + 2 * m * rows + 2 * m * cols, "flops": 2 * m * n,
                     "what": f"dX[{m},{cols}] = dY[{m},{rows}] . Wc (input gradient)"},
+        "gemm_lora": {"bytes": w4 + 2 * m * cols + 2 * m * rows + 2 * LORA_R * (rows + cols),
+                      "flops": 2 * m * n + 2 * m * LORA_R * (rows + cols),
+                      "what": f"Y[{m},{rows}] = X . Wc^T + 2 (X . A^T) . B^T, r = {LORA_R} (two launches)"},
     }
 
 
@@ -190,6 +194,13 @@ def run_ours(args):
     host_x = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
     host_X = torch.from_numpy(X_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
     host_dY = torch.from_numpy(dY_bits.view(np.int16)).view(torch.bfloat16)
+    # r = 16, lora_alpha = 32 adapter maps: down ~N(0, 1/cols), up ~N(0, 0.02) (seeds 1281, 1282)
+    host_down = torch.from_numpy(synth.f32_to_bf16_bits(
+        (synth.rng(1281).standard_normal((LORA_R, COLS)) / np.sqrt(COLS)).astype(np.float32)).view(np.int16)).view(
+        torch.bfloat16)
+    host_up = torch.from_numpy(synth.f32_to_bf16_bits(
+        (synth.rng(1282).standard_normal((ROWS, LORA_R)) * 0.02).astype(np.float32)).view(np.int16)).view(
+        torch.bfloat16)
     n = ROWS * COLS
     nb = n // 64
     per_copy = 2 * n + n // 2 + 4 * nb + nb + 2 * n + 2 * GEMM_M * (ROWS + COLS)
@@ -220,6 +231,9 @@ def run_ours(args):
         c.dY = host_dY.to(dev)
         c.dX = torch.empty(GEMM_M, COLS, dtype=torch.bfloat16, device=dev)
         c.dws = torch.zeros(max(nf4.gemm_dx_workspace_bytes(c.qw, GEMM_M), 16), dtype=torch.uint8, device=dev)
+        c.down, c.up = host_down.to(dev), host_up.to(dev)
+        c.Yl = torch.empty(GEMM_M, ROWS, dtype=torch.bfloat16, device=dev)
+        c.lws = torch.zeros(nf4.gemm_lora_workspace_bytes(c.qw, GEMM_M), dtype=torch.uint8, device=dev)
         cs.append(c)
     stream = torch.cuda.current_stream()
 
@@ -232,8 +246,10 @@ def run_ours(args):
                 lambda: nf4.gemm(c.qw, c.X, out=c.Y, workspace=c.gws))
 
     def next_calls(c):
-        """products beyond the step's five calls, timed on their own: the input gradient dX = dY . Wc"""
-        return (lambda: nf4.gemm_dx(c.qw, c.dY, out=c.dX, workspace=c.dws),)
+        """products beyond the step's five calls, timed on their own: the input gradient dX = dY . Wc and the
+        GEMM with an r = 16 adapter"""
+        return (lambda: nf4.gemm_dx(c.qw, c.dY, out=c.dX, workspace=c.dws),
+                lambda: nf4.gemm_lora(c.qw, c.X, c.down, c.up, LORA_ALPHA / LORA_R, out=c.Yl, workspace=c.lws))
 
     def step(c):
         for f in calls(c):

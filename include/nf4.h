@@ -172,6 +172,37 @@ NF4_API nf4_status nf4_gemm(const nf4_weight *w, const void *x, int64_t m, void 
                     size_t workspace_bytes, nf4_stream_t stream);
 NF4_API size_t nf4_gemm_workspace_bytes(const nf4_weight *w, int64_t m);
 
+/* A low-rank adapter on a frozen 4-bit weight, as QLoRA trains it ([bnb-tut]
+ * "QLoRA: Fine-Tuning a 4-bit Model"; [bnb-tools] "Fine-tuning with adapters
+ * on a 4-bit model": r = 16, lora_alpha = 32, scale = lora_alpha / r).
+ *   down   device bf16 [r, cols] (the adapter's first map, A), 16-byte aligned
+ *   up     device bf16 [rows, r] (the second map, B), 16-byte aligned
+ *   r      16 or 32;  scale  finite fp32 */
+typedef struct {
+  const void *down;
+  const void *up;
+  int32_t r;
+  float scale;
+} nf4_lora;
+
+/* nf4_gemm with the adapter added in the same accumulator:
+ *   v[m, j] = scale * sum_k X[m, k] * down[j, k]              (fp32 sum)
+ *   Y[m, n] = bf16_rn( sum_k Wc[n, k] * X[m, k] + sum_j v[m, j] * up[n, j] )
+ * v is not rounded to bf16: it reaches the tensor cores as a bf16 pair
+ * (hi = bf16_rn(v), lo = bf16_rn(v - hi); about 16 significant bits).  Two
+ * launches: the down map (v into the workspace), then the tcgen05 GEMM, which
+ * treats [hi | lo] as one more reduction stage of each output tile with
+ * [up | up] as that stage's weight.  Dropout is not applied.
+ *   x  device bf16 [m, cols];  y  device bf16 [m, rows];  m >= 1
+ *   cols % 64 == 0; rows % 128 == 0.
+ *   workspace  device scratch of nf4_gemm_lora_workspace_bytes(w, m) bytes,
+ *              16-byte aligned, never NULL for m >= 1: v, then the split
+ *              scratch under nf4_gemm's contract (zero-fill before the first
+ *              use, left ready by every completed call). */
+NF4_API nf4_status nf4_gemm_lora(const nf4_weight *w, const nf4_lora *lora, const void *x, int64_t m, void *y,
+                         void *workspace, size_t workspace_bytes, nf4_stream_t stream);
+NF4_API size_t nf4_gemm_lora_workspace_bytes(const nf4_weight *w, int64_t m);
+
 /* Input gradient of nf4_gemm, for training adapters on a frozen 4-bit base
  * ([bnb-tools] "Strengths and limitations": the quantized weights receive no
  * gradient, but the gradient flows through them to the adapters; [bnb-tut]

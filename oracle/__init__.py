@@ -73,6 +73,7 @@ def _load():
         "oracle_nf4_matmul_dx_sampled": (None, [P, P, I64, I64, I32, P, I64, P, P, I64, P]),
         "oracle_lora_down": (None, [P, I64, I64, P, I32, ctypes.c_float, P]),
         "oracle_nf4_matmul_lora": (None, [P, P, I64, I64, I32, P, I64, P, P, I32, ctypes.c_float, P]),
+        "oracle_nf4_matmul_lora_sampled": (None, [P, P, I64, I64, I32, P, P, P, I32, P, P, I64, P]),
         "oracle_set_threads": (None, [ctypes.c_int]),
         "oracle_get_threads": (ctypes.c_int, []),
     }
@@ -242,17 +243,17 @@ def matmul_dx_sampled(packed: np.ndarray, absmax: np.ndarray, N: int, K: int, dy
 
 
 def lora_down(x_bf16: np.ndarray, K: int, A_bf16: np.ndarray, r: int, scale: float) -> np.ndarray:
-    """bf16 bits t [B, r] = bf16_rn(fp32(scale * x . A^T)) (fp64 sums)."""
+    """fp64 t [B, r] = scale * x . A^T (not rounded)."""
     x = np.ascontiguousarray(x_bf16, dtype=np.uint16).reshape(-1, K)
     A = np.ascontiguousarray(A_bf16, dtype=np.uint16).reshape(r, K)
-    t = np.zeros((x.shape[0], r), np.uint16)
+    t = np.zeros((x.shape[0], r), np.float64)
     _load().oracle_lora_down(_p(x), x.shape[0], K, _p(A), r, float(scale), _p(t))
     return t
 
 
 def matmul_lora(packed: np.ndarray, absmax: np.ndarray, N: int, K: int, x_bf16: np.ndarray, A_bf16: np.ndarray,
                 B_bf16: np.ndarray, r: int, scale: float, blocksize: int = 64) -> np.ndarray:
-    """fp64 y [B, N] = x . Wc^T + t . B^T with t = lora_down(x)."""
+    """fp64 y [B, N] = x . Wc^T + t . B^T with t = lora_down(x) (fp64, not rounded)."""
     x = np.ascontiguousarray(x_bf16, dtype=np.uint16).reshape(-1, K)
     A = np.ascontiguousarray(A_bf16, dtype=np.uint16).reshape(r, K)
     Bu = np.ascontiguousarray(B_bf16, dtype=np.uint16).reshape(N, r)
@@ -260,4 +261,20 @@ def matmul_lora(packed: np.ndarray, absmax: np.ndarray, N: int, K: int, x_bf16: 
     _load().oracle_nf4_matmul_lora(_p(np.ascontiguousarray(packed, dtype=np.uint8)),
                                    _p(np.ascontiguousarray(absmax, dtype=np.float32)), N, K, blocksize, _p(x),
                                    x.shape[0], _p(A), _p(Bu), r, float(scale), _p(y))
+    return y
+
+
+def matmul_lora_sampled(packed: np.ndarray, absmax: np.ndarray, N: int, K: int, x_bf16: np.ndarray,
+                        A_bf16: np.ndarray, B_bf16: np.ndarray, r: int, scale: float, bs: np.ndarray,
+                        ns: np.ndarray, blocksize: int = 64) -> np.ndarray:
+    """fp64 y of ``matmul_lora`` at the given (b, n) coordinates only."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16).reshape(-1, K)
+    t = lora_down(x, K, A_bf16, r, scale)
+    Bu = np.ascontiguousarray(B_bf16, dtype=np.uint16).reshape(N, r)
+    bs = np.ascontiguousarray(bs, dtype=np.int64)
+    ns = np.ascontiguousarray(ns, dtype=np.int64)
+    y = np.zeros(bs.size, np.float64)
+    _load().oracle_nf4_matmul_lora_sampled(_p(np.ascontiguousarray(packed, dtype=np.uint8)),
+                                           _p(np.ascontiguousarray(absmax, dtype=np.float32)), N, K, blocksize,
+                                           _p(x), _p(t), _p(Bu), r, _p(bs), _p(ns), bs.size, _p(y))
     return y

@@ -459,37 +459,49 @@ void oracle_nf4_matmul_dx_sampled(const uint8_t *packed, const float *absmax, in
 /* with adapters on a 4-bit model" (LoraConfig r = 16, lora_alpha = 32: the   */
 /* frozen 4-bit base plus small trainable adapter matrices).  The adapter is  */
 /* the usual pair of bf16 linear maps, down A [r, K] and up B [N, r], scaled  */
-/* by s = lora_alpha / r:                                                     */
-/*   t[b,j]  = bf16_rn(fp32(s * sum_k x[b,k] * A[j,k]))   (the down map's      */
-/*             bf16 output, scale applied before its rounding)                */
+/* by s = lora_alpha / r, with no rounding of the intermediate:               */
+/*   t[b,j]  = s * sum_k x[b,k] * A[j,k]                                       */
 /*   y[b,n]  = sum_k Wc[n,k] * x[b,k] + sum_j t[b,j] * B[n,j]                  */
-/* Sums of exact bf16 products in fp64; dropout is not part of the product.   */
+/* all in fp64 (products of bf16 values are exact); dropout is not part of    */
+/* the product.                                                               */
 /* ------------------------------------------------------------------------- */
 
 void oracle_lora_down(const uint16_t *x, int64_t Bn, int64_t K, const uint16_t *A, int32_t r, float scale,
-                      uint16_t *t) {
+                      double *t) {
 #pragma omp parallel for schedule(static)
   for (int64_t b = 0; b < Bn; ++b)
     for (int32_t j = 0; j < r; ++j) {
       double acc = 0.0;
       for (int64_t k = 0; k < K; ++k)
         acc += (double)oracle_bf16_to_f32(x[b * K + k]) * (double)oracle_bf16_to_f32(A[(int64_t)j * K + k]);
-      t[b * r + j] = oracle_bf16_rn((float)((double)scale * acc));
+      t[b * r + j] = (double)scale * acc;
     }
+}
+
+static double lora_term(const double *trow, const uint16_t *Bup, int64_t n, int32_t r) {
+  double acc = 0.0;
+  for (int32_t j = 0; j < r; ++j) acc += trow[j] * (double)oracle_bf16_to_f32(Bup[n * r + j]);
+  return acc;
 }
 
 void oracle_nf4_matmul_lora(const uint8_t *packed, const float *absmax, int64_t N, int64_t K, int32_t blocksize,
                             const uint16_t *x, int64_t Bn, const uint16_t *A, const uint16_t *Bup, int32_t r,
                             float scale, double *y) {
-  uint16_t *t = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(Bn * r > 0 ? Bn * r : 1));
+  double *t = (double *)malloc(sizeof(double) * (size_t)(Bn * r > 0 ? Bn * r : 1));
   oracle_lora_down(x, Bn, K, A, r, scale, t);
 #pragma omp parallel for schedule(static)
   for (int64_t n = 0; n < N; ++n)
-    for (int64_t b = 0; b < Bn; ++b) {
-      double acc = dot_row(packed, absmax, K, blocksize, n, x + b * K);
-      for (int32_t j = 0; j < r; ++j)
-        acc += (double)oracle_bf16_to_f32(t[b * r + j]) * (double)oracle_bf16_to_f32(Bup[n * r + j]);
-      y[b * N + n] = acc;
-    }
+    for (int64_t b = 0; b < Bn; ++b)
+      y[b * N + n] = dot_row(packed, absmax, K, blocksize, n, x + b * K) + lora_term(t + b * r, Bup, n, r);
   free(t);
+}
+
+/* Same arithmetic for a list of (b, n) output coordinates only (t from oracle_lora_down). */
+void oracle_nf4_matmul_lora_sampled(const uint8_t *packed, const float *absmax, int64_t N, int64_t K,
+                                    int32_t blocksize, const uint16_t *x, const double *t, const uint16_t *Bup,
+                                    int32_t r, const int64_t *bs, const int64_t *ns, int64_t count, double *y) {
+  (void)N;
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < count; ++i)
+    y[i] = dot_row(packed, absmax, K, blocksize, ns[i], x + bs[i] * K) + lora_term(t + bs[i] * r, Bup, ns[i], r);
 }

@@ -99,13 +99,17 @@ void oracle_nf4_matmul_dx_sampled(const uint8_t *packed, const float *absmax, in
                                   const int64_t *bs, const int64_t *ks, int64_t count, double *dx);
 
 /* Low-rank adapter on the 4-bit matmul (QLoRA): down map A bf16 [r,K], up map
- * Bup bf16 [N,r], scale s.  t = bf16_rn(fp32(s * x . A^T)) ([Bn, r], fp64 sums);
+ * Bup bf16 [N,r], scale s.  t = s * x . A^T in fp64 ([Bn, r], not rounded);
  * y[b,n] = sum_k Wc[n,k]*x[b,k] + sum_j t[b,j]*Bup[n,j] in fp64. */
 void oracle_lora_down(const uint16_t *x, int64_t Bn, int64_t K, const uint16_t *A, int32_t r, float scale,
-                      uint16_t *t);
+                      double *t);
 void oracle_nf4_matmul_lora(const uint8_t *packed, const float *absmax, int64_t N, int64_t K, int32_t blocksize,
                             const uint16_t *x, int64_t Bn, const uint16_t *A, const uint16_t *Bup, int32_t r,
                             float scale, double *y);
+/* The adapter product at a list of (b, n) coordinates, given t = oracle_lora_down(x). */
+void oracle_nf4_matmul_lora_sampled(const uint8_t *packed, const float *absmax, int64_t N, int64_t K,
+                                    int32_t blocksize, const uint16_t *x, const double *t, const uint16_t *Bup,
+                                    int32_t r, const int64_t *bs, const int64_t *ns, int64_t count, double *y);
 
 /* Worker threads used by the loops marked parallel (0 = OpenMP default). */
 void oracle_set_threads(int n);

@@ -23,7 +23,8 @@ from . import _lib
 from ._lib import NF4_BF16, NF4_DQ_E4M3, NF4_DQ_INT8, NF4_F32, NF4Error
 
 __all__ = ["QuantizedWeight", "quantize", "double_quant", "quantize_weight", "dequantize", "gemv", "gemm",
-           "storage_bytes", "gemm_workspace_bytes", "gemm_dx", "gemm_dx_workspace_bytes", "code_table", "check_device_error", "kernel_launches", "NF4Error", "library_path"]
+           "storage_bytes", "gemm_workspace_bytes", "gemm_dx", "gemm_dx_workspace_bytes", "gemm_lora",
+           "gemm_lora_workspace_bytes", "code_table", "check_device_error", "kernel_launches", "NF4Error", "library_path"]
 
 BLOCKSIZE = 64
 DQ_BLOCKSIZE = 256
@@ -186,6 +187,39 @@ def gemm_workspace_bytes(qw: QuantizedWeight, m: int) -> int:
     """Scratch bytes nf4_gemm needs for `m` activation rows (0 when none)."""
     d = qw.descriptor()
     return int(_lib.load().nf4_gemm_workspace_bytes(ctypes.byref(d), m))
+
+
+def gemm_lora(qw: QuantizedWeight, x: torch.Tensor, down: torch.Tensor, up: torch.Tensor, scale: float,
+              out=None, workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Y = bf16(X . Wc^T + scale * (X . down^T) . up^T): the 4-bit matmul with a low-rank adapter
+    (down bf16 [r, cols], up bf16 [rows, r], r in {16, 32}); the adapter's intermediate is not rounded."""
+    for t, name in ((x, "x"), (down, "down"), (up, "up")):
+        _need_cuda(t, name)
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bfloat16")
+    r = down.shape[0]
+    if down.shape != (r, qw.cols) or up.shape != (qw.rows, r) or not down.is_contiguous() or not up.is_contiguous():
+        raise ValueError("down must be [r, cols] and up [rows, r], contiguous")
+    x2 = x.reshape(-1, qw.cols)
+    m = x2.shape[0]
+    lib = _lib.load()
+    d = qw.descriptor()
+    if out is None:
+        out = torch.empty(m, qw.rows, dtype=torch.bfloat16, device=x.device)
+    ws_bytes = lib.nf4_gemm_lora_workspace_bytes(ctypes.byref(d), m)
+    if workspace is None:
+        workspace = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=x.device)  # zeroed once, then reusable
+    lo = _lib.NF4Lora(_ptr(down), _ptr(up), r, float(scale))
+    st = lib.nf4_gemm_lora(ctypes.byref(d), ctypes.byref(lo), _ptr(x2), m, _ptr(out), _ptr(workspace),
+                           workspace.numel(), _stream(stream))
+    _lib.check(st, "nf4_gemm_lora")
+    return out
+
+
+def gemm_lora_workspace_bytes(qw: QuantizedWeight, m: int) -> int:
+    """Scratch bytes nf4_gemm_lora needs for `m` activation rows."""
+    d = qw.descriptor()
+    return int(_lib.load().nf4_gemm_lora_workspace_bytes(ctypes.byref(d), m))
 
 
 def gemm_dx(qw: QuantizedWeight, dy: torch.Tensor, out=None, workspace: Optional[torch.Tensor] = None,

@@ -30,6 +30,11 @@ class NF4Weight(ctypes.Structure):
                 ("rows", I64), ("cols", I64), ("blocksize", I32), ("dq_blocksize", I32), ("dq_code", I32)]
 
 
+class NF4Lora(ctypes.Structure):
+    """Mirror of the C struct nf4_lora."""
+    _fields_ = [("down", P), ("up", P), ("r", I32), ("scale", ctypes.c_float)]
+
+
 SIGNATURES = {
     "nf4_quantize": (ctypes.c_int, [P, I32, I64, I32, P, P, P]),
     "nf4_double_quant": (ctypes.c_int, [P, I64, I32, I32, P, P, P, P, SZ, P]),
@@ -39,6 +44,8 @@ SIGNATURES = {
     "nf4_gemv": (ctypes.c_int, [ctypes.POINTER(NF4Weight), P, I32, P, P]),
     "nf4_gemm": (ctypes.c_int, [ctypes.POINTER(NF4Weight), P, I64, P, P, SZ, P]),
     "nf4_gemm_workspace_bytes": (SZ, [ctypes.POINTER(NF4Weight), I64]),
+    "nf4_gemm_lora": (ctypes.c_int, [ctypes.POINTER(NF4Weight), ctypes.POINTER(NF4Lora), P, I64, P, P, SZ, P]),
+    "nf4_gemm_lora_workspace_bytes": (SZ, [ctypes.POINTER(NF4Weight), I64]),
     "nf4_gemm_dx": (ctypes.c_int, [ctypes.POINTER(NF4Weight), P, I64, P, P, SZ, P]),
     "nf4_gemm_dx_workspace_bytes": (SZ, [ctypes.POINTER(NF4Weight), I64]),
     "nf4_storage_bytes": (SZ, [I64, I32, I32, I32]),

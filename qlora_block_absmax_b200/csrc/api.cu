@@ -112,6 +112,11 @@ size_t nf4_gemm_workspace_bytes(const nf4_weight* w, int64_t m) {
   return nf4::gemm_workspace_bytes(w->rows, w->cols, m);
 }
 
+size_t nf4_gemm_lora_workspace_bytes(const nf4_weight* w, int64_t m) {
+  if (w == nullptr || w->rows <= 0 || w->cols <= 0 || m <= 0) return 0;
+  return nf4::gemm_lora_workspace_bytes(w->rows, w->cols, m);
+}
+
 size_t nf4_gemm_dx_workspace_bytes(const nf4_weight* w, int64_t m) {
   if (w == nullptr || w->rows <= 0 || w->cols <= 0 || m <= 0) return 0;
   if (w->rows % 64 != 0 || w->cols % 128 != 0) return 0;
@@ -260,6 +265,29 @@ nf4_status nf4_gemm(const nf4_weight* w, const void* x, int64_t m, void* y, void
   if ((st = device_info(&d)) != NF4_OK) return st;
   return from_cuda(nf4::launch_gemm(w->packed, s, w->rows, w->cols, x, m, y, workspace, d.error_word,
                                     reinterpret_cast<cudaStream_t>(stream), d.num_sms));
+}
+
+nf4_status nf4_gemm_lora(const nf4_weight* w, const nf4_lora* lora, const void* x, int64_t m, void* y,
+                         void* workspace, size_t workspace_bytes, nf4_stream_t stream) {
+  nf4::Scales s;
+  nf4_status st = check_weight(w, &s);
+  if (st != NF4_OK) return st;
+  if (m < 0 || lora == nullptr) return NF4_ERR_INVALID_ARG;
+  if (lora->r != 16 && lora->r != 32) return NF4_ERR_UNSUPPORTED;
+  if (!(lora->scale == lora->scale) || lora->scale - lora->scale != 0.0f) return NF4_ERR_INVALID_ARG;  // finite
+  if (w->cols % nf4::kBlock != 0 || w->rows % 128 != 0) return NF4_ERR_UNSUPPORTED;
+  if (m == 0 || w->rows == 0 || w->cols == 0) return NF4_OK;
+  if (x == nullptr || y == nullptr || lora->down == nullptr || lora->up == nullptr || workspace == nullptr)
+    return NF4_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(y, 16) || !aligned(lora->down, 16) || !aligned(lora->up, 16) ||
+      !aligned(workspace, 16))
+    return NF4_ERR_MISALIGNED;
+  if (workspace_bytes < nf4::gemm_lora_workspace_bytes(w->rows, w->cols, m)) return NF4_ERR_INVALID_ARG;
+  DeviceInfo d;
+  if ((st = device_info(&d)) != NF4_OK) return st;
+  return from_cuda(nf4::launch_gemm_lora(w->packed, s, w->rows, w->cols, x, m, lora->down, lora->up, lora->r,
+                                         lora->scale, y, workspace, d.error_word,
+                                         reinterpret_cast<cudaStream_t>(stream), d.num_sms));
 }
 
 nf4_status nf4_gemm_dx(const nf4_weight* w, const void* dy, int64_t m, void* dx, void* workspace,

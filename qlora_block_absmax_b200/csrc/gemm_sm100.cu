@@ -82,7 +82,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(Scales s, int rows, int cols, int m_total, int splits, const __grid_constant__ CUtensorMap xmap,
                 const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
                 __nv_bfloat16* __restrict__ y, float* __restrict__ part, unsigned* __restrict__ tile_count,
-                unsigned* err) {
+                unsigned* err, const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __restrict__ lora_up,
+                int lora_r) {
   extern __shared__ uint8_t smem_raw[];
   pdl_launch_dependents();
   const uint32_t raw = smem_u32(smem_raw);
@@ -143,14 +144,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float mu = kDQ ? *s.mean : 0.0f;
     const int64_t rb = cols / kBlock;
     const DecodeMul dm = decode_mul();
-    uint32_t it = 0;
+    uint32_t it = 0, wit = 0;  // stages (A ring, group alternation); weight stages (code ring)
     for (int u = blockIdx.x; u < wk.units; u += gridDim.x) {
       const int64_t row = (int64_t)wk.n0(u) + p;
       const int ks0 = wk.split(u) * wk.kps;
-      for (int ks = ks0; ks < ks0 + wk.kps; ++ks, ++it) {
+      const int ks1 = ks0 + wk.kps + (lora_r > 0 && wk.split(u) == 0 ? 1 : 0);  // + the adapter stage
+      for (int ks = ks0; ks < ks1; ++ks, ++it) {
+        const bool adapter = ks == ks0 + wk.kps;
+        if (!adapter) ++wit;
         if ((int)(it & 1) != group) continue;
-        const int ws = it % kWStages, as = it % kAStages;
-        const uint32_t wph = (it / kWStages) & 1, aph = (it / kAStages) & 1;
+        const int as = it % kAStages;
+        const uint32_t aph = (it / kAStages) & 1;
+        if (adapter) {
+          // adapter stage: this row of the up map B[n, 0..r) twice, [B | B] in the first r columns of the A slot
+          // (zeros after), against [T_hi | T_lo] of the down map
+          uint32_t r[32];
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            uint4 v = make_uint4(0, 0, 0, 0);
+            const int e = 2 * j;  // first element of these 8
+            if (e < 2 * lora_r)
+              v = __ldg(reinterpret_cast<const uint4*>(lora_up + row * lora_r + (e < lora_r ? e : e - lora_r)));
+            r[j] = v.x;
+            r[j + 1] = v.y;
+            r[j + 2] = v.z;
+            r[j + 3] = v.w;
+          }
+          if (!wait_or_abort(&sm->aempty[as], aph ^ 1, sm, err)) break;
+          const uint32_t ta = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(kAccCols + as * 32);
+          tmem_st32(ta, r);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm->afull[as]);
+          continue;
+        }
+        const int ws = (wit - 1) % kWStages;
+        const uint32_t wph = ((wit - 1) / kWStages) & 1;
         if (!wait_or_abort(&sm->wfull[ws], wph, sm, err)) break;  // codes + scale chunk landed
         const uint4* wsrc = reinterpret_cast<const uint4*>(w_gen0 + ws * kWBytes + p * 32);
         const uint4 w0 = wsrc[0], w1 = wsrc[1];
@@ -180,18 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           r[4 * c + 3] = d[3];
         }
         if (!wait_or_abort(&sm->aempty[as], aph ^ 1, sm, err)) break;  // the MMAs left this slot
-        {
-          const uint32_t ta = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(kAccCols + as * 32);
-          asm volatile(
-              "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-              "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n"
-              "tcgen05.wait::st.sync.aligned;" ::"r"(ta),
-              "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-              "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
-              "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
-              "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-              : "memory");
-        }
+        tmem_st32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(kAccCols + as * 32), r);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm->afull[as]);
@@ -205,13 +223,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0;
       for (int u = blockIdx.x; u < wk.units && !aborted(sm); u += gridDim.x) {
         const int ks0 = wk.split(u) * wk.kps;
+        const int ks1 = ks0 + wk.kps + (lora_r > 0 && wk.split(u) == 0 ? 1 : 0);
         const int m0 = wk.m0(u);
-        for (int ks = ks0; ks < ks0 + wk.kps; ++ks, ++it) {
+        for (int ks = ks0; ks < ks1; ++ks, ++it) {
           const int xs = it % kXStages;
           if (!wait_or_abort(&sm->xempty[xs], ((it / kXStages) & 1) ^ 1, sm, err)) break;
           if (it == 0) NF4_STAMP(1);
           mbar_expect_tx(&sm->xfull[xs], kBBytes);
-          tma_load_2d(b_smem0 + xs * kBBytes, &xmap, ks * kTileK, m0, &sm->xfull[xs]);
+          if (ks == ks0 + wk.kps)  // adapter stage: the rows of T = bf16(s * X . A^T), 64 wide
+            tma_load_2d(b_smem0 + xs * kBBytes, &tmap, 0, m0, &sm->xfull[xs]);
+          else
+            tma_load_2d(b_smem0 + xs * kBBytes, &xmap, ks * kTileK, m0, &sm->xfull[xs]);
         }
       }
       const uint32_t issued = it;  // drain the copies still in flight
@@ -252,7 +274,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem + acc * kAccCols;
         bool ok = true;
-        for (int j = 0; j < wk.kps; ++j, ++it) {
+        const int nst = wk.kps + (lora_r > 0 && wk.split(u) == 0 ? 1 : 0);  // + the adapter stage
+        for (int j = 0; j < nst; ++j, ++it) {
           const int as = it % kAStages, xs = it % kXStages;
           if (!wait_or_abort(&sm->afull[as], (it / kAStages) & 1, sm, err) ||
               !wait_or_abort(&sm->xfull[xs], (it / kXStages) & 1, sm, err)) {
@@ -262,9 +285,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           if (it == 0) NF4_STAMP(2);
           const uint32_t a_tm = tmem + (uint32_t)(kAccCols + as * 32), b_addr = b_smem0 + xs * kBBytes;
+          const int nkk = j < wk.kps ? kTileK / 16 : lora_r / 8;  // the adapter stage reduces over 2r only
 #pragma unroll
           for (int kk = 0; kk < kTileK / 16; ++kk)  // 16 bf16 per MMA along k: 8 TMEM columns, 32 smem bytes
-            tc_mma_ts(d_tmem, a_tm + kk * 8, smem_desc_sw128(b_addr + kk * 32), idesc, (j | kk) != 0);
+            if (kk < nkk) tc_mma_ts(d_tmem, a_tm + kk * 8, smem_desc_sw128(b_addr + kk * 32), idesc, (j | kk) != 0);
           tc_commit(&sm->aempty[as]);  // slots free once these MMAs have read them
           tc_commit(&sm->xempty[xs]);
         }
@@ -367,7 +391,8 @@ namespace {
 template <bool kDQ, bool kScaleTma>
 cudaError_t launch_variant(const Scales& s, int rows, int cols, int m, int splits, const CUtensorMap& xmap,
                            const CUtensorMap& wmap, const CUtensorMap& smap, __nv_bfloat16* y, float* part,
-                           unsigned* counters, unsigned* err, int grid, cudaStream_t stream) {
+                           unsigned* counters, unsigned* err, int grid, cudaStream_t stream, const CUtensorMap& tmap,
+                           const __nv_bfloat16* lora_up, int lora_r) {
   // the shared-memory opt-in is a per-device function attribute: set it once
   // per device (outside any stream capture that later calls may be part of)
   static std::atomic<uint64_t> attr_done{0};
@@ -380,25 +405,36 @@ cudaError_t launch_variant(const Scales& s, int rows, int cols, int m, int split
     attr_done.fetch_or(1ull << dev);
   }
   const cudaError_t e = launch_pdl(gemm_kernel<kDQ, kScaleTma>, dim3(grid), dim3(kThreads), kSmemBytes, stream, s,
-                                   rows, cols, m, splits, xmap, wmap, smap, y, part, counters, err);
+                                   rows, cols, m, splits, xmap, wmap, smap, y, part, counters, err, tmap, lora_up,
+                                   lora_r);
   count_launches(1);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_gemm(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x, int64_t m,
-                        void* y, void* workspace, unsigned* err, cudaStream_t stream, int num_sms) {
+namespace {
+
+// the tcgen05 kernel for m activation rows; with lora_r > 0 each output tile adds one adapter stage
+// (T = the [m, 64] bf16 down-map output [hi | lo | 0] at `t`, lora_up = B [rows, r])
+cudaError_t launch_tc(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x, int64_t m,
+                      void* y, int splits, void* workspace, unsigned* err, cudaStream_t stream, int num_sms,
+                      const void* t, const void* lora_up, int lora_r) {
   auto* yb = static_cast<__nv_bfloat16*>(y);
-  if (m <= 64) return launch_gemv(packed, s, rows, cols, x, (int)m, y, stream, num_sms);
   if (rows > INT32_MAX || cols > INT32_MAX || m > INT32_MAX) return cudaErrorInvalidValue;
   const bool dq = s.absmax == nullptr;
   const int64_t rb = cols / kBlock;  // level-1 blocks per weight row
-  CUtensorMap xmap, wmap, smap;
+  CUtensorMap xmap, wmap, smap, tmap;
   if (!make_map(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, cols, m, kTileK, kTileM, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, packed, cols / 2, rows, kTileK / 2, kTileN,
                 CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorNotSupported;
+  if (lora_r > 0) {
+    if (!make_map(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, t, kTileK, m, kTileK, kTileM, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorNotSupported;
+  } else {
+    tmap = xmap;  // unused
+  }
   // scale chunks through TMA when each row of scales is a whole number of 16-byte units
   const void* sbase = dq ? (const void*)s.q : (const void*)s.absmax;
   const size_t srow = dq ? (size_t)rb : (size_t)rb * 4;
@@ -409,7 +445,6 @@ cudaError_t launch_gemm(const uint8_t* packed, const Scales& s, int64_t rows, in
                    : make_map(&smap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, sbase, rb, rows, 4, kTileN,
                               CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!scale_tma) smap = wmap;  // unused by the kernel variant
-  const int splits = gemm_splits(rows, cols, m, num_sms);
   const int64_t ntiles = (rows / kTileN) * ((m + kTileM - 1) / kTileM);
   const int64_t units = ntiles * splits;
   const int grid = (int)(units < num_sms ? units : num_sms);
@@ -421,13 +456,52 @@ cudaError_t launch_gemm(const uint8_t* packed, const Scales& s, int64_t rows, in
     part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + cbytes);
   }
   const int R = (int)rows, C = (int)cols, M = (int)m;
+  const auto* up = static_cast<const __nv_bfloat16*>(lora_up);
   if (dq && scale_tma)
-    return launch_variant<true, true>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream);
+    return launch_variant<true, true>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
+                                      tmap, up, lora_r);
   if (dq)
-    return launch_variant<true, false>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream);
+    return launch_variant<true, false>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
+                                       tmap, up, lora_r);
   if (scale_tma)
-    return launch_variant<false, true>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream);
-  return launch_variant<false, false>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream);
+    return launch_variant<false, true>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
+                                       tmap, up, lora_r);
+  return launch_variant<false, false>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
+                                      tmap, up, lora_r);
+}
+
+// the adapter path: its own split choice (no GEMV route for small m), the [m, 64] bf16 down-map output first
+// in the workspace, the split-K scratch after it
+int lora_splits(int64_t rows, int64_t cols, int64_t m, int num_sms) {
+  return reduction_splits((rows / kTileN) * ((m + kTileM - 1) / kTileM), cols / kTileK, num_sms);
+}
+
+size_t lora_t_bytes(int64_t m) { return ((size_t)m * kTileK * 2 + 255) & ~(size_t)255; }
+
+}  // namespace
+
+cudaError_t launch_gemm(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x, int64_t m,
+                        void* y, void* workspace, unsigned* err, cudaStream_t stream, int num_sms) {
+  if (m <= 64) return launch_gemv(packed, s, rows, cols, x, (int)m, y, stream, num_sms);
+  return launch_tc(packed, s, rows, cols, x, m, y, gemm_splits(rows, cols, m, num_sms), workspace, err, stream,
+                   num_sms, nullptr, nullptr, 0);
+}
+
+size_t gemm_lora_workspace_bytes(int64_t rows, int64_t cols, int64_t m) {
+  const int64_t ntiles = (rows / kTileN) * ((m + kTileM - 1) / kTileM);
+  return lora_t_bytes(m) + split_workspace_bytes(ntiles, lora_splits(rows, cols, m, sm_count()));
+}
+
+cudaError_t launch_gemm_lora(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x,
+                             int64_t m, const void* lora_down, const void* lora_up, int lora_r, float lora_scale,
+                             void* y, void* workspace, unsigned* err, cudaStream_t stream, int num_sms) {
+  if (rows > INT32_MAX || cols > INT32_MAX || m > INT32_MAX) return cudaErrorInvalidValue;
+  void* t = workspace;
+  cudaError_t e = launch_lora_down(x, lora_down, m, cols, lora_r, lora_scale, t, stream);
+  if (e != cudaSuccess) return e;
+  void* split_ws = static_cast<uint8_t*>(workspace) + lora_t_bytes(m);
+  return launch_tc(packed, s, rows, cols, x, m, y, lora_splits(rows, cols, m, num_sms), split_ws, err, stream,
+                   num_sms, t, lora_up, lora_r);
 }
 
 }  // namespace nf4

@@ -60,6 +60,15 @@ size_t gemm_workspace_bytes(int64_t rows, int64_t cols, int64_t m);
 cudaError_t launch_gemm(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x,
                         int64_t m, void* y, void* workspace, unsigned* err, cudaStream_t stream, int num_sms);
 
+// 4-bit matmul plus a low-rank adapter: T = scale * X . A^T as a bf16 pair [hi | lo] into the first bytes of
+// the workspace ([m, 64] bf16), then the GEMM with one adapter stage per output tile (r in {16, 32})
+cudaError_t launch_lora_down(const void* x, const void* a, int64_t m, int64_t cols, int r, float scale, void* t,
+                             cudaStream_t stream);
+size_t gemm_lora_workspace_bytes(int64_t rows, int64_t cols, int64_t m);
+cudaError_t launch_gemm_lora(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x,
+                             int64_t m, const void* lora_down, const void* lora_up, int lora_r, float lora_scale,
+                             void* y, void* workspace, unsigned* err, cudaStream_t stream, int num_sms);
+
 // input gradient dX = dY . Wc (rows % 64 == 0, cols % 128 == 0)
 size_t gemm_dx_workspace_bytes(int64_t rows, int64_t cols, int64_t m);
 cudaError_t launch_gemm_dx(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* dy,

@@ -383,6 +383,110 @@ def test_gemm_scale_paths(cols, use_dq):
     check_matmul(y, oracle.matmul(p_ref, a_ref, rows, cols, x), f"gemm cols{cols} dq{use_dq}")
 
 
+# --------------------------------------------------------------------------- 4-bit matmul + low-rank adapter
+
+def lora_maps(rows, cols, r, seed):
+    """bf16 adapter maps: down ~N(0, 1/cols) (so T is O(1)), up ~N(0, 0.02)"""
+    down = synth.f32_to_bf16_bits((synth.rng(seed).standard_normal((r, cols)) / np.sqrt(cols)).astype(np.float32))
+    up = synth.f32_to_bf16_bits((synth.rng(seed + 1).standard_normal((rows, r)) * 0.02).astype(np.float32))
+    return down, up
+
+
+@pytest.mark.parametrize("m", [1, 16, 65, 256, 300])
+def test_gemm_lora_small(m):
+    rows, cols, r = 256, 512, 16
+    qw, p_ref, a_ref = quantized_pair(rows, cols, 111 + m, True)
+    x = synth.activations((m, cols), 112 + m)
+    down, up = lora_maps(rows, cols, r, 113 + m)
+    y = nf4.gemm_lora(qw, dev_bf16(x), dev_bf16(down), dev_bf16(up), 2.0)
+    check_matmul(y, oracle.matmul_lora(p_ref, a_ref, rows, cols, x, down, up, r, 2.0), f"gemm_lora m{m}")
+
+
+@pytest.mark.parametrize("r", [16, 32])
+@pytest.mark.parametrize("use_dq", [False, True])
+def test_gemm_lora_ranks(r, use_dq):
+    rows, cols, m = 384, 1024, 200
+    qw, p_ref, a_ref = quantized_pair(rows, cols, 120 + r, use_dq)
+    x = synth.activations((m, cols), 121 + r)
+    down, up = lora_maps(rows, cols, r, 122 + r)
+    y = nf4.gemm_lora(qw, dev_bf16(x), dev_bf16(down), dev_bf16(up), 32.0 / r)
+    check_matmul(y, oracle.matmul_lora(p_ref, a_ref, rows, cols, x, down, up, r, 32.0 / r), f"gemm_lora r{r}")
+
+
+@pytest.mark.parametrize("m", [65, 256, 300])
+def test_gemm_lora_split(m):
+    """few output tiles: the adapter stage rides with split 0 of each tile"""
+    rows, cols, r = 256, 2048, 16
+    qw, p_ref, a_ref = quantized_pair(rows, cols, 130 + m, True)
+    x = synth.activations((m, cols), 131 + m)
+    down, up = lora_maps(rows, cols, r, 132 + m)
+    y = nf4.gemm_lora(qw, dev_bf16(x), dev_bf16(down), dev_bf16(up), 2.0)
+    check_matmul(y, oracle.matmul_lora(p_ref, a_ref, rows, cols, x, down, up, r, 2.0), f"gemm_lora split m{m}")
+
+
+def test_gemm_lora_zero_up_is_gemm_bit_exact_and_down_map():
+    """with up = 0 the adapter stage adds exact zeros: the same bits as nf4_gemm (same tiles and splits).  The
+    down map left in the workspace as a bf16 pair [hi | lo | 0] holds v = s * X . A^T: lo is at most half a bf16
+    ulp of hi, and hi + lo is within 2^-15 relative of the oracle's fp64 value, plus fp32 summation error (1e-6 of
+    sum |x a|)"""
+    rows, cols, m, r = 4096, 4096, 256, 16
+    qw, p_ref, a_ref = quantized_pair(rows, cols, 140, True)
+    x = synth.activations((m, cols), 141)
+    down, _ = lora_maps(rows, cols, r, 142)
+    ws = torch.zeros(nf4.gemm_lora_workspace_bytes(qw, m), dtype=torch.uint8, device="cuda")
+    y = nf4.gemm_lora(qw, dev_bf16(x), dev_bf16(down), torch.zeros(rows, r, dtype=torch.bfloat16, device="cuda"),
+                      2.0, workspace=ws)
+    assert torch.equal(y.view(torch.int16), nf4.gemm(qw, dev_bf16(x)).view(torch.int16))
+    t = ws[:m * 64 * 2].view(torch.int16).view(m, 64).cpu().numpy().view(np.uint16)
+    assert np.all(t[:, 2 * r:] == 0)
+    hi = synth.bf16_bits_to_f32(t[:, :r]).astype(np.float64)
+    lo = synth.bf16_bits_to_f32(t[:, r:2 * r]).astype(np.float64)
+    v = hi + lo
+    assert np.all(np.abs(lo) <= 2.0 ** -8 * np.abs(hi))  # lo is the rounding remainder of hi
+    t_ref = oracle.lora_down(x, cols, down, r, 2.0)
+    absdot = np.abs(synth.bf16_bits_to_f32(x).astype(np.float64)) @ np.abs(
+        synth.bf16_bits_to_f32(down).astype(np.float64)).T
+    assert np.all(np.abs(v - t_ref) <= 2.0 ** -15 * np.abs(t_ref) + 1e-6 * 2.0 * absdot)
+
+
+def test_gemm_lora_adapter_only():
+    """zero-code weight: Y is the adapter term alone"""
+    rows, cols, m, r = 256, 1024, 300, 16
+    p = torch.full((rows * cols // 2,), 0x77, dtype=torch.uint8, device="cuda")
+    absmax = torch.ones(rows * cols // 64, dtype=torch.float32, device="cuda")
+    qw = nf4.QuantizedWeight(packed=p, rows=rows, cols=cols, absmax=absmax)
+    x = synth.activations((m, cols), 150)
+    down, up = lora_maps(rows, cols, r, 151)
+    y = nf4.gemm_lora(qw, dev_bf16(x), dev_bf16(down), dev_bf16(up), 2.0)
+    ref = oracle.matmul_lora(np.full(rows * cols // 2, 0x77, np.uint8), np.ones(rows * cols // 64, np.float32),
+                             rows, cols, x, down, up, r, 2.0)
+    check_matmul(y, ref, "gemm_lora adapter only")
+
+
+@pytest.mark.parametrize("m", [16, 256, 1024, 4096])
+def test_gemm_lora_config4_sampled(m):
+    """W 14336x4096 NF4+DQ with an r = 16, alpha = 32 adapter at the prefill sizes: 2048 sampled outputs and
+    all of row 0 against the oracle; ten identical calls give identical bits"""
+    rows, cols, r = 14336, 4096, 16
+    qw, p_ref, a_ref = quantized_pair(rows, cols, 1020, True)
+    x = synth.activations((m, cols), 1021 + m)
+    down, up = lora_maps(rows, cols, r, 160)
+    ws = torch.zeros(nf4.gemm_lora_workspace_bytes(qw, m), dtype=torch.uint8, device="cuda")
+    args = (qw, dev_bf16(x), dev_bf16(down), dev_bf16(up), 2.0)
+    y = nf4.gemm_lora(*args, workspace=ws)
+    for _ in range(3):
+        assert torch.equal(nf4.gemm_lora(*args, workspace=ws).view(torch.int16), y.view(torch.int16))
+    rg = synth.rng(170 + m)
+    bs, ns = rg.integers(0, m, 2048), rg.integers(0, rows, 2048)
+    ref = oracle.matmul_lora_sampled(p_ref, a_ref, rows, cols, x, down, up, r, 2.0, bs, ns)
+    full_row = oracle.matmul_lora(p_ref, a_ref, rows, cols, x[:1], down, up, r, 2.0)
+    rms = np.sqrt(np.mean(full_row ** 2))
+    got = y.float().cpu().numpy().astype(np.float64)[bs, ns]
+    assert np.all(np.abs(got - ref) <= REL_TOL * np.maximum(np.abs(ref), FLOOR * rms))
+    check_matmul(y[:1], full_row, f"gemm_lora m{m} row 0")
+    nf4.check_device_error()
+
+
 # --------------------------------------------------------------------------- input gradient dX = dY . Wc
 
 def check_dx_sampled(dx: torch.Tensor, p_ref, a_ref, rows, cols, dy, seed, count=2048):
