@@ -133,7 +133,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  pdl_wait();  // everything above is on-chip set-up; from here on global memory is read and written
+  // Everything above is on-chip set-up; from here on global memory is read and written.  With an adapter
+  // (lora_r > 0) the launch before this one is the down map, which let this grid start only after its own
+  // predecessor had finished: X, the weight and the outputs are safe to touch now, and only the adapter
+  // stage's load of the down map's output waits for that grid (in the activation TMA warp).
+  if (lora_r == 0) pdl_wait();
   const uint32_t tmem = sm->tmem_base;
   if (threadIdx.x == 0) NF4_STAMP(0);
 
@@ -230,10 +234,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!wait_or_abort(&sm->xempty[xs], ((it / kXStages) & 1) ^ 1, sm, err)) break;
           if (it == 0) NF4_STAMP(1);
           mbar_expect_tx(&sm->xfull[xs], kBBytes);
-          if (ks == ks0 + wk.kps)  // adapter stage: the rows of T = bf16(s * X . A^T), 64 wide
+          if (ks == ks0 + wk.kps) {  // adapter stage: the down map's [hi | lo | 0] rows, 64 wide
+            pdl_wait();              // the down-map grid has finished and its writes are visible
             tma_load_2d(b_smem0 + xs * kBBytes, &tmap, 0, m0, &sm->xfull[xs]);
-          else
+          } else {
             tma_load_2d(b_smem0 + xs * kBBytes, &xmap, ks * kTileK, m0, &sm->xfull[xs]);
+          }
         }
       }
       const uint32_t issued = it;  // drain the copies still in flight

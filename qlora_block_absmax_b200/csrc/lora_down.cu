@@ -40,8 +40,11 @@ __global__ void __launch_bounds__(kWarps * 32) lora_down_kernel(const __nv_bfloa
                                                                  const __nv_bfloat16* __restrict__ a, int m_total,
                                                                  int cols, float scale, __nv_bfloat16* __restrict__ t) {
   __shared__ float red[kWarps][16][NT * 8];
-  pdl_launch_dependents();
+  // the GEMM that consumes T starts once every CTA is past this wait, i.e. once this launch's own
+  // predecessor has finished: the GEMM can then read X and the weight at once and waits for this grid
+  // only before its adapter stage loads T
   pdl_wait();
+  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, q = lane & 3;
   const int m0 = blockIdx.x * 16;
