@@ -156,6 +156,19 @@ NF4_API nf4_status nf4_dequantize(const nf4_weight *w, void *out, int32_t out_dt
  *   1 <= batch <= 8; cols % 64 == 0; rows % 16 == 0. */
 NF4_API nf4_status nf4_gemv(const nf4_weight *w, const void *x, int32_t batch, void *y, nf4_stream_t stream);
 
+/* nf4_gemv for up to 4 weights that read the same input, in one launch (the
+ * q/k/v projections of an attention block, or gate/up of an MLP, in the
+ * decode pass over a whole 4-bit model such as the Llama-3.1-8B of [bnb-tut]
+ * "4-bit Loading with NF4").  Each weight gets exactly the results nf4_gemv
+ * would give it.
+ *   ws     host array of `count` weight descriptors (1 <= count <= 4), all
+ *          with the same cols and the same scale kind (plain or double-quant)
+ *   x      device bf16 [batch, cols];  ys  host array of `count` device bf16
+ *          outputs, ys[i] of shape [batch, ws[i]->rows]
+ *   1 <= batch <= 8; cols % 64 == 0; every rows % 16 == 0. */
+NF4_API nf4_status nf4_gemv_grouped(const nf4_weight *const *ws, int32_t count, const void *x, int32_t batch,
+                            void *const *ys, nf4_stream_t stream);
+
 /* Prefill GEMM, same arithmetic as nf4_gemv for m activation rows:
  *   Y[m, n] = bf16_rn( sum_k Wc[n, k] * X[m, k] )
  * on tcgen05 tensor cores (bf16 x bf16 -> fp32 in tensor memory).

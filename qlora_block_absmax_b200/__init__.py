@@ -23,7 +23,7 @@ from . import _lib
 from ._lib import NF4_BF16, NF4_DQ_E4M3, NF4_DQ_INT8, NF4_F32, NF4Error
 
 __all__ = ["QuantizedWeight", "quantize", "double_quant", "quantize_weight", "dequantize", "gemv", "gemm",
-           "storage_bytes", "gemm_workspace_bytes", "gemm_dx", "gemm_dx_workspace_bytes", "gemm_lora",
+           "storage_bytes", "gemm_workspace_bytes", "gemm_dx", "gemm_dx_workspace_bytes", "gemm_lora", "gemv_grouped",
            "gemm_lora_workspace_bytes", "code_table", "check_device_error", "kernel_launches", "NF4Error", "library_path"]
 
 BLOCKSIZE = 64
@@ -160,6 +160,24 @@ def gemv(qw: QuantizedWeight, x: torch.Tensor, out=None, stream=None) -> torch.T
     st = _lib.load().nf4_gemv(ctypes.byref(d), _ptr(x2), x2.shape[0], _ptr(out), _stream(stream))
     _lib.check(st, "nf4_gemv")
     return out
+
+
+def gemv_grouped(qws, x: torch.Tensor, outs=None, stream=None) -> list:
+    """nf4_gemv of up to 4 weights with the same cols on one input x (bf16 [B, cols], B <= 8), in one launch."""
+    _need_cuda(x, "x")
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be bfloat16")
+    qws = list(qws)
+    cols = qws[0].cols
+    x2 = x.reshape(-1, cols)
+    if outs is None:
+        outs = [torch.empty(x2.shape[0], q.rows, dtype=torch.bfloat16, device=x.device) for q in qws]
+    ds = [q.descriptor() for q in qws]
+    arr = (ctypes.POINTER(_lib.NF4Weight) * len(ds))(*[ctypes.pointer(d) for d in ds])
+    ys = (ctypes.c_void_p * len(outs))(*[_ptr(o) for o in outs])
+    st = _lib.load().nf4_gemv_grouped(arr, len(ds), _ptr(x2), x2.shape[0], ys, _stream(stream))
+    _lib.check(st, "nf4_gemv_grouped")
+    return outs
 
 
 def gemm(qw: QuantizedWeight, x: torch.Tensor, out=None, workspace: Optional[torch.Tensor] = None,

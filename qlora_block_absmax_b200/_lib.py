@@ -42,6 +42,7 @@ SIGNATURES = {
     "nf4_double_quant_noalloc": (ctypes.c_int, [P, I64, I32, I32, P, P, P, P]),
     "nf4_dequantize": (ctypes.c_int, [ctypes.POINTER(NF4Weight), P, I32, P]),
     "nf4_gemv": (ctypes.c_int, [ctypes.POINTER(NF4Weight), P, I32, P, P]),
+    "nf4_gemv_grouped": (ctypes.c_int, [ctypes.POINTER(ctypes.POINTER(NF4Weight)), I32, P, I32, ctypes.POINTER(P), P]),
     "nf4_gemm": (ctypes.c_int, [ctypes.POINTER(NF4Weight), P, I64, P, P, SZ, P]),
     "nf4_gemm_workspace_bytes": (SZ, [ctypes.POINTER(NF4Weight), I64]),
     "nf4_gemm_lora": (ctypes.c_int, [ctypes.POINTER(NF4Weight), ctypes.POINTER(NF4Lora), P, I64, P, P, SZ, P]),

@@ -248,6 +248,39 @@ nf4_status nf4_gemv(const nf4_weight* w, const void* x, int32_t batch, void* y, 
                                     reinterpret_cast<cudaStream_t>(stream), d.num_sms));
 }
 
+nf4_status nf4_gemv_grouped(const nf4_weight* const* ws, int32_t count, const void* x, int32_t batch, void* const* ys,
+                            nf4_stream_t stream) {
+  if (ws == nullptr || ys == nullptr || count < 1 || count > nf4::kMaxGroup) return NF4_ERR_INVALID_ARG;
+  if (batch < 1 || batch > 8) return NF4_ERR_INVALID_ARG;
+  nf4::Scales s[nf4::kMaxGroup];
+  const uint8_t* packed[nf4::kMaxGroup];
+  int64_t rows[nf4::kMaxGroup];
+  void* y[nf4::kMaxGroup];
+  int n = 0;
+  for (int i = 0; i < count; ++i) {
+    nf4_status st = check_weight(ws[i], &s[n]);
+    if (st != NF4_OK) return st;
+    const nf4_weight* w = ws[i];
+    if (w->cols != ws[0]->cols || (w->absmax == nullptr) != (ws[0]->absmax == nullptr)) return NF4_ERR_INVALID_ARG;
+    if (w->cols % nf4::kBlock != 0 || w->rows % 16 != 0) return NF4_ERR_UNSUPPORTED;
+    if (w->rows == 0) continue;  // nothing to compute for an empty weight
+    if (ys[i] == nullptr) return NF4_ERR_INVALID_ARG;
+    if (!aligned(ys[i], 4)) return NF4_ERR_MISALIGNED;
+    packed[n] = w->packed;
+    rows[n] = w->rows;
+    y[n] = ys[i];
+    ++n;
+  }
+  if (n == 0 || ws[0]->cols == 0) return NF4_OK;
+  if (x == nullptr) return NF4_ERR_INVALID_ARG;
+  if (!aligned(x, 16)) return NF4_ERR_MISALIGNED;
+  DeviceInfo d;
+  nf4_status st = device_info(&d);
+  if (st != NF4_OK) return st;
+  return from_cuda(nf4::launch_gemv_group(packed, s, rows, n, ws[0]->cols, x, batch, y,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
 nf4_status nf4_gemm(const nf4_weight* w, const void* x, int64_t m, void* y, void* workspace, size_t workspace_bytes,
                     nf4_stream_t stream) {
   nf4::Scales s;

@@ -42,6 +42,16 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kStepK = 256;  // k per warp step (4 level-1 blocks)
+
+// up to kMaxGroup weights sharing cols, the scale kind and the input x; CTA b works on 16-row tile
+// b - tile_end[i - 1] of weight i, the first i with b < tile_end[i]
+struct GemvGroup {
+  const uint8_t* packed[kMaxGroup];
+  Scales s[kMaxGroup];
+  __nv_bfloat16* y[kMaxGroup];
+  int tile_end[kMaxGroup];
+  int count;
+};
 constexpr int kPairTableBytes = 256 * 32 * 8;  // fp32 code pairs, one copy per bank
 
 __constant__ float c_code_gemv[16] = NF4_CODE_INIT;
@@ -90,12 +100,27 @@ __device__ __forceinline__ void load_step(StepData& d, const uint8_t* __restrict
 
 template <int NT, bool kDQ, bool kTable>
 __global__ void __launch_bounds__(kWarps * 32, NT >= 4 ? 1 : 2)
-    gemv_kernel(const uint8_t* __restrict__ packed, Scales s, int64_t rows, int64_t cols,
-                const __nv_bfloat16* __restrict__ x, int batch, __nv_bfloat16* __restrict__ y) {
+    gemv_kernel(GemvGroup grp, int64_t cols, const __nv_bfloat16* __restrict__ x, int batch) {
   __shared__ float unit_lut[kDQ ? 256 : 1];
   __shared__ float red[kWarps][16][8 * NT];
   extern __shared__ __align__(16) uint8_t pair_table[];  // entry v of lane l at 256 v + 8 l
   pdl_launch_dependents();
+  // this CTA's weight of the group (every index below is a compile-time constant)
+  const uint8_t* __restrict__ packed = grp.packed[0];
+  Scales s = grp.s[0];
+  __nv_bfloat16* __restrict__ y = grp.y[0];
+  int tile0 = 0, tile1 = grp.tile_end[0];
+#pragma unroll
+  for (int i = 1; i < kMaxGroup; ++i)
+    if (i < grp.count && (int)blockIdx.x >= grp.tile_end[i - 1]) {
+      packed = grp.packed[i];
+      s = grp.s[i];
+      y = grp.y[i];
+      tile0 = grp.tile_end[i - 1];
+      tile1 = grp.tile_end[i];
+    }
+  const int tile = (int)blockIdx.x - tile0;
+  const int64_t rows = (int64_t)(tile1 - tile0) * 16;
   if (kDQ) unit_lut[threadIdx.x & 255] = dq_unit(threadIdx.x & 255, s.dq_code);
   if (kTable) {
 #pragma unroll
@@ -111,7 +136,7 @@ __global__ void __launch_bounds__(kWarps * 32, NT >= 4 ? 1 : 2)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
-  const int64_t row0 = (int64_t)blockIdx.x * 16 + g;
+  const int64_t row0 = (int64_t)tile * 16 + g;
   const int64_t nblk = cols / kBlock;
   const int64_t nsteps = (cols + kStepK - 1) / kStepK;
 
@@ -199,17 +224,14 @@ __global__ void __launch_bounds__(kWarps * 32, NT >= 4 ? 1 : 2)
     float sum = 0.0f;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) sum += red[w][r][b];
-    y[(int64_t)b * rows + (int64_t)blockIdx.x * 16 + r] = __float2bfloat16_rn(sum);
+    y[(int64_t)b * rows + (int64_t)tile * 16 + r] = __float2bfloat16_rn(sum);
   }
 }
 
 template <int NT>
-cudaError_t launch_nt(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x, int batch,
-                      void* y, cudaStream_t stream) {
-  const unsigned grid = (unsigned)(rows / 16);
+cudaError_t launch_nt(const GemvGroup& grp, int64_t cols, const void* x, int batch, bool dq, cudaStream_t stream) {
+  const unsigned grid = (unsigned)grp.tile_end[grp.count - 1];
   const auto* xb = static_cast<const __nv_bfloat16*>(x);
-  auto* yb = static_cast<__nv_bfloat16*>(y);
-  const bool dq = s.absmax == nullptr;
   cudaError_t e;
   if (NT == 1 && batch == 1) {  // decode at batch 1: the mixed decode with the 64 KB pair table
     // the table needs the shared-memory opt-in: set it once per device and variant
@@ -222,18 +244,25 @@ cudaError_t launch_nt(const uint8_t* packed, const Scales& s, int64_t rows, int6
       if (e != cudaSuccess) return e;
       attr_done[dq].fetch_or(1ull << dev);
     }
-    e = dq ? launch_pdl(gemv_kernel<NT, true, true>, dim3(grid), dim3(kWarps * 32), kPairTableBytes, stream, packed,
-                        s, rows, cols, xb, batch, yb)
-           : launch_pdl(gemv_kernel<NT, false, true>, dim3(grid), dim3(kWarps * 32), kPairTableBytes, stream, packed,
-                        s, rows, cols, xb, batch, yb);
+    e = dq ? launch_pdl(gemv_kernel<NT, true, true>, dim3(grid), dim3(kWarps * 32), kPairTableBytes, stream, grp,
+                        cols, xb, batch)
+           : launch_pdl(gemv_kernel<NT, false, true>, dim3(grid), dim3(kWarps * 32), kPairTableBytes, stream, grp,
+                        cols, xb, batch);
   } else {
-    e = dq ? launch_pdl(gemv_kernel<NT, true, false>, dim3(grid), dim3(kWarps * 32), 0, stream, packed, s, rows, cols,
-                        xb, batch, yb)
-           : launch_pdl(gemv_kernel<NT, false, false>, dim3(grid), dim3(kWarps * 32), 0, stream, packed, s, rows, cols,
-                        xb, batch, yb);
+    e = dq ? launch_pdl(gemv_kernel<NT, true, false>, dim3(grid), dim3(kWarps * 32), 0, stream, grp, cols, xb, batch)
+           : launch_pdl(gemv_kernel<NT, false, false>, dim3(grid), dim3(kWarps * 32), 0, stream, grp, cols, xb,
+                        batch);
   }
   count_launches(1);
   return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+cudaError_t launch_group(const GemvGroup& grp, int64_t cols, const void* x, int batch, bool dq,
+                         cudaStream_t stream) {
+  if (batch <= 8) return launch_nt<1>(grp, cols, x, batch, dq, stream);
+  if (batch <= 16) return launch_nt<2>(grp, cols, x, batch, dq, stream);
+  if (batch <= 32) return launch_nt<4>(grp, cols, x, batch, dq, stream);
+  return launch_nt<8>(grp, cols, x, batch, dq, stream);
 }
 
 }  // namespace
@@ -241,10 +270,33 @@ cudaError_t launch_nt(const uint8_t* packed, const Scales& s, int64_t rows, int6
 // batch <= 64: the activation rows are spread over ceil(batch / 8) n-tiles
 cudaError_t launch_gemv(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x, int batch,
                         void* y, cudaStream_t stream, int /*num_sms*/) {
-  if (batch <= 8) return launch_nt<1>(packed, s, rows, cols, x, batch, y, stream);
-  if (batch <= 16) return launch_nt<2>(packed, s, rows, cols, x, batch, y, stream);
-  if (batch <= 32) return launch_nt<4>(packed, s, rows, cols, x, batch, y, stream);
-  return launch_nt<8>(packed, s, rows, cols, x, batch, y, stream);
+  if (rows / 16 > INT32_MAX) return cudaErrorInvalidValue;
+  GemvGroup grp = {};
+  grp.packed[0] = packed;
+  grp.s[0] = s;
+  grp.y[0] = static_cast<__nv_bfloat16*>(y);
+  grp.tile_end[0] = (int)(rows / 16);
+  grp.count = 1;
+  return launch_group(grp, cols, x, batch, s.absmax == nullptr, stream);
+}
+
+// several weights with the same cols and scale kind, one input x: one launch whose CTAs cover the 16-row
+// tiles of every weight in turn
+cudaError_t launch_gemv_group(const uint8_t* const* packed, const Scales* s, const int64_t* rows, int count,
+                              int64_t cols, const void* x, int batch, void* const* y, cudaStream_t stream) {
+  if (count < 1 || count > kMaxGroup) return cudaErrorInvalidValue;
+  GemvGroup grp = {};
+  int64_t tiles = 0;
+  for (int i = 0; i < count; ++i) {
+    tiles += rows[i] / 16;
+    if (tiles > INT32_MAX) return cudaErrorInvalidValue;
+    grp.packed[i] = packed[i];
+    grp.s[i] = s[i];
+    grp.y[i] = static_cast<__nv_bfloat16*>(y[i]);
+    grp.tile_end[i] = (int)tiles;
+  }
+  grp.count = count;
+  return launch_group(grp, cols, x, batch, s[0].absmax == nullptr, stream);
 }
 
 }  // namespace nf4

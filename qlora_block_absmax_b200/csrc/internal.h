@@ -56,6 +56,11 @@ cudaError_t launch_dequantize(const uint8_t* packed, const Scales& s, int64_t n,
 cudaError_t launch_gemv(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x,
                         int batch, void* y, cudaStream_t stream, int num_sms);
 
+// several weights (same cols and scale kind) on one input in one launch, count <= kMaxGroup
+constexpr int kMaxGroup = 4;
+cudaError_t launch_gemv_group(const uint8_t* const* packed, const Scales* s, const int64_t* rows, int count,
+                              int64_t cols, const void* x, int batch, void* const* y, cudaStream_t stream);
+
 size_t gemm_workspace_bytes(int64_t rows, int64_t cols, int64_t m);
 cudaError_t launch_gemm(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x,
                         int64_t m, void* y, void* workspace, unsigned* err, cudaStream_t stream, int num_sms);

@@ -106,3 +106,51 @@ def test_device_query_without_gpu_is_safe(lib):
     if torch.cuda.is_available():
         pytest.skip("GPU present")
     assert lib.nf4_device_supported() == 0
+
+
+def test_host_validation_new_entry_points(lib):
+    """nf4_gemm_dx, nf4_gemm_lora and nf4_gemv_grouped reject bad arguments on the host, before any CUDA call"""
+    E = {v: k for k, v in _lib.STATUS_NAMES.items()}
+    s = None
+    w = weight(rows=128, cols=256)
+    # input gradient: rows % 64, cols % 128, m >= 0, alignment, workspace
+    assert lib.nf4_gemm_dx(ctypes.byref(weight(rows=96, cols=256)), 0x9000, 4, 0xa000, None, 0, s) == \
+        E["NF4_ERR_UNSUPPORTED"]
+    assert lib.nf4_gemm_dx(ctypes.byref(weight(rows=128, cols=192)), 0x9000, 4, 0xa000, None, 0, s) == \
+        E["NF4_ERR_UNSUPPORTED"]
+    assert lib.nf4_gemm_dx(ctypes.byref(w), 0x9000, -1, 0xa000, None, 0, s) == E["NF4_ERR_INVALID_ARG"]
+    assert lib.nf4_gemm_dx(ctypes.byref(w), 0x9000, 0, 0xa000, None, 0, s) == E["NF4_OK"]
+    assert lib.nf4_gemm_dx(ctypes.byref(w), 0x9004, 4, 0xa000, None, 0, s) == E["NF4_ERR_MISALIGNED"]
+    assert lib.nf4_gemm_dx(ctypes.byref(w), None, 4, 0xa000, None, 0, s) == E["NF4_ERR_INVALID_ARG"]
+    # adapter: r in {16, 32}, finite scale, workspace present and large enough
+    lo = _lib.NF4Lora(0xb000, 0xc000, 16, 2.0)
+    assert lib.nf4_gemm_lora(ctypes.byref(w), None, 0x9000, 4, 0xa000, 0xd000, 1 << 20, s) == E["NF4_ERR_INVALID_ARG"]
+    bad_r = _lib.NF4Lora(0xb000, 0xc000, 8, 2.0)
+    assert lib.nf4_gemm_lora(ctypes.byref(w), ctypes.byref(bad_r), 0x9000, 4, 0xa000, 0xd000, 1 << 20, s) == \
+        E["NF4_ERR_UNSUPPORTED"]
+    nan_s = _lib.NF4Lora(0xb000, 0xc000, 16, float("nan"))
+    assert lib.nf4_gemm_lora(ctypes.byref(w), ctypes.byref(nan_s), 0x9000, 4, 0xa000, 0xd000, 1 << 20, s) == \
+        E["NF4_ERR_INVALID_ARG"]
+    inf_s = _lib.NF4Lora(0xb000, 0xc000, 16, float("inf"))
+    assert lib.nf4_gemm_lora(ctypes.byref(w), ctypes.byref(inf_s), 0x9000, 4, 0xa000, 0xd000, 1 << 20, s) == \
+        E["NF4_ERR_INVALID_ARG"]
+    assert lib.nf4_gemm_lora(ctypes.byref(w), ctypes.byref(lo), 0x9000, 4, 0xa000, None, 0, s) == \
+        E["NF4_ERR_INVALID_ARG"]
+    unaligned = _lib.NF4Lora(0xb008, 0xc000, 16, 2.0)
+    assert lib.nf4_gemm_lora(ctypes.byref(w), ctypes.byref(unaligned), 0x9000, 4, 0xa000, 0xd000, 1 << 20, s) == \
+        E["NF4_ERR_MISALIGNED"]
+    assert lib.nf4_gemm_lora(ctypes.byref(w), ctypes.byref(lo), 0x9000, 0, 0xa000, None, 0, s) == E["NF4_OK"]
+    # grouped GEMV: 1..4 weights, equal cols and scale kind, batch 1..8
+    ws = (ctypes.POINTER(_lib.NF4Weight) * 5)(*[ctypes.pointer(weight()) for _ in range(5)])
+    ys = (ctypes.c_void_p * 5)(*[0xa000] * 5)
+    assert lib.nf4_gemv_grouped(ws, 0, 0x9000, 1, ys, s) == E["NF4_ERR_INVALID_ARG"]
+    assert lib.nf4_gemv_grouped(ws, 5, 0x9000, 1, ys, s) == E["NF4_ERR_INVALID_ARG"]
+    assert lib.nf4_gemv_grouped(ws, 2, 0x9000, 9, ys, s) == E["NF4_ERR_INVALID_ARG"]
+    mixed = (ctypes.POINTER(_lib.NF4Weight) * 2)(ctypes.pointer(weight(cols=128)), ctypes.pointer(weight(cols=256)))
+    assert lib.nf4_gemv_grouped(mixed, 2, 0x9000, 1, ys, s) == E["NF4_ERR_INVALID_ARG"]
+    kinds = (ctypes.POINTER(_lib.NF4Weight) * 2)(
+        ctypes.pointer(weight()), ctypes.pointer(weight(absmax=0, q=0x3000, scale=0x4000, mean=0x5000)))
+    assert lib.nf4_gemv_grouped(kinds, 2, 0x9000, 1, ys, s) == E["NF4_ERR_INVALID_ARG"]
+    odd = (ctypes.POINTER(_lib.NF4Weight) * 2)(ctypes.pointer(weight()), ctypes.pointer(weight(rows=40)))
+    assert lib.nf4_gemv_grouped(odd, 2, 0x9000, 1, ys, s) == E["NF4_ERR_UNSUPPORTED"]
+    assert lib.nf4_gemv_grouped(ws, 2, 0x9008, 1, ys, s) == E["NF4_ERR_MISALIGNED"]

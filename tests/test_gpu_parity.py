@@ -383,6 +383,37 @@ def test_gemm_scale_paths(cols, use_dq):
     check_matmul(y, oracle.matmul(p_ref, a_ref, rows, cols, x), f"gemm cols{cols} dq{use_dq}")
 
 
+# --------------------------------------------------------------------------- grouped GEMV (several weights, one input)
+
+@pytest.mark.parametrize("batch", [1, 4, 8])
+def test_gemv_grouped_qkv_matches_separate_and_oracle(batch):
+    """the q, k, v projections of one 8B-shaped layer (4096, 1024, 1024 rows x 4096) in one launch: each output
+    is bit-identical to its own nf4_gemv call (the same per-tile arithmetic) and within the matmul tolerance of
+    the oracle"""
+    cols = 4096
+    pairs = [quantized_pair(rows, cols, 180 + i, True) for i, rows in enumerate((4096, 1024, 1024))]
+    x = synth.activations((batch, cols), 183 + batch)
+    xd = dev_bf16(x)
+    ys = nf4.gemv_grouped([p[0] for p in pairs], xd)
+    for (qw, p_ref, a_ref), y in zip(pairs, ys):
+        assert torch.equal(y.view(torch.int16), nf4.gemv(qw, xd).view(torch.int16))
+        check_matmul(y, oracle.matmul(p_ref, a_ref, qw.rows, cols, x), f"grouped {qw.rows} b{batch}")
+
+
+@pytest.mark.parametrize("rows_list,use_dq", [((16,), True), ((48, 16, 64, 32), True), ((14336, 14336), True),
+                                              ((128, 4096, 16), False)])
+def test_gemv_grouped_shapes(rows_list, use_dq):
+    """one to four weights, single-tile and mixed sizes, plain and double-quantized scales (each weight
+    quantized with its own seed: its own mean and scales)"""
+    cols = 1024
+    pairs = [quantized_pair(rows, cols, 190 + 7 * i + rows // 16, use_dq) for i, rows in enumerate(rows_list)]
+    x = synth.activations((3, cols), 199)
+    ys = nf4.gemv_grouped([p[0] for p in pairs], dev_bf16(x))
+    for (qw, p_ref, a_ref), y in zip(pairs, ys):
+        check_matmul(y, oracle.matmul(p_ref, a_ref, qw.rows, cols, x), f"grouped {rows_list} {qw.rows}")
+    nf4.check_device_error()
+
+
 # --------------------------------------------------------------------------- 4-bit matmul + low-rank adapter
 
 def lora_maps(rows, cols, r, seed):
