@@ -34,7 +34,8 @@ ROWS, COLS, GEMV_B, GEMM_M = 4096, 4096, 1, 256
 WORKLOAD = "nf4_path_bf16_4096x4096_outliers_gemv1_gemm256"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNELS = ("quantize", "double_quant", "dequantize", "gemv", "gemm")
-NEXT_KERNELS = ("gemm_dx", "gemm_lora")  # timed beside the step, not part of it
+NEXT_KERNELS = ("gemm_dx", "gemm_lora", "gemv_grouped")  # timed beside the step, not part of it
+QKV_SHAPES = ((4096, 4096), (1024, 4096), (1024, 4096))  # q, k, v of an 8B-shaped layer
 LORA_R, LORA_ALPHA = 16, 32.0
 
 
@@ -53,6 +54,10 @@ def work_per_step(rows=ROWS, cols=COLS, b=GEMV_B, m=GEMM_M):
         "gemm": {"bytes": w4 + 2 * m * cols + 2 * m * rows, "flops": 2 * m * n},
         "gemm_dx": {"bytes": w4 + 2 * m * rows + 2 * m * cols, "flops": 2 * m * n,
                     "what": f"dX[{m},{cols}] = dY[{m},{rows}] . Wc (input gradient)"},
+        "gemv_grouped": {"bytes": sum(r * c // 2 + r * c // 64 + 4 * (r * c // 64 // 256) + 4 + 2 * b * c + 2 * b * r
+                                      for r, c in QKV_SHAPES),
+                         "flops": sum(2 * b * r * c for r, c in QKV_SHAPES), "bound": "hbm",
+                         "what": f"q, k, v of an 8B layer (4096/1024/1024 x 4096) on one x, batch {b}, one launch"},
         "gemm_lora": {"bytes": w4 + 2 * m * cols + 2 * m * rows + 2 * LORA_R * (rows + cols),
                       "flops": 2 * m * n + 2 * m * LORA_R * (rows + cols),
                       "what": f"Y[{m},{rows}] = X . Wc^T + 2 (X . A^T) . B^T, r = {LORA_R} (two launches)"},
@@ -210,6 +215,18 @@ def run_ours(args):
     class Copy:
         pass
 
+    # the q, k, v projections of one 8B-shaped layer for the grouped GEMV, drawn on the device (seeds 2000-2002,
+    # config-5 recipe) and quantized by the library at set-up; enough sets (13 MB of codes each) that successive
+    # launches read them cold from HBM
+    qkv_bytes = sum(r * c * 0.5159 for r, c in QKV_SHAPES)
+    qkv_sets = [[nf4.quantize_weight(synth.normal_weights_device(shape, 2000 + j, device=dev))
+                 for j, shape in enumerate(QKV_SHAPES)] for _ in range(max(copies, -(-3 * l2 // int(qkv_bytes))))]
+    qkv_turn = [0]
+
+    def next_qkv():
+        qkv_turn[0] += 1
+        return qkv_sets[qkv_turn[0] % len(qkv_sets)]
+
     cs = []
     for _ in range(copies):
         c = Copy()
@@ -234,6 +251,7 @@ def run_ours(args):
         c.down, c.up = host_down.to(dev), host_up.to(dev)
         c.Yl = torch.empty(GEMM_M, ROWS, dtype=torch.bfloat16, device=dev)
         c.lws = torch.zeros(nf4.gemm_lora_workspace_bytes(c.qw, GEMM_M), dtype=torch.uint8, device=dev)
+        c.qkv_y = [torch.empty(GEMV_B, r, dtype=torch.bfloat16, device=dev) for r, _ in QKV_SHAPES]
         cs.append(c)
     stream = torch.cuda.current_stream()
 
@@ -249,7 +267,8 @@ def run_ours(args):
         """products beyond the step's five calls, timed on their own: the input gradient dX = dY . Wc and the
         GEMM with an r = 16 adapter"""
         return (lambda: nf4.gemm_dx(c.qw, c.dY, out=c.dX, workspace=c.dws),
-                lambda: nf4.gemm_lora(c.qw, c.X, c.down, c.up, LORA_ALPHA / LORA_R, out=c.Yl, workspace=c.lws))
+                lambda: nf4.gemm_lora(c.qw, c.X, c.down, c.up, LORA_ALPHA / LORA_R, out=c.Yl, workspace=c.lws),
+                lambda: nf4.gemv_grouped(next_qkv(), c.x, outs=c.qkv_y))
 
     def step(c):
         for f in calls(c):
@@ -407,12 +426,16 @@ def run_ours(args):
     nexts = {}
     for k in NEXT_KERNELS:
         t = next_ms[k] / args.steps * 1e-3
-        ach = work[k]["flops"] / t / 1e12
-        nexts[k] = {"what": work[k]["what"], "ms": round(t * 1e3, 5), "gbs": round(work[k]["bytes"] / t / 1e9, 1),
-                    "tflops": round(ach, 2), "roofline": {"bound": "tensor", "achieved": round(ach, 2),
-                                                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                                                          "frac": round(ach / peaks["bf16_tflops"], 4),
-                                                          "traffic": TRAFFIC.get(k)}}
+        gbs = work[k]["bytes"] / t / 1e9
+        tfl = work[k]["flops"] / t / 1e12
+        if work[k].get("bound") == "hbm":
+            roof_k = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                      "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": TRAFFIC.get(k)}
+        else:
+            roof_k = {"bound": "tensor", "achieved": round(tfl, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                      "frac": round(tfl / peaks["bf16_tflops"], 4), "traffic": TRAFFIC.get(k)}
+        nexts[k] = {"what": work[k]["what"], "ms": round(t * 1e3, 5), "gbs": round(gbs, 1), "tflops": round(tfl, 2),
+                    "roofline": roof_k}
     dom = max(KERNELS, key=lambda k: per_kernel_ms[k])
     t_dom = per_kernel_ms[dom] / args.steps * 1e-3
     if dom == "gemm":
