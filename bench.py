@@ -139,7 +139,7 @@ def oracle_sample_step(sample_rows: int, w_bits, x_bits, X_bits):
 def cpu_baseline(sample_rows: int, reps: int = 1):
     import oracle
     from qlora_block_absmax_b200 import synth
-    w = synth.config2_weight()
+    w = synth.bf16_4096x4096_outlier_weight()
     x = synth.activations((GEMV_B, COLS), 1013)
     X = synth.activations((GEMM_M, COLS), 1277)
     oracle.build()
@@ -191,7 +191,7 @@ def run_ours(args):
     dev = torch.device("cuda", local)
 
     # ---- inputs (identical values in every copy; distinct memory)
-    w_bits = synth.config2_weight()
+    w_bits = synth.bf16_4096x4096_outlier_weight()
     x_bits = synth.activations((GEMV_B, COLS), 1013)
     X_bits = synth.activations((GEMM_M, COLS), 1277)
     dY_bits = synth.activations((GEMM_M, ROWS), 1279)  # gradient of Y for the input-gradient product
@@ -216,7 +216,7 @@ def run_ours(args):
         pass
 
     # the q, k, v projections of one 8B-shaped layer for the grouped GEMV, drawn on the device (seeds 2000-2002,
-    # config-5 recipe) and quantized by the library at set-up; enough sets (13 MB of codes each) that successive
+    # the whole-model recipe) and quantized by the library at set-up; enough sets (13 MB of codes each) that successive
     # launches read them cold from HBM
     qkv_bytes = sum(r * c * 0.5159 for r, c in QKV_SHAPES)
     qkv_sets = [[nf4.quantize_weight(synth.normal_weights_device(shape, 2000 + j, device=dev))
@@ -495,7 +495,7 @@ def run_reference(args):
     import oracle
     from qlora_block_absmax_b200 import synth
     oracle.build()
-    w = synth.config2_weight()
+    w = synth.bf16_4096x4096_outlier_weight()
     x = synth.activations((GEMV_B, COLS), 1013)
     X = synth.activations((GEMM_M, COLS), 1277)
     rows = args.ref_rows

@@ -65,12 +65,12 @@ def activations(shape, seed: int) -> np.ndarray:
     return f32_to_bf16_bits(rng(seed).standard_normal(shape).astype(np.float32))
 
 
-def config1_weight() -> np.ndarray:
+def fp32_1024x1024_weight() -> np.ndarray:
     """fp32 1024x1024 ~N(0, 0.02), seed 1001 (round-trip case)."""
     return normal_weights((1024, 1024), 1001)
 
 
-def config2_weight() -> np.ndarray:
+def bf16_4096x4096_outlier_weight() -> np.ndarray:
     """bf16 4096x4096 ~N(0, 0.02) with 0.1% x20 outliers (seeds 1002, 1003)."""
     w = add_outliers(normal_weights((4096, 4096), 1002), 1003)
     return f32_to_bf16_bits(w)

@@ -105,10 +105,10 @@ def test_quantize_special_blocks(dtype):
     assert np.array_equal(p.cpu().numpy(), p_ref)
 
 
-def test_quantize_config1_roundtrip():
+def test_quantize_fp32_1024x1024_roundtrip():
     """fp32 1024x1024 ~N(0,0.02): codes, absmax, fp32 dequantization and
     re-quantization all bit-exact."""
-    w = synth.config1_weight().reshape(-1)
+    w = synth.fp32_1024x1024_weight().reshape(-1)
     p_ref, a_ref = oracle.quantize(w)
     p, a = nf4.quantize(dev(w))
     assert np.array_equal(p.cpu().numpy(), p_ref)
@@ -119,25 +119,25 @@ def test_quantize_config1_roundtrip():
     assert np.array_equal(wh.cpu().numpy().reshape(-1).view(np.uint32), wh_ref.view(np.uint32))
     p2, a2 = nf4.quantize(wh.reshape(-1))
     assert np.array_equal(p2.cpu().numpy(), p_ref) and np.array_equal(a2.cpu().numpy(), a_ref)
-    print(f"config1: near-midpoint elements {near_threshold_count(w, a_ref)}")
+    print(f"fp32 1024x1024: near-midpoint elements {near_threshold_count(w, a_ref)}")
 
 
-def test_quantize_config2_bf16_outliers():
-    bits = synth.config2_weight().reshape(-1)
+def test_quantize_bf16_4096x4096_outliers():
+    bits = synth.bf16_4096x4096_outlier_weight().reshape(-1)
     p_ref, a_ref = oracle.quantize(bits)
     p, a = nf4.quantize(dev_bf16(bits))
     assert np.array_equal(a.cpu().numpy(), a_ref)
     assert np.array_equal(p.cpu().numpy(), p_ref)
-    print(f"config2: near-midpoint elements {near_threshold_count(synth.bf16_bits_to_f32(bits), a_ref)}")
+    print(f"bf16 4096x4096: near-midpoint elements {near_threshold_count(synth.bf16_bits_to_f32(bits), a_ref)}")
 
 
 # --------------------------------------------------------------------------- double quant
 
 def dq_cases():
     r = synth.rng(99)
-    _, a2 = oracle.quantize(synth.config2_weight().reshape(-1))
+    _, a2 = oracle.quantize(synth.bf16_4096x4096_outlier_weight().reshape(-1))
     return {
-        "config2": a2,
+        "bf16_4096_outliers": a2,
         "one": np.array([0.3], np.float32),
         "255": np.abs(r.standard_normal(255)).astype(np.float32),
         "257": np.abs(r.standard_normal(257)).astype(np.float32),
@@ -165,8 +165,8 @@ def test_double_quant_workspace_reused():
     every call leaves its barrier and exact-sum buffers ready for the next, so each result is exact"""
     cases = dq_cases()
     ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
-    for name, code in [("config2", "e4m3"), ("one", "int8"), ("wide", "e4m3"), ("257", "int8"),
-                       ("config2", "int8"), ("signed", "e4m3"), ("zeros_and_tiny", "e4m3"), ("config2", "e4m3")]:
+    for name, code in [("bf16_4096_outliers", "e4m3"), ("one", "int8"), ("wide", "e4m3"), ("257", "int8"),
+                       ("bf16_4096_outliers", "int8"), ("signed", "e4m3"), ("zeros_and_tiny", "e4m3"), ("bf16_4096_outliers", "e4m3")]:
         a = cases[name]
         c = oracle.DQ_E4M3 if code == "e4m3" else oracle.DQ_INT8
         q_ref, s_ref, m_ref = oracle.double_quant(a, 256, c)
@@ -198,8 +198,8 @@ def test_dequantize_bit_exact(use_dq, code, out, rows, cols):
         assert np.array_equal(host_bf16_bits(got).reshape(-1), ref)
 
 
-def test_dequantize_config2_double_quant_bf16():
-    bits = synth.config2_weight()
+def test_dequantize_bf16_4096x4096_double_quant():
+    bits = synth.bf16_4096x4096_outlier_weight()
     qw = nf4.quantize_weight(dev_bf16(bits), use_double_quant=True, code="e4m3")
     p_ref, a_ref = oracle.quantize(bits.reshape(-1))
     q_ref, s_ref, m_ref = oracle.double_quant(a_ref, 256, oracle.DQ_E4M3)
@@ -234,7 +234,7 @@ def test_gemv_small(rows, cols, batch, use_dq):
 
 @pytest.mark.parametrize("shape", [(4096, 4096), (14336, 4096), (4096, 14336), (1024, 4096)])
 @pytest.mark.parametrize("batch", [1, 4, 8])
-def test_gemv_config3_shapes(shape, batch):
+def test_gemv_llama8b_shapes(shape, batch):
     rows, cols = shape
     qw, p_ref, a_ref = quantized_pair(rows, cols, 1010 + rows // 1024 + cols // 1024, True)
     x = synth.activations((batch, cols), 1013)
@@ -307,7 +307,7 @@ def test_gemm_small(m):
 
 
 @pytest.mark.parametrize("m", [16, 64, 256, 1024, 4096])
-def test_gemm_config4_sampled(m):
+def test_gemm_14336x4096_sampled(m):
     """W 14336x4096 NF4+DQ, X [m, 4096]: 2048 sampled outputs against the oracle,
     plus every output of the first activation row."""
     rows, cols = 14336, 4096
@@ -495,7 +495,7 @@ def test_gemm_lora_adapter_only():
 
 
 @pytest.mark.parametrize("m", [16, 256, 1024, 4096])
-def test_gemm_lora_config4_sampled(m):
+def test_gemm_lora_14336x4096_sampled(m):
     """W 14336x4096 NF4+DQ with an r = 16, alpha = 32 adapter at the prefill sizes: 2048 sampled outputs and
     all of row 0 against the oracle; ten identical calls give identical bits"""
     rows, cols, r = 14336, 4096, 16
@@ -623,9 +623,9 @@ def test_gemm_dx_adjoint_of_gemm():
     assert abs(float(t1.sum()) - float(t2.sum())) <= 2.0 ** -6 * scale
 
 
-# --------------------------------------------------------------------------- whole model (config 5)
+# --------------------------------------------------------------------------- whole 8B-shaped model
 
-def test_whole_model_8b_config5():
+def test_whole_model_8b():
     """An 8B-shaped decoder stack: 32 layers x (q, k, v, o, gate, up, down), 6.98e9 bf16 weights ~N(0, 0.02), each
     matrix from its own seed, quantized to NF4 with E4M3 double quant on the GPU, then a GEMV pass over all 224
     matrices in layer order at batch 1, 4 and 8.  One matrix of each projection type (from different layers) is
