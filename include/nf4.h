@@ -217,9 +217,10 @@ NF4_API nf4_status nf4_gemm_lora(const nf4_weight *w, const nf4_lora *lora, cons
 NF4_API size_t nf4_gemm_lora_workspace_bytes(const nf4_weight *w, int64_t m);
 
 /* Input gradient of nf4_gemm, for training adapters on a frozen 4-bit base
- * ([bnb-tools] "Strengths and limitations": the quantized weights receive no
- * gradient, but the gradient flows through them to the adapters; [bnb-tut]
- * "QLoRA: Fine-Tuning a 4-bit Model": the 4-bit base stays frozen):
+ * ([bnb-tools] "Strengths and limitations": the quantized weights are not
+ * trained, yet the loss gradient must pass through them to reach the
+ * adapters; [bnb-tut] "QLoRA: Fine-Tuning a 4-bit Model": only the adapters
+ * train, the 4-bit base is fixed):
  *   dX[m, k] = bf16_rn( sum_n dY[m, n] * Wc[n, k] ),  Wc as in nf4_gemv,
  * on tcgen05 tensor cores, accumulated in fp32 (order unspecified).  The
  * packed weight is read in its stored [rows, cols] layout; no transposed copy

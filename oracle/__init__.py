@@ -74,6 +74,12 @@ def _load():
         "oracle_lora_down": (None, [P, I64, I64, P, I32, ctypes.c_float, P]),
         "oracle_nf4_matmul_lora": (None, [P, P, I64, I64, I32, P, I64, P, P, I32, ctypes.c_float, P]),
         "oracle_nf4_matmul_lora_sampled": (None, [P, P, I64, I64, I32, P, P, P, I32, P, P, I64, P]),
+        "oracle_fp4_codebook": (None, [P, P]),
+        "oracle_fp4_nearest_code": (ctypes.c_int, [ctypes.c_float]),
+        "oracle_fp4_quantize_f32": (None, [P, I64, I32, P, P]),
+        "oracle_fp4_quantize_bf16": (None, [P, I64, I32, P, P]),
+        "oracle_fp4_dequantize_f32": (None, [P, P, I64, I32, P]),
+        "oracle_fp4_dequantize_bf16": (None, [P, P, I64, I32, P]),
         "oracle_set_threads": (None, [ctypes.c_int]),
         "oracle_get_threads": (ctypes.c_int, []),
     }
@@ -278,3 +284,47 @@ def matmul_lora_sampled(packed: np.ndarray, absmax: np.ndarray, N: int, K: int, 
                                            _p(np.ascontiguousarray(absmax, dtype=np.float32)), N, K, blocksize,
                                            _p(x), _p(t), _p(Bu), r, _p(bs), _p(ns), bs.size, _p(y))
     return y
+
+
+# ---------------------------------------------------------------- FP4 (E2M1 / 6, stored as the bit pattern)
+
+def fp4_codebook():
+    """(fp64 levels, fp32 levels) indexed by the 4-bit pattern s e1 e0 m."""
+    c64 = np.zeros(16, np.float64)
+    c32 = np.zeros(16, np.float32)
+    _load().oracle_fp4_codebook(_p(c64), _p(c32))
+    return c64, c32
+
+
+def fp4_nearest_code(x: float) -> int:
+    return int(_load().oracle_fp4_nearest_code(float(x)))
+
+
+def fp4_quantize(w: np.ndarray, blocksize: int = 64):
+    """w: float32, or uint16 bf16 bit patterns -> (packed u8, absmax f32), FP4 codes."""
+    w = np.ascontiguousarray(w).reshape(-1)
+    n = w.size
+    packed = np.zeros((n + 1) // 2, np.uint8)
+    absmax = np.zeros((n + blocksize - 1) // blocksize, np.float32)
+    if w.dtype == np.float32:
+        _load().oracle_fp4_quantize_f32(_p(w), n, blocksize, _p(packed), _p(absmax))
+    elif w.dtype == np.uint16:
+        _load().oracle_fp4_quantize_bf16(_p(w), n, blocksize, _p(packed), _p(absmax))
+    else:
+        raise TypeError("fp4_quantize takes float32 or bf16 bit patterns (uint16)")
+    return packed, absmax
+
+
+def fp4_dequantize(packed: np.ndarray, absmax: np.ndarray, n: int, blocksize: int = 64,
+                   out_dtype: str = "f32") -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    absmax = np.ascontiguousarray(absmax, dtype=np.float32)
+    if out_dtype == "f32":
+        out = np.zeros(n, np.float32)
+        _load().oracle_fp4_dequantize_f32(_p(packed), _p(absmax), n, blocksize, _p(out))
+    elif out_dtype == "bf16":
+        out = np.zeros(n, np.uint16)
+        _load().oracle_fp4_dequantize_bf16(_p(packed), _p(absmax), n, blocksize, _p(out))
+    else:
+        raise ValueError(out_dtype)
+    return out

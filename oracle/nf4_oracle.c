@@ -40,8 +40,8 @@ int oracle_get_threads(void) {
 /* ------------------------------------------------------------------------- */
 /* NF4 code book.                                                             */
 /*                                                                            */
-/* [bnb-tools] "How NF4 works": the 16 code values are placed so that each    */
-/* covers an equal share of the bell curve of normally distributed weights.   */
+/* [bnb-tools] "How NF4 works": the 16 levels split the normal distribution  */
+/* of the weights into pieces of equal probability.                          */
 /* [bnb-tut] "How NF4 Works": a grid for normally distributed data, levels    */
 /* densest near zero.  The QLoRA construction read here: quantiles of N(0,1)  */
 /* taken at equally spaced probabilities, 8 on the positive side and 7 on the */
@@ -419,8 +419,9 @@ void oracle_nf4_matmul_sampled(const uint8_t *packed, const float *absmax, int64
 /* ------------------------------------------------------------------------- */
 /* Input gradient of the same matmul.  [bnb-tools] "Strengths and            */
 /* limitations" (Limitations) and [bnb-tut] "QLoRA: Fine-Tuning a 4-bit       */
-/* Model": the 4-bit base weight stays frozen and receives no gradient of its */
-/* own, but the gradient passes through it to the adapters and layers below: */
+/* Model": the 4-bit base weight is not trained (it gets no gradient of its  */
+/* own), yet the loss gradient has to pass through it to reach the adapters  */
+/* and the layers below:                                                      */
 /* dx[b,k] = sum_n dy[b,n] * Wc[n,k], with Wc the same 16-bit expanded weight */
 /* as above.  Products of two bf16 values are exact in fp64; summed in fp64   */
 /* over n in ascending order.                                                 */
@@ -504,4 +505,96 @@ void oracle_nf4_matmul_lora_sampled(const uint8_t *packed, const float *absmax, 
 #pragma omp parallel for schedule(static)
   for (int64_t i = 0; i < count; ++i)
     y[i] = dot_row(packed, absmax, K, blocksize, ns[i], x + bs[i] * K) + lora_term(t + bs[i] * r, Bup, ns[i], r);
+}
+
+/* ------------------------------------------------------------------------- */
+/* FP4 variant of the 4-bit code: [bnb-tools] "Glossary" (the FP4 entry) and */
+/* "What it is" (4-bit linear layers in either format); [env-tf]             */
+/* "Description".  The pages name the type but give no layout.  Reading: the */
+/* OCP E2M1 format (sign, 2 exponent bits with bias 1, 1 mantissa bit, no     */
+/* infinities or NaN), magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6, divided by 6 so */
+/* that the block absmax maps to +-1 as with NF4.  The stored 4-bit value is  */
+/* the E2M1 bit pattern s e1 e0 m itself.  Blocking, absmax, packing and      */
+/* double quantization are those of NF4.                                      */
+/* ------------------------------------------------------------------------- */
+
+void oracle_fp4_codebook(double *c64, float *c32) {
+  for (int nib = 0; nib < 16; ++nib) {
+    int s = nib >> 3, e = (nib >> 1) & 3, m = nib & 1;
+    double mag = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1); /* subnormal when e == 0 */
+    double v = (s ? -mag : mag) / 6.0;
+    c64[nib] = v;
+    c32[nib] = (float)v;
+  }
+}
+
+static float g_fp4[16];
+static int g_fp4_ready = 0;
+
+static const float *fp4_codebook32(void) {
+  if (!g_fp4_ready) {
+    double c64[16];
+    oracle_fp4_codebook(c64, g_fp4);
+    g_fp4_ready = 1;
+  }
+  return g_fp4;
+}
+
+/* Nearest FP4 level of x (the fp32 levels, distance in exact arithmetic); a tie
+ * goes to the level with an even mantissa bit (the format's round-half-even);
+ * a result of zero keeps the sign of x (-0 is pattern 8). */
+int oracle_fp4_nearest_code(float x) {
+  const float *c = fp4_codebook32();
+  int neg = signbit(x) ? 1 : 0;
+  double ax = fabs((double)x);
+  int best = 0; /* magnitude pattern 0..7 (levels c[0..7] ascend) */
+  double bd = ax - (double)c[0];
+  for (int k = 1; k < 8; ++k) {
+    double d = fabs(ax - (double)c[k]);
+    if (d < bd || (d == bd && (k & 1) == 0)) { bd = d; best = k; }
+  }
+  return (neg << 3) | best;
+}
+
+void oracle_fp4_quantize_f32(const float *w, int64_t n, int32_t blocksize, uint8_t *packed, float *absmax) {
+  int64_t nb = (n + blocksize - 1) / blocksize;
+  uint8_t *idx = (uint8_t *)malloc((size_t)(n > 0 ? n : 1));
+  (void)fp4_codebook32();
+#pragma omp parallel for schedule(static)
+  for (int64_t b = 0; b < nb; ++b) {
+    int64_t lo = b * blocksize, hi = lo + blocksize < n ? lo + blocksize : n;
+    float a = 0.0f;
+    for (int64_t i = lo; i < hi; ++i) a = fabsf(w[i]) > a ? fabsf(w[i]) : a;
+    absmax[b] = a;
+    for (int64_t i = lo; i < hi; ++i) {
+      if (a == 0.0f) { idx[i] = 0; continue; } /* all-zero block: every value is +0 */
+      idx[i] = (uint8_t)oracle_fp4_nearest_code(w[i] / a);
+    }
+  }
+  for (int64_t j = 0; j < (n + 1) / 2; ++j) {
+    uint8_t hi4 = idx[2 * j];
+    uint8_t lo4 = (2 * j + 1 < n) ? idx[2 * j + 1] : 0; /* an odd tail's partner is +0 */
+    packed[j] = (uint8_t)((hi4 << 4) | lo4);
+  }
+  free(idx);
+}
+
+void oracle_fp4_quantize_bf16(const uint16_t *w, int64_t n, int32_t blocksize, uint8_t *packed, float *absmax) {
+  float *wf = (float *)malloc((size_t)(n > 0 ? n : 1) * sizeof(float));
+  for (int64_t i = 0; i < n; ++i) wf[i] = oracle_bf16_to_f32(w[i]);
+  oracle_fp4_quantize_f32(wf, n, blocksize, packed, absmax);
+  free(wf);
+}
+
+void oracle_fp4_dequantize_f32(const uint8_t *packed, const float *absmax, int64_t n, int32_t blocksize, float *out) {
+  const float *c = fp4_codebook32();
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i) out[i] = c[code_at(packed, i)] * absmax[i / blocksize];
+}
+
+void oracle_fp4_dequantize_bf16(const uint8_t *packed, const float *absmax, int64_t n, int32_t blocksize,
+                                uint16_t *out) {
+  const float *c = fp4_codebook32();
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i) out[i] = oracle_bf16_rn(c[code_at(packed, i)] * absmax[i / blocksize]);
 }

@@ -111,6 +111,18 @@ void oracle_nf4_matmul_lora_sampled(const uint8_t *packed, const float *absmax, 
                                     int32_t blocksize, const uint16_t *x, const double *t, const uint16_t *Bup,
                                     int32_t r, const int64_t *bs, const int64_t *ns, int64_t count, double *y);
 
+/* FP4 (OCP E2M1 values / 6, indexed by the 4-bit pattern s e1 e0 m): code
+ * book, nearest code (ties to an even mantissa bit, zero keeps the sign of x),
+ * blockwise quantization (all-zero block and odd-tail partner: +0) and
+ * dequantization; blocking, absmax and packing as for NF4. */
+void oracle_fp4_codebook(double *c64, float *c32);
+int oracle_fp4_nearest_code(float x);
+void oracle_fp4_quantize_f32(const float *w, int64_t n, int32_t blocksize, uint8_t *packed, float *absmax);
+void oracle_fp4_quantize_bf16(const uint16_t *w, int64_t n, int32_t blocksize, uint8_t *packed, float *absmax);
+void oracle_fp4_dequantize_f32(const uint8_t *packed, const float *absmax, int64_t n, int32_t blocksize, float *out);
+void oracle_fp4_dequantize_bf16(const uint8_t *packed, const float *absmax, int64_t n, int32_t blocksize,
+                                uint16_t *out);
+
 /* Worker threads used by the loops marked parallel (0 = OpenMP default). */
 void oracle_set_threads(int n);
 int oracle_get_threads(void);

@@ -474,3 +474,84 @@ def test_lora_sum_of_parts():
     assert np.allclose(y, oracle.matmul(p, a, N, K, x) + adapter, rtol=1e-13, atol=1e-12)
     bs, ns = np.array([0, 3, 2, 1, 3]), np.array([0, 63, 17, 40, 5])
     assert np.array_equal(oracle.matmul_lora_sampled(p, a, N, K, x, A, B, r, 2.0, bs, ns), y[bs, ns])
+
+
+# ---------------------------------------------------------------- FP4 variant (E2M1 / 6, stored as the bit pattern)
+
+# OCP microscaling spec, FP4 E2M1: the value of each 3-bit magnitude pattern e1 e0 m (bias 1, subnormals at e = 0)
+E2M1_SPEC = {0b000: 0.0, 0b001: 0.5, 0b010: 1.0, 0b011: 1.5, 0b100: 2.0, 0b101: 3.0, 0b110: 4.0, 0b111: 6.0}
+
+
+def test_fp4_codebook_is_the_e2m1_table_over_6():
+    c64, c32 = oracle.fp4_codebook()
+    for nib in range(16):
+        v = E2M1_SPEC[nib & 7] / 6.0 * (-1.0 if nib & 8 else 1.0)
+        assert c64[nib] == v and c32[nib] == np.float32(v)
+        assert math.copysign(1.0, c64[nib]) == (-1.0 if nib & 8 else 1.0)  # pattern 8 is -0
+
+
+def _fp4_brute(x: float) -> int:
+    """exact nearest of the fp32 levels by rational arithmetic; tie -> even mantissa bit; sign of x kept"""
+    _, c32 = oracle.fp4_codebook()
+    ax = abs(Fraction(float(x)))
+    best, bd = None, None
+    for k in range(8):
+        d = abs(ax - Fraction(float(c32[k])))
+        if bd is None or d < bd or (d == bd and k % 2 == 0):
+            best, bd = k, d
+    return best | (8 if math.copysign(1.0, x) < 0 else 0)
+
+
+def test_fp4_nearest_code_brute_force():
+    _, c32 = oracle.fp4_codebook()
+    xs = [0.0, -0.0, 1.0, -1.0, 1e-30, -1e-30]
+    for k in range(8):  # every level, its neighbours in fp32, and every midpoint with its neighbours
+        lv = np.float32(c32[k])
+        xs += [float(lv), float(np.nextafter(lv, np.float32(2))), float(np.nextafter(lv, np.float32(-2)))]
+        if k < 7:
+            mid = (Fraction(float(c32[k])) + Fraction(float(c32[k + 1]))) / 2
+            m32 = np.float32(float(mid))
+            for v in (m32, np.nextafter(m32, np.float32(2)), np.nextafter(m32, np.float32(-2))):
+                xs += [float(v), -float(v)]
+    xs += list(synth.rng(91).uniform(-1, 1, 4000).astype(np.float32).astype(float))
+    for x in xs:
+        assert oracle.fp4_nearest_code(x) == _fp4_brute(x), x
+    # the one exactly representable midpoint (half of the fp32 level 1/12) ties to zero, keeping the sign
+    half = float(np.float32(c32[1]) / np.float32(2))
+    assert oracle.fp4_nearest_code(half) == 0 and oracle.fp4_nearest_code(-half) == 8
+
+
+def test_fp4_quantize_block_rules_and_round_trip():
+    w = synth.normal_weights((64 * 40 + 17,), 92)
+    w[64:128] = 0.0                # all-zero block -> +0 codes, absmax 0
+    w[128:192] = -0.0
+    w[200] = -0.0                  # a signed zero inside a normal block keeps its sign
+    p, a = oracle.fp4_quantize(w, 64)
+    codes = np.stack([p >> 4, p & 15], axis=1).reshape(-1)[:w.size]
+    assert np.all(codes[64:192] == 0) and a[1] == 0 and a[2] == 0
+    assert codes[200] == 8
+    blocks = [(b * 64, min(b * 64 + 64, w.size)) for b in range(len(a))]
+    for b, (lo, hi) in enumerate(blocks):  # the block's largest magnitude maps to +-1 (pattern 7 or 15)
+        if a[b] > 0:
+            j = lo + int(np.argmax(np.abs(w[lo:hi])))
+            assert codes[j] == (15 if w[j] < 0 else 7)
+    assert (p[-1] & 15) == 0  # odd tail: the partner is +0
+    for i in range(0, w.size, 37):  # brute force on the same inputs
+        if a[i // 64] > 0:
+            assert codes[i] == _fp4_brute(float(np.float32(w[i]) / np.float32(a[i // 64])))
+    # dequantize(quantize) is a fixed point: quantizing the dequantized tensor gives the same codes and scales
+    d = oracle.fp4_dequantize(p, a, w.size, 64, "f32")
+    p2, a2 = oracle.fp4_quantize(d, 64)
+    assert np.array_equal(p2, p) and np.array_equal(a2, a)
+    _, c32 = oracle.fp4_codebook()
+    assert np.array_equal(d, (c32[codes] * np.repeat(a, 64)[:w.size]).astype(np.float32))
+
+
+def test_fp4_bf16_input_and_output():
+    bits = synth.normal_weights((64 * 8,), 93, dtype="bf16")
+    p, a = oracle.fp4_quantize(bits, 64)
+    pf, af = oracle.fp4_quantize(synth.bf16_bits_to_f32(bits), 64)
+    assert np.array_equal(p, pf) and np.array_equal(a, af)  # widening bf16 to fp32 is exact
+    d16 = oracle.fp4_dequantize(p, a, bits.size, 64, "bf16")
+    d32 = oracle.fp4_dequantize(p, a, bits.size, 64, "f32")
+    assert np.array_equal(d16, synth.f32_to_bf16_bits(d32))
