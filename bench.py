@@ -12,6 +12,10 @@ independent copies that every step's working set is cold in the 126 MB L2.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
+Beside the step (each timed from its own graph, not part of `value`): the
+input gradient dX = dY . Wc (M = 256), the GEMM with an r = 16 adapter, and the
+grouped GEMV over the q/k/v projections of an 8B-shaped layer (batch 1).
+
 With N > 1 (torchrun, one process per GPU) every rank runs its own replica
 (the path has no cross-GPU exchange); value = all ranks' bytes / max time.
 Prints one JSON line on rank 0.

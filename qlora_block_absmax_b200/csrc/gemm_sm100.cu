@@ -21,6 +21,13 @@
 //   warp 12     TMA producer: activation tile (256 x 64 bf16, 128B swizzle)
 //   warp 13     TMEM allocator and MMA issuer (one elected thread)
 //   warp 14     TMA producer: packed codes and 16-byte scale chunks
+// With a low-rank adapter (QLoRA: "bitsandbytes quantization tutorial",
+// "QLoRA: Fine-Tuning a 4-bit Model") each output tile runs one more stage:
+// the producers put [B | B] rows of the up map in the TMEM slot, the TMA warp
+// loads the down map's [hi | lo] rows (lora_down.cu) in place of an activation
+// tile, and the MMA reduces over 2r, so the adapter lands in the same
+// accumulator.  The descriptors, MMA wrappers, work split and epilogue shared
+// with the input-gradient kernel live in umma.cuh.
 // Every mbarrier wait is bounded; on timeout the device error word is set and
 // the roles leave their loops, so a fault cannot hang the GPU.
 #include <cuda.h>

@@ -31,6 +31,10 @@
 // larger batches decode both rows with byte permutes.
 // Partial sums of the 8 warps are added in a fixed order through shared
 // memory, so results are deterministic.
+// One launch may cover up to four weights that read the same x (q/k/v or
+// gate/up of a decoder layer): the grid is the concatenation of their 16-row
+// tiles and each CTA picks its weight from the cumulative tile counts, so
+// small projections share the GPU with large ones instead of leaving SMs idle.
 #include <atomic>
 
 #include "nf4_common.cuh"
