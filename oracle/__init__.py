@@ -80,6 +80,7 @@ def _load():
         "oracle_fp4_quantize_bf16": (None, [P, I64, I32, P, P]),
         "oracle_fp4_dequantize_f32": (None, [P, P, I64, I32, P]),
         "oracle_fp4_dequantize_bf16": (None, [P, P, I64, I32, P]),
+        "oracle_fp4_matmul": (None, [P, P, I64, I64, I32, P, I64, P]),
         "oracle_set_threads": (None, [ctypes.c_int]),
         "oracle_get_threads": (ctypes.c_int, []),
     }
@@ -328,3 +329,14 @@ def fp4_dequantize(packed: np.ndarray, absmax: np.ndarray, n: int, blocksize: in
     else:
         raise ValueError(out_dtype)
     return out
+
+
+def fp4_matmul(packed: np.ndarray, absmax: np.ndarray, N: int, K: int, x_bf16: np.ndarray,
+               blocksize: int = 64) -> np.ndarray:
+    """x_bf16: uint16 [B, K] -> fp64 y [B, N] = x . Wc^T with FP4 levels."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16).reshape(-1, K)
+    y = np.zeros((x.shape[0], N), np.float64)
+    _load().oracle_fp4_matmul(_p(np.ascontiguousarray(packed, dtype=np.uint8)),
+                              _p(np.ascontiguousarray(absmax, dtype=np.float32)), N, K, blocksize, _p(x),
+                              x.shape[0], _p(y))
+    return y

@@ -388,9 +388,8 @@ void oracle_nf4_dequantize_bf16(const uint8_t *packed, const float *absmax, int6
 /* in fp64 and are summed in fp64.                                            */
 /* ------------------------------------------------------------------------- */
 
-static double dot_row(const uint8_t *packed, const float *absmax, int64_t K, int32_t blocksize,
-                      int64_t n, const uint16_t *xrow) {
-  const float *c = codebook32();
+static double dot_row_cb(const uint8_t *packed, const float *absmax, int64_t K, int32_t blocksize,
+                         int64_t n, const uint16_t *xrow, const float *c) {
   double acc = 0.0;
   for (int64_t k = 0; k < K; ++k) {
     int64_t i = n * K + k;
@@ -398,6 +397,11 @@ static double dot_row(const uint8_t *packed, const float *absmax, int64_t K, int
     acc += (double)wc * (double)oracle_bf16_to_f32(xrow[k]);
   }
   return acc;
+}
+
+static double dot_row(const uint8_t *packed, const float *absmax, int64_t K, int32_t blocksize,
+                      int64_t n, const uint16_t *xrow) {
+  return dot_row_cb(packed, absmax, K, blocksize, n, xrow, codebook32());
 }
 
 void oracle_nf4_matmul(const uint8_t *packed, const float *absmax, int64_t N, int64_t K,
@@ -597,4 +601,14 @@ void oracle_fp4_dequantize_bf16(const uint8_t *packed, const float *absmax, int6
   const float *c = fp4_codebook32();
 #pragma omp parallel for schedule(static)
   for (int64_t i = 0; i < n; ++i) out[i] = oracle_bf16_rn(c[code_at(packed, i)] * absmax[i / blocksize]);
+}
+
+/* The 4-bit matmul of FP4 weights: the same arithmetic as oracle_nf4_matmul with
+ * the FP4 levels, Wc = bf16_rn(fp4[code] * a). */
+void oracle_fp4_matmul(const uint8_t *packed, const float *absmax, int64_t N, int64_t K, int32_t blocksize,
+                       const uint16_t *x, int64_t B, double *y) {
+  const float *c = fp4_codebook32();
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t b = 0; b < B; ++b) y[b * N + n] = dot_row_cb(packed, absmax, K, blocksize, n, x + b * K, c);
 }

@@ -123,6 +123,10 @@ void oracle_fp4_dequantize_f32(const uint8_t *packed, const float *absmax, int64
 void oracle_fp4_dequantize_bf16(const uint8_t *packed, const float *absmax, int64_t n, int32_t blocksize,
                                 uint16_t *out);
 
+/* The 4-bit matmul with FP4 levels: y[b,n] = sum_k bf16_rn(fp4[code]*a)*x[b,k] (fp64). */
+void oracle_fp4_matmul(const uint8_t *packed, const float *absmax, int64_t N, int64_t K, int32_t blocksize,
+                       const uint16_t *x, int64_t B, double *y);
+
 /* Worker threads used by the loops marked parallel (0 = OpenMP default). */
 void oracle_set_threads(int n);
 int oracle_get_threads(void);

@@ -555,3 +555,53 @@ def test_fp4_bf16_input_and_output():
     d16 = oracle.fp4_dequantize(p, a, bits.size, 64, "bf16")
     d32 = oracle.fp4_dequantize(p, a, bits.size, 64, "f32")
     assert np.array_equal(d16, synth.f32_to_bf16_bits(d32))
+
+
+def test_fp4_matmul_one_hot_and_numpy():
+    """one-hot activations read bf16_rn(fp4[code] * a) back exactly; random activations match a numpy product"""
+    N, K = 32, 192
+    w = synth.normal_weights((N, K), 94)
+    p, a = oracle.fp4_quantize(w, 64)
+    wc = synth.bf16_bits_to_f32(oracle.fp4_dequantize(p, a, N * K, 64, "bf16")).reshape(N, K)
+    ks = [0, 63, 64, 191]
+    eye = synth.f32_to_bf16_bits(np.eye(K, dtype=np.float32)[ks])
+    assert np.array_equal(oracle.fp4_matmul(p, a, N, K, eye), wc[:, ks].T.astype(np.float64))
+    x = synth.activations((3, K), 95)
+    ref = synth.bf16_bits_to_f32(x).astype(np.float64) @ wc.astype(np.float64).T
+    assert np.allclose(oracle.fp4_matmul(p, a, N, K, x), ref, rtol=1e-12, atol=1e-15)
+    # the NF4 and FP4 products of the same weight differ (different levels), so the code book is really swapped
+    pn, an = oracle.quantize(w, 64)
+    assert not np.allclose(oracle.matmul(pn, an, N, K, x), ref)
+
+
+# ---------------------------------------------------------------- block sizes other than 64
+
+@pytest.mark.parametrize("bs", [32, 128, 256, 4096])
+def test_other_blocksizes_quantize_dequantize_matmul(bs):
+    """the blockwise rules at other block sizes (the pages give 64 only as an example size): absmax per block
+    equals numpy's max |w| per block, the block's largest element maps to +-1, every code is the brute-force
+    nearest level, and dequantize / matmul follow from them"""
+    N, K = 16, 4096
+    w = synth.normal_weights((N * K + 7,), 96 + bs)  # ragged last block
+    p, a = oracle.quantize(w, bs)
+    nb = (w.size + bs - 1) // bs
+    pad = np.zeros(nb * bs, np.float32)
+    pad[:w.size] = w
+    assert np.array_equal(a, np.abs(pad.reshape(nb, bs)).max(axis=1))
+    codes = np.stack([p >> 4, p & 15], axis=1).reshape(-1)[:w.size]
+    _, c32 = oracle.codebook()
+    for b in range(0, nb, max(1, nb // 40)):
+        lo, hi = b * bs, min(b * bs + bs, w.size)
+        j = lo + int(np.argmax(np.abs(w[lo:hi])))
+        assert codes[j] == (0 if w[j] < 0 else 15)
+    for i in range(0, w.size, 997):
+        x = np.float32(w[i]) / np.float32(a[i // bs])
+        d = [abs(Fraction(float(x)) - Fraction(float(c))) for c in c32]
+        assert codes[i] == min(range(16), key=lambda k: (d[k], k))
+    d32 = oracle.dequantize(p, a, w.size, bs, "f32")
+    assert np.array_equal(d32, (c32[codes] * np.repeat(a, bs)[:w.size]).astype(np.float32))
+    pm, am = oracle.quantize(w[:N * K], bs)
+    x = synth.activations((2, K), 97)
+    wc = synth.bf16_bits_to_f32(oracle.dequantize(pm, am, N * K, bs, "bf16")).reshape(N, K)
+    ref = synth.bf16_bits_to_f32(x).astype(np.float64) @ wc.astype(np.float64).T
+    assert np.allclose(oracle.matmul(pm, am, N, K, x, bs), ref, rtol=1e-12, atol=1e-15)
