@@ -26,7 +26,9 @@ def _init(name):
 
 def _hexf(s):
     s = s.rstrip("f")
-    return 0.0 if s in ("0.0", "-0.0") else float.fromhex(s)
+    if s in ("0.0", "-0.0"):
+        return -0.0 if s.startswith("-") else 0.0
+    return float.fromhex(s)
 
 
 def test_thresholds_are_rd32_of_the_oracle_midpoints():
@@ -69,3 +71,46 @@ def test_bucket_rule_decides_every_fp32_in_range():
 def _init_scalar(name):
     text = open(HEADER).read()
     return re.search(r"#define " + name + r" (\S+)", text).group(1)
+
+
+def test_fp4_tables_match_the_oracle_and_decide_every_magnitude():
+    """FP4 tables: the levels are the oracle's E2M1 / 6 by pattern (signed zero included); the magnitude
+    thresholds are the largest fp32 values not above the exact midpoints; the 16-bucket rule on |q| gives the
+    threshold count for every fp32 magnitude in [0, 1] it trusts; and sign + count is the oracle's nearest code"""
+    _, f4 = oracle.fp4_codebook()
+    code = np.array([_hexf(s) for s in _init("FP4_CODE_INIT")], np.float32)
+    assert np.array_equal(code.view(np.uint32), f4.view(np.uint32))  # bit for bit, -0 at pattern 8
+    thr = np.array([_hexf(s) for s in _init("FP4_THRESHOLD_INIT")], np.float32)
+    for i in range(7):
+        mid = (Fraction(float(f4[i])) + Fraction(float(f4[i + 1]))) / 2
+        assert Fraction(float(thr[i])) <= mid < Fraction(float(np.nextafter(thr[i], np.float32(2))))
+    q16 = np.array([int(s.rstrip("u"), 16) for s in _init("FP4_Q16_INIT")], np.uint32)
+    scale16 = np.float32(16.0) * np.float32(_hexf(_init_scalar("NF4_Q32_SCALE")))
+    e_thr = q16.view(np.float32)
+    near = np.float32(2.0 ** -19)
+    top = int(np.float32(1.0).view(np.uint32)) + 1
+    checked = 0
+    for lo in range(0, top, 1 << 24):
+        q = np.arange(lo, min(lo + (1 << 24), top), dtype=np.uint32).view(np.float32)
+        bucket = np.floor(q.astype(np.float64) * np.float64(scale16)).astype(np.int64) & 15  # RD(16 S q + 2^23)
+        e = q16[bucket]
+        t = e_thr[bucket]
+        fast = (e & 15).astype(np.int64) + (q > t)
+        truth = np.searchsorted(thr, q, side="left")
+        trusted = np.abs(q - t) > near
+        assert not (trusted & (fast != truth)).any()
+        checked += int(trusted.sum())
+    assert checked > 1_000_000_000
+    # sign + threshold count is the oracle's nearest FP4 code (ties to even, signed zero), around every threshold
+    xs = []
+    for t in thr:
+        v = np.float32(t)
+        for k in range(-3, 4):
+            w = v
+            for _ in range(abs(k)):
+                w = np.nextafter(w, np.float32(2.0 if k > 0 else -2.0))
+            xs += [float(w), -float(w)]
+    xs += [0.0, -0.0, 1.0, -1.0] + list(np.random.default_rng(5).uniform(-1, 1, 2000).astype(np.float32).astype(float))
+    for x in xs:
+        mag = int(np.searchsorted(thr, np.float32(abs(x)), side="left"))
+        assert oracle.fp4_nearest_code(x) == (8 if np.signbit(x) else 0) | mag, x
