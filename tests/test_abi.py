@@ -154,3 +154,17 @@ def test_host_validation_new_entry_points(lib):
     odd = (ctypes.POINTER(_lib.NF4Weight) * 2)(ctypes.pointer(weight()), ctypes.pointer(weight(rows=40)))
     assert lib.nf4_gemv_grouped(odd, 2, 0x9000, 1, ys, s) == E["NF4_ERR_UNSUPPORTED"]
     assert lib.nf4_gemv_grouped(ws, 2, 0x9008, 1, ys, s) == E["NF4_ERR_MISALIGNED"]
+
+
+def test_plain_c_client(tmp_path):
+    """the header compiles as C and a C program linked against libnf4.so gets the documented host-side results"""
+    import os
+    import subprocess
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.dirname(_lib.load()._name)
+    exe = str(tmp_path / "abi_check")
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Werror", "-I", os.path.join(root, "include"),
+                    os.path.join(root, "tests", "c_abi", "abi_check.c"), "-L", libdir, "-lnf4",
+                    "-Wl,-rpath," + libdir, "-lm", "-o", exe], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stderr
