@@ -1,8 +1,10 @@
 /*
  * nf4.h -- C ABI of libnf4: blockwise NF4 4-bit weight quantization with double
  * quantization of the absmax constants, dequantization, and the 4-bit-weight x
- * bf16-activation matmul that dequantizes on the fly (GEMV for decode, GEMM for
- * prefill), for NVIDIA B200 (sm_100a).
+ * bf16-activation matmul that dequantizes on the fly (GEMV for decode, also
+ * grouped over weights that share an input; GEMM for prefill, also with a
+ * low-rank adapter in the same accumulator; and the GEMM's input gradient
+ * through the frozen weight), for NVIDIA B200 (sm_100a).
  *
  * Method sources (web pages on bitsandbytes / QLoRA):
  *   [bnb-tools] "bitsandbytes" (ozercemkelahmet.com/tools/bitsandbytes):
