@@ -9,9 +9,11 @@
  * Method sources (web pages on bitsandbytes / QLoRA):
  *   [bnb-tools] "bitsandbytes" (ozercemkelahmet.com/tools/bitsandbytes):
  *               "How it works" Steps 1-5, "How NF4 works", "Double quantization",
- *               "A worked example".
+ *               "A worked example", "Fine-tuning with adapters on a 4-bit
+ *               model", "Strengths and limitations".
  *   [bnb-tut]   "bitsandbytes quantization tutorial: 4-bit and 8-bit models"
- *               (mljourney.com): "4-bit Loading with NF4", "How NF4 Works".
+ *               (mljourney.com): "4-bit Loading with NF4", "How NF4 Works",
+ *               "QLoRA: Fine-Tuning a 4-bit Model".
  *
  * Conventions for every entry point:
  *   - Memory: all buffers are allocated and owned by the caller; the library
