@@ -69,6 +69,18 @@ typedef enum { NF4_F32 = 0, NF4_BF16 = 1 } nf4_dtype;
  *              "A worked example"), top code 127. */
 typedef enum { NF4_DQ_E4M3 = 0, NF4_DQ_INT8 = 1 } nf4_dq_code;
 
+/* The 4-bit code book ([bnb-tools] "What it is": 4-bit layers in NF4 or FP4;
+ * "Glossary", the FP4 entry; [bnb-tut] "4-bit Loading with NF4").
+ * NF4_QUANT_NF4: the 16 NF4 levels (normal quantiles scaled to [-1, 1],
+ *                ascending, index 7 = 0).
+ * NF4_QUANT_FP4: the 4-bit float E2M1 (sign, 2 exponent bits with bias 1,
+ *                1 mantissa bit) divided by 6 so that +-6 maps to +-1; the
+ *                4-bit code is the E2M1 bit pattern (8 = -0).  Nearest level
+ *                with ties to the even mantissa bit; a zero result keeps the
+ *                sign of the value; an all-zero block and an odd tail's
+ *                partner are +0. */
+typedef enum { NF4_QUANT_NF4 = 0, NF4_QUANT_FP4 = 1 } nf4_quant_type;
+
 /* A quantized weight W of shape [rows, cols] (row-major, rows = output
  * features N, cols = input features K), flattened for quantization so the
  * level-1 blocks run along a row.  All pointers are device pointers.
@@ -79,7 +91,9 @@ typedef enum { NF4_DQ_E4M3 = 0, NF4_DQ_INT8 = 1 } nf4_dq_code;
  *   absmax_q      nb 8-bit codes of the mean-removed scales (double quant)
  *   absmax_scale  ceil(nb/dq_blocksize) fp32 second-level block absmax values
  *   absmax_mean   1 fp32: the mean removed before second-level quantization
- *   blocksize     64 (only value implemented); dq_blocksize 256; dq_code nf4_dq_code */
+ *   blocksize     64 (only value implemented); dq_blocksize 256; dq_code nf4_dq_code
+ *   quant_type    nf4_quant_type of the codes (0 = NF4: a zero-initialised
+ *                 descriptor describes NF4 codes) */
 typedef struct {
   const uint8_t *packed;
   const float *absmax;
@@ -88,6 +102,7 @@ typedef struct {
   const float *absmax_mean;
   int64_t rows, cols;
   int32_t blocksize, dq_blocksize, dq_code;
+  int32_t quant_type;
 } nf4_weight;
 
 /* Blockwise NF4 quantization, [bnb-tools] "How it works" Steps 1-4.
@@ -100,6 +115,15 @@ typedef struct {
  * blocksize must be 64 (else NF4_ERR_UNSUPPORTED). */
 NF4_API nf4_status nf4_quantize(const void *src, int32_t src_dtype, int64_t n, int32_t blocksize,
                         uint8_t *packed_out, float *absmax_out, nf4_stream_t stream);
+
+/* nf4_quantize with the code book chosen by quant_type (nf4_quant_type): the
+ * same blocking, absmax, packing and arguments; with NF4_QUANT_FP4 the code of
+ * x = fp32(w / a) is the nearest FP4 level (see nf4_quant_type), an all-zero
+ * block is all +0 codes and an odd tail's low nibble is 0.
+ * nf4_quantize(...) is nf4_quantize_typed(..., NF4_QUANT_NF4, ...). */
+NF4_API nf4_status nf4_quantize_typed(const void *src, int32_t src_dtype, int64_t n, int32_t blocksize,
+                                      int32_t quant_type, uint8_t *packed_out, float *absmax_out,
+                                      nf4_stream_t stream);
 
 /* Double quantization of the fp32 absmax array, [bnb-tut] "How NF4 Works"
  * (scale constants quantized from float32 to float8) and [bnb-tools] "Double
@@ -117,7 +141,11 @@ NF4_API nf4_status nf4_quantize(const void *src, int32_t src_dtype, int64_t n, i
  *               next one (no clearing between calls).  Calls that may run at
  *               the same time need separate buffers; after
  *               nf4_check_device_error reports an error, zero it again.
- * dq_blocksize must be 256.  nb == 0 launches nothing and leaves mean_out unset. */
+ * dq_blocksize must be 256.  nb == 0 launches nothing and leaves mean_out unset.
+ * Limit: nb <= NF4_DQ_MAX_NB.  The exact sum is kept as 32-bit digits in
+ * signed 64-bit limbs, which stay exact for up to 2^31 - 1 values; larger nb
+ * returns NF4_ERR_INVALID_ARG. */
+#define NF4_DQ_MAX_NB 2147483647LL
 NF4_API nf4_status nf4_double_quant(const float *absmax, int64_t nb, int32_t dq_blocksize, int32_t dq_code,
                             uint8_t *q_out, float *scale_out, float *mean_out, void *workspace,
                             size_t workspace_bytes, nf4_stream_t stream);
@@ -139,7 +167,7 @@ NF4_API size_t nf4_double_quant_workspace_bytes(int64_t nb);
  *   streams, other host threads) race and must be ordered by the caller.
  *   Limit: nb <= NF4_DQ_NOALLOC_MAX_NB (the exact-sum digits in the array
  *   stay exact up to this count); larger nb returns NF4_ERR_INVALID_ARG. */
-#define NF4_DQ_NOALLOC_MAX_NB 2147483647LL
+#define NF4_DQ_NOALLOC_MAX_NB NF4_DQ_MAX_NB
 NF4_API nf4_status nf4_double_quant_noalloc(const float *absmax, int64_t nb, int32_t dq_blocksize, int32_t dq_code,
                                             uint8_t *q_out, float *scale_out, float *mean_out, nf4_stream_t stream);
 
@@ -166,12 +194,34 @@ NF4_API nf4_status nf4_gemv(const nf4_weight *w, const void *x, int32_t batch, v
  * "4-bit Loading with NF4").  Each weight gets exactly the results nf4_gemv
  * would give it.
  *   ws     host array of `count` weight descriptors (1 <= count <= 4), all
- *          with the same cols and the same scale kind (plain or double-quant)
+ *          with the same cols, scale kind (plain or double-quant) and quant_type
  *   x      device bf16 [batch, cols];  ys  host array of `count` device bf16
  *          outputs, ys[i] of shape [batch, ws[i]->rows]
  *   1 <= batch <= 8; cols % 64 == 0; every rows % 16 == 0. */
 NF4_API nf4_status nf4_gemv_grouped(const nf4_weight *const *ws, int32_t count, const void *x, int32_t batch,
                             void *const *ys, nf4_stream_t stream);
+
+/* Decode GEMV over a list of weights, each with its own input and output, in
+ * one launch: the decode pass over the linear layers of a whole 4-bit model
+ * (such as the Llama-3.1-8B of [bnb-tut] "4-bit Loading with NF4"), each
+ * block expanded on the fly as in [bnb-tools] Step 5.  Every weight gets
+ * exactly the results nf4_gemv would give it:
+ *   ys[i][b, n] = bf16_rn( sum_k Wc_i[n, k] * xs[i][b, k] )
+ * The weights' 16-row tiles are spread over one persistent grid (one CTA per
+ * SM), so small and large weights share the GPU and the pass pays one launch.
+ *   ws     host array of `count` weight descriptors (by value), each with its
+ *          own shape and scale kind, all with the same quant_type;
+ *          rows % 16 == 0, cols % 64 == 0
+ *   xs     host array of `count` device bf16 inputs, xs[i] of shape
+ *          [batch, ws[i].cols], 16-byte aligned
+ *   ys     host array of `count` device bf16 outputs, ys[i] of shape
+ *          [batch, ws[i].rows], 4-byte aligned; no output may overlap any
+ *          input or another output
+ *   1 <= count <= NF4_GEMV_STREAM_MAX; 1 <= batch <= 8.
+ * Weights with rows == 0 or cols == 0 are skipped. */
+#define NF4_GEMV_STREAM_MAX 256
+NF4_API nf4_status nf4_gemv_stream(const nf4_weight *ws, const void *const *xs, void *const *ys, int32_t count,
+                                   int32_t batch, nf4_stream_t stream);
 
 /* Prefill GEMM, same arithmetic as nf4_gemv for m activation rows:
  *   Y[m, n] = bf16_rn( sum_k Wc[n, k] * X[m, k] )
@@ -194,7 +244,9 @@ NF4_API size_t nf4_gemm_workspace_bytes(const nf4_weight *w, int64_t m);
  * on a 4-bit model": r = 16, lora_alpha = 32, scale = lora_alpha / r).
  *   down   device bf16 [r, cols] (the adapter's first map, A), 16-byte aligned
  *   up     device bf16 [rows, r] (the second map, B), 16-byte aligned
- *   r      16 or 32;  scale  finite fp32 */
+ *   r      16 or 32;  scale  finite fp32
+ * nf4_gemm_lora and nf4_gemm_dx take NF4 codes only (NF4_ERR_UNSUPPORTED for
+ * quant_type FP4). */
 typedef struct {
   const void *down;
   const void *up;

@@ -20,15 +20,16 @@ from typing import Optional
 import torch
 
 from . import _lib
-from ._lib import NF4_BF16, NF4_DQ_E4M3, NF4_DQ_INT8, NF4_F32, NF4Error
+from ._lib import NF4_BF16, NF4_DQ_E4M3, NF4_DQ_INT8, NF4_F32, NF4_QUANT_FP4, NF4_QUANT_NF4, NF4Error
 
 __all__ = ["QuantizedWeight", "quantize", "double_quant", "quantize_weight", "dequantize", "gemv", "gemm",
-           "storage_bytes", "gemm_workspace_bytes", "gemm_dx", "gemm_dx_workspace_bytes", "gemm_lora", "gemv_grouped",
+           "storage_bytes", "gemm_workspace_bytes", "gemm_dx", "gemm_dx_workspace_bytes", "gemm_lora", "gemv_grouped", "gemv_stream",
            "gemm_lora_workspace_bytes", "code_table", "check_device_error", "kernel_launches", "NF4Error", "library_path"]
 
 BLOCKSIZE = 64
 DQ_BLOCKSIZE = 256
 _DQ_CODES = {"e4m3": NF4_DQ_E4M3, "int8": NF4_DQ_INT8}
+_QUANT_TYPES = {"nf4": NF4_QUANT_NF4, "fp4": NF4_QUANT_FP4}
 
 
 def library_path() -> str:
@@ -67,6 +68,7 @@ class QuantizedWeight:
     dq_code: int = NF4_DQ_E4M3
     blocksize: int = BLOCKSIZE
     dq_blocksize: int = DQ_BLOCKSIZE
+    quant_type: int = NF4_QUANT_NF4
 
     @property
     def double_quant(self) -> bool:
@@ -75,14 +77,14 @@ class QuantizedWeight:
     def descriptor(self) -> _lib.NF4Weight:
         return _lib.NF4Weight(_ptr(self.packed), _ptr(self.absmax), _ptr(self.absmax_q), _ptr(self.absmax_scale),
                               _ptr(self.absmax_mean), self.rows, self.cols, self.blocksize, self.dq_blocksize,
-                              self.dq_code)
+                              self.dq_code, self.quant_type)
 
     def storage_bytes(self) -> int:
         return storage_bytes(self.rows * self.cols, self.double_quant)
 
 
-def quantize(w: torch.Tensor, blocksize: int = BLOCKSIZE, out=None, stream=None):
-    """Level-1 NF4 quantization of a flattened fp32/bf16 tensor.
+def quantize(w: torch.Tensor, blocksize: int = BLOCKSIZE, out=None, stream=None, quant_type: str = "nf4"):
+    """Level-1 4-bit quantization (NF4, or FP4 with quant_type="fp4") of a flattened fp32/bf16 tensor.
     Returns (packed uint8 [ceil(n/2)], absmax fp32 [ceil(n/64)])."""
     _need_cuda(w, "w")
     if w.dtype not in (torch.float32, torch.bfloat16):
@@ -93,9 +95,9 @@ def quantize(w: torch.Tensor, blocksize: int = BLOCKSIZE, out=None, stream=None)
         absmax = torch.empty((n + blocksize - 1) // blocksize, dtype=torch.float32, device=w.device)
     else:
         packed, absmax = out
-    st = _lib.load().nf4_quantize(_ptr(w), NF4_BF16 if w.dtype == torch.bfloat16 else NF4_F32, n, blocksize,
-                                  _ptr(packed), _ptr(absmax), _stream(stream))
-    _lib.check(st, "nf4_quantize")
+    st = _lib.load().nf4_quantize_typed(_ptr(w), NF4_BF16 if w.dtype == torch.bfloat16 else NF4_F32, n, blocksize,
+                                        _QUANT_TYPES[quant_type], _ptr(packed), _ptr(absmax), _stream(stream))
+    _lib.check(st, "nf4_quantize_typed")
     return packed, absmax
 
 
@@ -122,16 +124,17 @@ def double_quant(absmax: torch.Tensor, code: str = "e4m3", dq_blocksize: int = D
 
 
 def quantize_weight(w: torch.Tensor, use_double_quant: bool = True, code: str = "e4m3",
-                    stream=None) -> QuantizedWeight:
-    """Quantize a 2-D weight [rows, cols] (nn.Linear layout: out x in)."""
+                    stream=None, quant_type: str = "nf4") -> QuantizedWeight:
+    """Quantize a 2-D weight [rows, cols] (nn.Linear layout: out x in) to NF4 (or FP4: quant_type="fp4")."""
     if w.dim() != 2:
         raise ValueError("quantize_weight takes a 2-D [rows, cols] tensor")
-    packed, absmax = quantize(w, stream=stream)
-    qw = QuantizedWeight(packed=packed, rows=w.shape[0], cols=w.shape[1], absmax=absmax)
+    packed, absmax = quantize(w, stream=stream, quant_type=quant_type)
+    qt = _QUANT_TYPES[quant_type]
+    qw = QuantizedWeight(packed=packed, rows=w.shape[0], cols=w.shape[1], absmax=absmax, quant_type=qt)
     if use_double_quant:
         q, scale, mean = double_quant(absmax, code, stream=stream)
         qw = QuantizedWeight(packed=packed, rows=w.shape[0], cols=w.shape[1], absmax_q=q, absmax_scale=scale,
-                             absmax_mean=mean, dq_code=_DQ_CODES[code])
+                             absmax_mean=mean, dq_code=_DQ_CODES[code], quant_type=qt)
     return qw
 
 
@@ -177,6 +180,34 @@ def gemv_grouped(qws, x: torch.Tensor, outs=None, stream=None) -> list:
     ys = (ctypes.c_void_p * len(outs))(*[_ptr(o) for o in outs])
     st = _lib.load().nf4_gemv_grouped(arr, len(ds), _ptr(x2), x2.shape[0], ys, _stream(stream))
     _lib.check(st, "nf4_gemv_grouped")
+    return outs
+
+
+GEMV_STREAM_MAX = 256
+
+
+def gemv_stream(qws, xs, outs=None, stream=None) -> list:
+    """nf4_gemv of up to 256 weights, each on its own input xs[i] (bf16 [B, cols_i], the same B <= 8 for all),
+    in one launch.  Returns the outputs (bf16 [B, rows_i])."""
+    qws, xs = list(qws), list(xs)
+    if len(qws) != len(xs) or not qws:
+        raise ValueError("gemv_stream takes one input per weight")
+    x2 = []
+    for q, x in zip(qws, xs):
+        _need_cuda(x, "x")
+        if x.dtype != torch.bfloat16:
+            raise TypeError("x must be bfloat16")
+        x2.append(x.reshape(-1, q.cols))
+    batch = x2[0].shape[0]
+    if any(x.shape[0] != batch for x in x2):
+        raise ValueError("every input needs the same batch")
+    if outs is None:
+        outs = [torch.empty(batch, q.rows, dtype=torch.bfloat16, device=x2[0].device) for q in qws]
+    ds = (_lib.NF4Weight * len(qws))(*[q.descriptor() for q in qws])
+    xp = (ctypes.c_void_p * len(x2))(*[_ptr(x) for x in x2])
+    yp = (ctypes.c_void_p * len(outs))(*[_ptr(o) for o in outs])
+    st = _lib.load().nf4_gemv_stream(ds, xp, yp, len(qws), batch, _stream(stream))
+    _lib.check(st, "nf4_gemv_stream")
     return outs
 
 

@@ -16,6 +16,7 @@ STATUS_NAMES = {0: "NF4_OK", 1: "NF4_ERR_INVALID_ARG", 2: "NF4_ERR_MISALIGNED", 
                 4: "NF4_ERR_ARCH", 5: "NF4_ERR_CUDA", 6: "NF4_ERR_TIMEOUT"}
 NF4_F32, NF4_BF16 = 0, 1
 NF4_DQ_E4M3, NF4_DQ_INT8 = 0, 1
+NF4_QUANT_NF4, NF4_QUANT_FP4 = 0, 1
 
 # every symbol include/nf4.h declares: name -> (restype, argtypes)
 P = ctypes.c_void_p
@@ -27,7 +28,8 @@ SZ = ctypes.c_size_t
 class NF4Weight(ctypes.Structure):
     """Mirror of the C struct nf4_weight."""
     _fields_ = [("packed", P), ("absmax", P), ("absmax_q", P), ("absmax_scale", P), ("absmax_mean", P),
-                ("rows", I64), ("cols", I64), ("blocksize", I32), ("dq_blocksize", I32), ("dq_code", I32)]
+                ("rows", I64), ("cols", I64), ("blocksize", I32), ("dq_blocksize", I32), ("dq_code", I32),
+                ("quant_type", I32)]
 
 
 class NF4Lora(ctypes.Structure):
@@ -37,12 +39,14 @@ class NF4Lora(ctypes.Structure):
 
 SIGNATURES = {
     "nf4_quantize": (ctypes.c_int, [P, I32, I64, I32, P, P, P]),
+    "nf4_quantize_typed": (ctypes.c_int, [P, I32, I64, I32, I32, P, P, P]),
     "nf4_double_quant": (ctypes.c_int, [P, I64, I32, I32, P, P, P, P, SZ, P]),
     "nf4_double_quant_workspace_bytes": (SZ, [I64]),
     "nf4_double_quant_noalloc": (ctypes.c_int, [P, I64, I32, I32, P, P, P, P]),
     "nf4_dequantize": (ctypes.c_int, [ctypes.POINTER(NF4Weight), P, I32, P]),
     "nf4_gemv": (ctypes.c_int, [ctypes.POINTER(NF4Weight), P, I32, P, P]),
     "nf4_gemv_grouped": (ctypes.c_int, [ctypes.POINTER(ctypes.POINTER(NF4Weight)), I32, P, I32, ctypes.POINTER(P), P]),
+    "nf4_gemv_stream": (ctypes.c_int, [ctypes.POINTER(NF4Weight), ctypes.POINTER(P), ctypes.POINTER(P), I32, I32, P]),
     "nf4_gemm": (ctypes.c_int, [ctypes.POINTER(NF4Weight), P, I64, P, P, SZ, P]),
     "nf4_gemm_workspace_bytes": (SZ, [ctypes.POINTER(NF4Weight), I64]),
     "nf4_gemm_lora": (ctypes.c_int, [ctypes.POINTER(NF4Weight), ctypes.POINTER(NF4Lora), P, I64, P, P, SZ, P]),

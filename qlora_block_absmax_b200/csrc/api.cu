@@ -1,7 +1,7 @@
 // api.cu -- extern "C" entry points of libnf4 (declared in include/nf4.h).
 // Host-side validation happens before any launch; kernels live in the other
 // translation units (quantize.cu, double_quant.cu, dequantize.cu, gemv.cu,
-// gemm_sm100.cu).
+// gemv_stream.cu, gemm_sm100.cu, gemm_dx_sm100.cu, lora_down.cu).
 #include <atomic>
 #include <mutex>
 
@@ -54,17 +54,18 @@ nf4_status check_weight(const nf4_weight* w, nf4::Scales* s) {
   if (w == nullptr || w->packed == nullptr) return NF4_ERR_INVALID_ARG;
   if (w->rows < 0 || w->cols < 0) return NF4_ERR_INVALID_ARG;
   if (w->blocksize != nf4::kBlock) return NF4_ERR_UNSUPPORTED;
+  if (w->quant_type != NF4_QUANT_NF4 && w->quant_type != NF4_QUANT_FP4) return NF4_ERR_INVALID_ARG;
   if (!aligned(w->packed, 16)) return NF4_ERR_MISALIGNED;
   if (w->absmax != nullptr) {
     if (!aligned(w->absmax, 4)) return NF4_ERR_MISALIGNED;
-    *s = nf4::Scales{w->absmax, nullptr, nullptr, nullptr, 0};
+    *s = nf4::Scales{w->absmax, nullptr, nullptr, nullptr, 0, w->quant_type};
     return NF4_OK;
   }
   if (w->absmax_q == nullptr || w->absmax_scale == nullptr || w->absmax_mean == nullptr) return NF4_ERR_INVALID_ARG;
   if (w->dq_blocksize != nf4::kDqBlock) return NF4_ERR_UNSUPPORTED;
   if (w->dq_code != NF4_DQ_E4M3 && w->dq_code != NF4_DQ_INT8) return NF4_ERR_INVALID_ARG;
   if (!aligned(w->absmax_scale, 4) || !aligned(w->absmax_mean, 4)) return NF4_ERR_MISALIGNED;
-  *s = nf4::Scales{nullptr, w->absmax_q, w->absmax_scale, w->absmax_mean, w->dq_code};
+  *s = nf4::Scales{nullptr, w->absmax_q, w->absmax_scale, w->absmax_mean, w->dq_code, w->quant_type};
   return NF4_OK;
 }
 
@@ -130,7 +131,13 @@ int32_t nf4_device_supported(void) {
 
 nf4_status nf4_quantize(const void* src, int32_t src_dtype, int64_t n, int32_t blocksize, uint8_t* packed_out,
                         float* absmax_out, nf4_stream_t stream) {
+  return nf4_quantize_typed(src, src_dtype, n, blocksize, NF4_QUANT_NF4, packed_out, absmax_out, stream);
+}
+
+nf4_status nf4_quantize_typed(const void* src, int32_t src_dtype, int64_t n, int32_t blocksize, int32_t quant_type,
+                              uint8_t* packed_out, float* absmax_out, nf4_stream_t stream) {
   if (n < 0) return NF4_ERR_INVALID_ARG;
+  if (quant_type != NF4_QUANT_NF4 && quant_type != NF4_QUANT_FP4) return NF4_ERR_INVALID_ARG;
   if (src_dtype != NF4_F32 && src_dtype != NF4_BF16) return NF4_ERR_INVALID_ARG;
   if (blocksize != nf4::kBlock) return NF4_ERR_UNSUPPORTED;
   if (n == 0) return NF4_OK;
@@ -139,14 +146,14 @@ nf4_status nf4_quantize(const void* src, int32_t src_dtype, int64_t n, int32_t b
   DeviceInfo d;
   nf4_status st = device_info(&d);
   if (st != NF4_OK) return st;
-  return from_cuda(nf4::launch_quantize(src, src_dtype == NF4_BF16, n, packed_out, absmax_out,
+  return from_cuda(nf4::launch_quantize(src, src_dtype == NF4_BF16, n, packed_out, absmax_out, quant_type,
                                         reinterpret_cast<cudaStream_t>(stream), d.num_sms));
 }
 
 nf4_status nf4_double_quant(const float* absmax, int64_t nb, int32_t dq_blocksize, int32_t dq_code, uint8_t* q_out,
                             float* scale_out, float* mean_out, void* workspace, size_t workspace_bytes,
                             nf4_stream_t stream) {
-  if (nb < 0) return NF4_ERR_INVALID_ARG;
+  if (nb < 0 || nb > NF4_DQ_MAX_NB) return NF4_ERR_INVALID_ARG;
   if (dq_code != NF4_DQ_E4M3 && dq_code != NF4_DQ_INT8) return NF4_ERR_INVALID_ARG;
   if (dq_blocksize != nf4::kDqBlock) return NF4_ERR_UNSUPPORTED;
   if (nb == 0) return NF4_OK;
@@ -244,7 +251,7 @@ nf4_status nf4_gemv(const nf4_weight* w, const void* x, int32_t batch, void* y, 
   if (!aligned(x, 16) || !aligned(y, 4)) return NF4_ERR_MISALIGNED;
   DeviceInfo d;
   if ((st = device_info(&d)) != NF4_OK) return st;
-  return from_cuda(nf4::launch_gemv(w->packed, s, w->rows, w->cols, x, batch, y,
+  return from_cuda(nf4::launch_gemv(w->packed, s, w->rows, w->cols, x, batch, y, d.error_word,
                                     reinterpret_cast<cudaStream_t>(stream), d.num_sms));
 }
 
@@ -261,7 +268,9 @@ nf4_status nf4_gemv_grouped(const nf4_weight* const* ws, int32_t count, const vo
     nf4_status st = check_weight(ws[i], &s[n]);
     if (st != NF4_OK) return st;
     const nf4_weight* w = ws[i];
-    if (w->cols != ws[0]->cols || (w->absmax == nullptr) != (ws[0]->absmax == nullptr)) return NF4_ERR_INVALID_ARG;
+    if (w->cols != ws[0]->cols || (w->absmax == nullptr) != (ws[0]->absmax == nullptr) ||
+        w->quant_type != ws[0]->quant_type)
+      return NF4_ERR_INVALID_ARG;
     if (w->cols % nf4::kBlock != 0 || w->rows % 16 != 0) return NF4_ERR_UNSUPPORTED;
     if (w->rows == 0) continue;  // nothing to compute for an empty weight
     if (ys[i] == nullptr) return NF4_ERR_INVALID_ARG;
@@ -277,8 +286,36 @@ nf4_status nf4_gemv_grouped(const nf4_weight* const* ws, int32_t count, const vo
   DeviceInfo d;
   nf4_status st = device_info(&d);
   if (st != NF4_OK) return st;
-  return from_cuda(nf4::launch_gemv_group(packed, s, rows, n, ws[0]->cols, x, batch, y,
-                                          reinterpret_cast<cudaStream_t>(stream)));
+  return from_cuda(nf4::launch_gemv_group(packed, s, rows, n, ws[0]->cols, x, batch, y, d.error_word,
+                                          reinterpret_cast<cudaStream_t>(stream), d.num_sms));
+}
+
+nf4_status nf4_gemv_stream(const nf4_weight* ws, const void* const* xs, void* const* ys, int32_t count, int32_t batch,
+                           nf4_stream_t stream) {
+  if (ws == nullptr || xs == nullptr || ys == nullptr || count < 1 || count > NF4_GEMV_STREAM_MAX)
+    return NF4_ERR_INVALID_ARG;
+  if (batch < 1 || batch > 8) return NF4_ERR_INVALID_ARG;
+  static_assert(NF4_GEMV_STREAM_MAX <= nf4::kMaxStreamItems, "stream capacity");
+  nf4::GemvItem items[NF4_GEMV_STREAM_MAX];
+  int n = 0;
+  for (int i = 0; i < count; ++i) {
+    const nf4_weight* w = &ws[i];
+    nf4::Scales s;
+    nf4_status st = check_weight(w, &s);
+    if (st != NF4_OK) return st;
+    if (w->quant_type != ws[0].quant_type) return NF4_ERR_INVALID_ARG;  // one code book per launch
+    if (w->cols % nf4::kBlock != 0 || w->rows % 16 != 0) return NF4_ERR_UNSUPPORTED;
+    if (w->rows == 0 || w->cols == 0) continue;  // nothing to compute for an empty weight
+    if (xs[i] == nullptr || ys[i] == nullptr) return NF4_ERR_INVALID_ARG;
+    if (!aligned(xs[i], 16) || !aligned(ys[i], 4)) return NF4_ERR_MISALIGNED;
+    items[n++] = nf4::GemvItem{w->packed, s, xs[i], ys[i], w->rows, w->cols};
+  }
+  if (n == 0) return NF4_OK;
+  DeviceInfo d;
+  nf4_status st = device_info(&d);
+  if (st != NF4_OK) return st;
+  return from_cuda(nf4::launch_gemv_items(items, n, batch, d.error_word, reinterpret_cast<cudaStream_t>(stream),
+                                          d.num_sms));
 }
 
 nf4_status nf4_gemm(const nf4_weight* w, const void* x, int64_t m, void* y, void* workspace, size_t workspace_bytes,
@@ -305,6 +342,7 @@ nf4_status nf4_gemm_lora(const nf4_weight* w, const nf4_lora* lora, const void* 
   nf4::Scales s;
   nf4_status st = check_weight(w, &s);
   if (st != NF4_OK) return st;
+  if (w->quant_type != NF4_QUANT_NF4) return NF4_ERR_UNSUPPORTED;  // NF4 codes only
   if (m < 0 || lora == nullptr) return NF4_ERR_INVALID_ARG;
   if (lora->r != 16 && lora->r != 32) return NF4_ERR_UNSUPPORTED;
   if (!(lora->scale == lora->scale) || lora->scale - lora->scale != 0.0f) return NF4_ERR_INVALID_ARG;  // finite
@@ -328,6 +366,7 @@ nf4_status nf4_gemm_dx(const nf4_weight* w, const void* dy, int64_t m, void* dx,
   nf4::Scales s;
   nf4_status st = check_weight(w, &s);
   if (st != NF4_OK) return st;
+  if (w->quant_type != NF4_QUANT_NF4) return NF4_ERR_UNSUPPORTED;  // NF4 codes only
   if (m < 0) return NF4_ERR_INVALID_ARG;
   if (w->rows % 64 != 0 || w->cols % 128 != 0) return NF4_ERR_UNSUPPORTED;
   if (m == 0 || w->rows == 0 || w->cols == 0) return NF4_OK;

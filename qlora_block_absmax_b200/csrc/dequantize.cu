@@ -1,4 +1,4 @@
-// dequantize.cu -- NF4 dequantization.
+// dequantize.cu -- NF4 (and FP4) dequantization.
 //
 // "bitsandbytes" (ozercemkelahmet.com/tools), "How it works" Step 5: a block is
 // expanded back with its scale and the code book: w^ = RN(code[idx] * a).
@@ -15,7 +15,7 @@
 namespace nf4 {
 namespace {
 
-__constant__ float c_code[16] = NF4_CODE_INIT;
+__constant__ float c_code[2][16] = {NF4_CODE_INIT, FP4_CODE_INIT};  // by code book: NF4, FP4
 
 template <bool kDQ>
 __device__ __forceinline__ float block_scale(const Scales& s, const float* unit_lut, int64_t b) {
@@ -23,13 +23,13 @@ __device__ __forceinline__ float block_scale(const Scales& s, const float* unit_
   return dq_absmax(unit_lut[s.q[b]], s.scale[b / kDqBlock], *s.mean);
 }
 
-template <bool kDQ, bool kBF16>
+template <bool kDQ, bool kBF16, int kBook>
 __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restrict__ packed, Scales s, int64_t n,
                                                          void* __restrict__ out) {
   pdl_launch_dependents();
   __shared__ float code[16];
   __shared__ float unit_lut[kDQ ? 256 : 1];
-  if (threadIdx.x < 16) code[threadIdx.x] = c_code[threadIdx.x];
+  if (threadIdx.x < 16) code[threadIdx.x] = c_code[kBook][threadIdx.x];
   if (kDQ) unit_lut[threadIdx.x & 255] = dq_unit(threadIdx.x & 255, s.dq_code);
   __syncthreads();
   pdl_wait();
@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restri
 // the matmuls use) and expands its 32 code bytes with byte permutes.  The
 // warp's 32 consecutive blocks (4 KB of bf16) go through a swizzled shared
 // tile so the global stores are 512 contiguous bytes per instruction.
-template <bool kDQ>
+template <bool kDQ, int kBook>
 __global__ void __launch_bounds__(256) dequantize_bf16_kernel(const uint8_t* __restrict__ packed, Scales s,
                                                               int64_t n, __nv_bfloat16* __restrict__ out) {
   __shared__ float unit_lut[kDQ ? 256 : 1];
@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(256) dequantize_bf16_kernel(const uint8_t* __r
     if (full_warp) {
       const uint4* src = reinterpret_cast<const uint4*>(packed + b * (kBlock / 2));
       const uint4 w0 = __ldcs(src), w1 = __ldcs(src + 1);
-      const Table T = make_table(block_scale<kDQ>(s, unit_lut, b));
+      const Table T = make_table<kBook>(block_scale<kDQ>(s, unit_lut, b));
       const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
@@ -138,7 +138,7 @@ __global__ void __launch_bounds__(256) dequantize_bf16_kernel(const uint8_t* __r
       }
       __syncwarp();
     } else if (b < nblocks) {
-      const Table T = make_table(block_scale<kDQ>(s, unit_lut, b));
+      const Table T = make_table<kBook>(block_scale<kDQ>(s, unit_lut, b));
       if (b < nfull) {
         const uint4* src = reinterpret_cast<const uint4*>(packed + b * (kBlock / 2));
         const uint4 w0 = __ldcs(src), w1 = __ldcs(src + 1);
@@ -164,38 +164,39 @@ __global__ void __launch_bounds__(256) dequantize_bf16_kernel(const uint8_t* __r
   }
 }
 
-}  // namespace
-
-cudaError_t launch_dequantize(const uint8_t* packed, const Scales& s, int64_t n, void* out, bool out_bf16,
-                              cudaStream_t stream, int num_sms) {
+template <int kBook>
+cudaError_t launch_book(const uint8_t* packed, const Scales& s, int64_t n, void* out, bool out_bf16,
+                        cudaStream_t stream, int num_sms) {
   const int64_t nblocks = (n + kBlock - 1) / kBlock;
-  int64_t grid = (nblocks + 255) / 256;
   const int64_t cap = (int64_t)num_sms * 8;
-  if (grid > cap) grid = cap;
-  if (grid < 1) grid = 1;
   const bool dq = s.absmax == nullptr;
+  cudaError_t e;
   if (out_bf16) {
     int64_t g2 = (nblocks + 255) / 256;  // 8 warps x 32 blocks per CTA per pass
     if (g2 > cap) g2 = cap;
     if (g2 < 1) g2 = 1;
     auto* ob = static_cast<__nv_bfloat16*>(out);
-    const cudaError_t e = dq ? launch_pdl(dequantize_bf16_kernel<true>, dim3((unsigned)g2), dim3(256), 0, stream,
-                                          packed, s, n, ob)
-                             : launch_pdl(dequantize_bf16_kernel<false>, dim3((unsigned)g2), dim3(256), 0, stream,
-                                          packed, s, n, ob);
-    count_launches(1);
-    return e != cudaSuccess ? e : cudaGetLastError();
+    e = dq ? launch_pdl(dequantize_bf16_kernel<true, kBook>, dim3((unsigned)g2), dim3(256), 0, stream, packed, s, n, ob)
+           : launch_pdl(dequantize_bf16_kernel<false, kBook>, dim3((unsigned)g2), dim3(256), 0, stream, packed, s, n,
+                        ob);
+  } else {
+    int64_t grid = (nblocks + 255) / 256;
+    if (grid > cap) grid = cap;
+    if (grid < 1) grid = 1;
+    const dim3 g((unsigned)grid), b(256);
+    e = dq ? launch_pdl(dequantize_kernel<true, false, kBook>, g, b, 0, stream, packed, s, n, out)
+           : launch_pdl(dequantize_kernel<false, false, kBook>, g, b, 0, stream, packed, s, n, out);
   }
-  const dim3 g((unsigned)grid), b(256);
-  cudaError_t e;
-  if (dq)
-    e = out_bf16 ? launch_pdl(dequantize_kernel<true, true>, g, b, 0, stream, packed, s, n, out)
-                 : launch_pdl(dequantize_kernel<true, false>, g, b, 0, stream, packed, s, n, out);
-  else
-    e = out_bf16 ? launch_pdl(dequantize_kernel<false, true>, g, b, 0, stream, packed, s, n, out)
-                 : launch_pdl(dequantize_kernel<false, false>, g, b, 0, stream, packed, s, n, out);
   count_launches(1);
   return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_dequantize(const uint8_t* packed, const Scales& s, int64_t n, void* out, bool out_bf16,
+                              cudaStream_t stream, int num_sms) {
+  return s.book ? launch_book<1>(packed, s, n, out, out_bf16, stream, num_sms)
+                : launch_book<0>(packed, s, n, out, out_bf16, stream, num_sms);
 }
 
 }  // namespace nf4

@@ -9,19 +9,18 @@
 // or int8 (Q = 127, half away from zero, clamped).  The mean is removed first
 // (one fp32 per tensor): mu = fp32(fp64(exact sum) / nb).
 //
-// Sum: every fp32 value is an integer multiple of 2^-149, so each thread adds
-// its values into ten signed 64-bit limbs holding 32 bits each of a 320-bit
-// fixed-point number; integer addition makes the total exact and independent
-// of order.  Warp shuffles and shared memory combine threads, 64-bit atomics
-// combine CTAs.  After a grid barrier every CTA normalises the same limbs,
-// rounds the sum once to fp64 and derives mu.
-//
-// The workspace keeps itself ready for the next call: the barrier is a
-// counter the last arriving CTA resets before it advances an epoch word (the
-// others wait for the epoch to change), and the limbs are double-buffered by
-// epoch parity -- a call adds into limbs[e & 1] and clears limbs[(e + 1) & 1],
-// which the previous call used.  Only the first call needs a zeroed buffer.
-// Codes: one warp per 256-value block.
+// Two kernels, chained with programmatic dependent launch (no grid barrier):
+//   sum     every fp32 value is an integer multiple of 2^-149, so each thread
+//           adds its values into ten signed 64-bit limbs holding 32 bits each
+//           of a 320-bit fixed-point number; integer addition makes the total
+//           exact and independent of order.  Warp shuffles and shared memory
+//           combine threads, 64-bit atomics combine CTAs.  The CTA that
+//           arrives last (a counter in the workspace) normalises the limbs,
+//           rounds the sum once to fp64, writes mu and resets the limbs and
+//           the counter, so the workspace is ready for the next call (only the
+//           first call needs a zeroed buffer).
+//   encode  one warp per 256-value block: residuals, block absmax, codes; it
+//           reads mu after waiting for the sum kernel.
 #include "nf4_common.cuh"
 #include "internal.h"
 
@@ -31,9 +30,8 @@ namespace {
 constexpr int kLimbs = 10;
 
 struct SumWorkspace {
-  unsigned long long limb[2][kLimbs];  // two's-complement running sums of 32-bit digits, by epoch parity
-  unsigned int count;                  // CTAs arrived at the barrier of the current epoch
-  unsigned int epoch;                  // barrier generation
+  unsigned long long limb[kLimbs];  // two's-complement running sums of 32-bit digits
+  unsigned int count;               // CTAs of the running sum that have added their share
 };
 static_assert(sizeof(SumWorkspace) <= kDoubleQuantWorkspace, "workspace");
 
@@ -134,28 +132,11 @@ __device__ float finish_mean(const long long (&limb_in)[kLimbs], int64_t nb) {
   return __double2float_rn(__ddiv_rn(s, (double)nb));
 }
 
-#ifdef NF4_TRACE  // diagnostics build only
-__device__ unsigned long long g_dq_trace[1024 * 8];
-#define DQ_STAMP(slot) (g_dq_trace[blockIdx.x * 8 + (slot)] = global_ns())
-#else
-#define DQ_STAMP(slot) ((void)0)
-#endif
-
-// One cooperative launch (every CTA resident): exact sum -> grid barrier ->
-// codes.  The barrier spins on a counter with a wall-clock bound; if it runs
-// out the error word is set and the codes are skipped.
-__global__ void __launch_bounds__(256) dq_fused_kernel(const float* __restrict__ a, int64_t nb, int dq_code,
-                                                       uint8_t* __restrict__ q, float* __restrict__ scale,
-                                                       float* __restrict__ mean_out, SumWorkspace* __restrict__ ws,
-                                                       unsigned* __restrict__ err) {
-  pdl_launch_dependents();  // the next kernel may set itself up; it still waits for this one to finish
-  // ---- phase 1: this thread's values into the integer limbs of this call's epoch (the epoch
-  // cannot advance before every CTA, this one included, has arrived at the barrier)
-  __shared__ unsigned s_epoch;
-  if (threadIdx.x == 0) {
-    DQ_STAMP(0);
-    s_epoch = *reinterpret_cast<volatile unsigned*>(&ws->epoch);
-  }
+// Exact sum of the absmax values; the last CTA derives mu, writes it and resets the workspace.
+__global__ void __launch_bounds__(256) dq_sum_kernel(const float* __restrict__ a, int64_t nb,
+                                                     float* __restrict__ mean_out, SumWorkspace* __restrict__ ws) {
+  pdl_launch_dependents();  // the encode kernel may set itself up; it waits for this one to finish
+  pdl_wait();
   long long acc[kLimbs];
 #pragma unroll
   for (int L = 0; L < kLimbs; ++L) acc[L] = 0;
@@ -175,62 +156,40 @@ __global__ void __launch_bounds__(256) dq_fused_kernel(const float* __restrict__
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc[L] += __shfl_xor_sync(0xffffffffu, acc[L], off);
   __shared__ long long red[8][kLimbs];
-  __shared__ float s_mu;
-  __shared__ int s_ok;
+  __shared__ int s_last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (lane == 0)
 #pragma unroll
     for (int L = 0; L < kLimbs; ++L) red[warp][L] = acc[L];
   __syncthreads();
-  const unsigned epoch = s_epoch;
-  unsigned long long* limb = ws->limb[epoch & 1];
   if (threadIdx.x < kLimbs) {
     long long t = 0;
     for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w][threadIdx.x];
-    atomicAdd(&limb[threadIdx.x], (unsigned long long)t);  // wraps mod 2^64 = signed add
-  } else if (blockIdx.x == 0 && threadIdx.x < 2 * kLimbs) {
-    ws->limb[(epoch + 1) & 1][threadIdx.x - kLimbs] = 0ull;  // ready for the next call
+    // values of similar magnitude touch two or three limbs: skip the zero ones (all limbs share one cache line)
+    if (t != 0) atomicAdd(&ws->limb[threadIdx.x], (unsigned long long)t);  // wraps mod 2^64 = signed add
   }
   __threadfence();
   __syncthreads();
-
-  // ---- grid barrier (bounded): the last CTA to arrive resets the count and advances the epoch
-  if (threadIdx.x == 0) {
-    DQ_STAMP(1);
-    int ok = 1;
-    if (atomicAdd(&ws->count, 1u) == gridDim.x - 1) {
-      ws->count = 0;
-      __threadfence();
-      atomicExch(&ws->epoch, epoch + 1);
-    } else {
-      const unsigned long long t0 = global_ns();
-      // poll with plain loads (an atomic per poll would contend with the arrivals)
-      while (*reinterpret_cast<volatile unsigned*>(&ws->epoch) == epoch) {
-        __nanosleep(64);
-        if (global_ns() - t0 > kWaitLimitNs) {
-          atomicOr(err, kErrTimeout);
-          ok = 0;
-          break;
-        }
-      }
-    }
-    __threadfence();
-    DQ_STAMP(2);
-    if (ok) {
-      long long l[kLimbs];
-#pragma unroll
-      for (int L = 0; L < kLimbs; ++L) l[L] = (long long)atomicAdd(&limb[L], 0ull);
-      s_mu = finish_mean(l, nb);  // the same integers in every CTA: the same mu
-      if (blockIdx.x == 0) *mean_out = s_mu;
-    }
-    s_ok = ok;
-    DQ_STAMP(3);
-  }
+  if (threadIdx.x == 0) s_last = atomicAdd(&ws->count, 1u) == gridDim.x - 1;
   __syncthreads();
-  if (!s_ok) return;
-  const float mu = s_mu;
+  if (s_last && threadIdx.x == 0) {  // every other CTA has added its share
+    __threadfence();
+    long long l[kLimbs];
+#pragma unroll
+    for (int L = 0; L < kLimbs; ++L) l[L] = (long long)atomicExch(&ws->limb[L], 0ull);  // read and reset
+    *mean_out = finish_mean(l, nb);
+    ws->count = 0;
+  }
+}
 
-  // ---- phase 2: one warp per block of kDqBlock residuals
+// Codes: one warp per block of kDqBlock residuals.
+__global__ void __launch_bounds__(256) dq_encode_kernel(const float* __restrict__ a, int64_t nb, int dq_code,
+                                                        uint8_t* __restrict__ q, float* __restrict__ scale,
+                                                        const float* __restrict__ mean) {
+  pdl_launch_dependents();
+  pdl_wait();  // the sum kernel has finished: mu is in memory
+  const float mu = *mean;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t ngroups = (nb + kDqBlock - 1) / kDqBlock;
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
   const float Q = dq_code == 0 ? kE4M3Top : kInt8Top;
@@ -286,35 +245,26 @@ __global__ void __launch_bounds__(256) dq_fused_kernel(const float* __restrict__
 }  // namespace
 
 cudaError_t launch_double_quant(const float* absmax, int64_t nb, int dq_code, uint8_t* q, float* scale,
-                                float* mean, void* workspace, bool clear, unsigned* err, cudaStream_t stream,
+                                float* mean, void* workspace, bool clear, unsigned* /*err*/, cudaStream_t stream,
                                 int num_sms) {
   cudaError_t e = cudaSuccess;
   if (clear && (e = cudaMemsetAsync(workspace, 0, sizeof(SumWorkspace), stream)) != cudaSuccess) return e;
-  // one CTA per SM: 256 threads and ~1 KB of shared memory, so all are resident
-  int64_t grid = (nb + 256 * 4 - 1) / (256 * 4);
-  if (grid > num_sms) grid = num_sms;
-  if (grid < 1) grid = 1;
   auto* ws = static_cast<SumWorkspace*>(workspace);
-  void* args[] = {(void*)&absmax, (void*)&nb, (void*)&dq_code, (void*)&q, (void*)&scale, (void*)&mean, (void*)&ws,
-                  (void*)&err};
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(256);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelExC(&cfg, (const void*)dq_fused_kernel, args);
+  // sum: each thread at least 16 values (fewer CTAs, fewer atomics on the limbs), at most one CTA per SM
+  int64_t grid = (nb + 256 * 16 - 1) / (256 * 16);
+  grid = grid < 1 ? 1 : (grid > num_sms ? num_sms : grid);
+  e = launch_pdl(dq_sum_kernel, dim3((unsigned)grid), dim3(256), 0, stream, absmax, nb, mean, ws);
   count_launches(1);
-  return e;
+  if (e != cudaSuccess) return e;
+  // encode: one warp per 256-value block, up to 8 CTAs of 8 warps per SM
+  const int64_t ngroups = (nb + kDqBlock - 1) / kDqBlock;
+  int64_t grid2 = (ngroups + 7) / 8;
+  grid2 = grid2 < 1 ? 1 : (grid2 > 8 * (int64_t)num_sms ? 8 * (int64_t)num_sms : grid2);
+  e = launch_pdl(dq_encode_kernel, dim3((unsigned)grid2), dim3(256), 0, stream, (const float*)absmax, nb, dq_code, q,
+                 scale, (const float*)mean);
+  count_launches(1);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace nf4
 
-#ifdef NF4_TRACE
-extern "C" __attribute__((visibility("default"))) int nf4_dq_trace_read(unsigned long long* host) {
-  return (int)cudaMemcpyFromSymbol(host, nf4::g_dq_trace, sizeof(nf4::g_dq_trace));
-}
-#endif

@@ -80,7 +80,7 @@ struct Smem {
   float unit_lut[256];
 };
 
-template <bool kDQ, bool kScaleTma>
+template <bool kDQ, bool kScaleTma, int kBook>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_dx_kernel(Scales s, int rows, int cols, int m_total, int splits, const __grid_constant__ CUtensorMap ymap,
                    const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           a = dq_absmax(sm->unit_lut[kScaleTma ? qcode : s.q[b]], __ldg(s.scale + b / kDqBlock), mu);
         else
           a = kScaleTma ? plain : __ldg(s.absmax + b);
-        const Table T = make_table(a);
+        const Table T = make_table<kBook>(a);
         const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
         uint32_t q[32];  // q[j] = columns 2j, 2j+1 of this row as bf16x2
 #pragma unroll
@@ -301,7 +301,7 @@ int dx_splits(int64_t rows, int64_t cols, int64_t m, int num_sms) {
   return reduction_splits((cols / kTileN) * ((m + kTileM - 1) / kTileM), rows / kTileR, num_sms);
 }
 
-template <bool kDQ, bool kScaleTma>
+template <bool kDQ, bool kScaleTma, int kBook>
 cudaError_t launch_variant(const Scales& s, int rows, int cols, int m, int splits, const CUtensorMap& ymap,
                            const CUtensorMap& wmap, const CUtensorMap& smap, __nv_bfloat16* dx, float* part,
                            unsigned* counters, unsigned* err, int grid, cudaStream_t stream) {
@@ -309,12 +309,12 @@ cudaError_t launch_variant(const Scales& s, int rows, int cols, int m, int split
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!(attr_done.load() & (1ull << dev))) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_dx_kernel<kDQ, kScaleTma>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(gemm_dx_kernel<kDQ, kScaleTma, kBook>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_done.fetch_or(1ull << dev);
   }
-  const cudaError_t e = launch_pdl(gemm_dx_kernel<kDQ, kScaleTma>, dim3(grid), dim3(kThreads), kSmemBytes, stream,
+  const cudaError_t e = launch_pdl(gemm_dx_kernel<kDQ, kScaleTma, kBook>, dim3(grid), dim3(kThreads), kSmemBytes, stream,
                                    s, rows, cols, m, splits, ymap, wmap, smap, dx, part, counters, err);
   count_launches(1);
   return e != cudaSuccess ? e : cudaGetLastError();
@@ -361,12 +361,12 @@ cudaError_t launch_gemm_dx(const uint8_t* packed, const Scales& s, int64_t rows,
   auto* dxb = static_cast<__nv_bfloat16*>(dx);
   const int R = (int)rows, C = (int)cols, M = (int)m;
   if (dq && scale_tma)
-    return launch_variant<true, true>(s, R, C, M, splits, ymap, wmap, smap, dxb, part, counters, err, grid, stream);
+    return s.book ? launch_variant<true, true, 1>(s, R, C, M, splits, ymap, wmap, smap, dxb, part, counters, err, grid, stream) : launch_variant<true, true, 0>(s, R, C, M, splits, ymap, wmap, smap, dxb, part, counters, err, grid, stream);
   if (dq)
-    return launch_variant<true, false>(s, R, C, M, splits, ymap, wmap, smap, dxb, part, counters, err, grid, stream);
+    return s.book ? launch_variant<true, false, 1>(s, R, C, M, splits, ymap, wmap, smap, dxb, part, counters, err, grid, stream) : launch_variant<true, false, 0>(s, R, C, M, splits, ymap, wmap, smap, dxb, part, counters, err, grid, stream);
   if (scale_tma)
-    return launch_variant<false, true>(s, R, C, M, splits, ymap, wmap, smap, dxb, part, counters, err, grid, stream);
-  return launch_variant<false, false>(s, R, C, M, splits, ymap, wmap, smap, dxb, part, counters, err, grid, stream);
+    return s.book ? launch_variant<false, true, 1>(s, R, C, M, splits, ymap, wmap, smap, dxb, part, counters, err, grid, stream) : launch_variant<false, true, 0>(s, R, C, M, splits, ymap, wmap, smap, dxb, part, counters, err, grid, stream);
+  return s.book ? launch_variant<false, false, 1>(s, R, C, M, splits, ymap, wmap, smap, dxb, part, counters, err, grid, stream) : launch_variant<false, false, 0>(s, R, C, M, splits, ymap, wmap, smap, dxb, part, counters, err, grid, stream);
 }
 
 }  // namespace nf4

@@ -84,7 +84,7 @@ __device__ unsigned long long g_trace[1024 * 16];
 #define NF4_STAMP(slot) ((void)0)
 #endif
 
-template <bool kDQ, bool kScaleTma>
+template <bool kDQ, bool kScaleTma, int kBook>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(Scales s, int rows, int cols, int m_total, int splits, const __grid_constant__ CUtensorMap xmap,
                 const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           a = dq_absmax(sm->unit_lut[kScaleTma ? qcode : s.q[b]], __ldg(s.scale + b / kDqBlock), mu);
         else
           a = kScaleTma ? plain : __ldg(s.absmax + b);
-        const Table T = make_table(a);
+        const Table T = make_table<kBook>(a);
         const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
         uint32_t r[32];  // column j of the row: codes 2j, 2j+1 as bf16x2
 #pragma unroll
@@ -401,7 +401,7 @@ size_t gemm_workspace_bytes(int64_t rows, int64_t cols, int64_t m) {
 
 namespace {
 
-template <bool kDQ, bool kScaleTma>
+template <bool kDQ, bool kScaleTma, int kBook>
 cudaError_t launch_variant(const Scales& s, int rows, int cols, int m, int splits, const CUtensorMap& xmap,
                            const CUtensorMap& wmap, const CUtensorMap& smap, __nv_bfloat16* y, float* part,
                            unsigned* counters, unsigned* err, int grid, cudaStream_t stream, const CUtensorMap& tmap,
@@ -412,12 +412,12 @@ cudaError_t launch_variant(const Scales& s, int rows, int cols, int m, int split
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!(attr_done.load() & (1ull << dev))) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<kDQ, kScaleTma>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<kDQ, kScaleTma, kBook>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_done.fetch_or(1ull << dev);
   }
-  const cudaError_t e = launch_pdl(gemm_kernel<kDQ, kScaleTma>, dim3(grid), dim3(kThreads), kSmemBytes, stream, s,
+  const cudaError_t e = launch_pdl(gemm_kernel<kDQ, kScaleTma, kBook>, dim3(grid), dim3(kThreads), kSmemBytes, stream, s,
                                    rows, cols, m, splits, xmap, wmap, smap, y, part, counters, err, tmap, lora_up,
                                    lora_r);
   count_launches(1);
@@ -471,15 +471,19 @@ cudaError_t launch_tc(const uint8_t* packed, const Scales& s, int64_t rows, int6
   const int R = (int)rows, C = (int)cols, M = (int)m;
   const auto* up = static_cast<const __nv_bfloat16*>(lora_up);
   if (dq && scale_tma)
-    return launch_variant<true, true>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
+    return s.book ? launch_variant<true, true, 1>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
+                                      tmap, up, lora_r) : launch_variant<true, true, 0>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
                                       tmap, up, lora_r);
   if (dq)
-    return launch_variant<true, false>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
+    return s.book ? launch_variant<true, false, 1>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
+                                       tmap, up, lora_r) : launch_variant<true, false, 0>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
                                        tmap, up, lora_r);
   if (scale_tma)
-    return launch_variant<false, true>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
+    return s.book ? launch_variant<false, true, 1>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
+                                       tmap, up, lora_r) : launch_variant<false, true, 0>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
                                        tmap, up, lora_r);
-  return launch_variant<false, false>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
+  return s.book ? launch_variant<false, false, 1>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
+                                      tmap, up, lora_r) : launch_variant<false, false, 0>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
                                       tmap, up, lora_r);
 }
 
@@ -495,7 +499,7 @@ size_t lora_t_bytes(int64_t m) { return ((size_t)m * kTileK * 2 + 255) & ~(size_
 
 cudaError_t launch_gemm(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x, int64_t m,
                         void* y, void* workspace, unsigned* err, cudaStream_t stream, int num_sms) {
-  if (m <= 64) return launch_gemv(packed, s, rows, cols, x, (int)m, y, stream, num_sms);
+  if (m <= 64) return launch_gemv(packed, s, rows, cols, x, (int)m, y, err, stream, num_sms);
   return launch_tc(packed, s, rows, cols, x, m, y, gemm_splits(rows, cols, m, num_sms), workspace, err, stream,
                    num_sms, nullptr, nullptr, 0);
 }

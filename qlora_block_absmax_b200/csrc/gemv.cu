@@ -58,7 +58,7 @@ struct GemvGroup {
 };
 constexpr int kPairTableBytes = 256 * 32 * 8;  // fp32 code pairs, one copy per bank
 
-__constant__ float c_code_gemv[16] = NF4_CODE_INIT;
+__constant__ float c_code_gemv[2][16] = {NF4_CODE_INIT, FP4_CODE_INIT};  // by code book: NF4, FP4
 
 __device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -102,7 +102,7 @@ __device__ __forceinline__ void load_step(StepData& d, const uint8_t* __restrict
   }
 }
 
-template <int NT, bool kDQ, bool kTable>
+template <int NT, bool kDQ, bool kTable, int kBook>
 __global__ void __launch_bounds__(kWarps * 32, NT >= 4 ? 1 : 2)
     gemv_kernel(GemvGroup grp, int64_t cols, const __nv_bfloat16* __restrict__ x, int batch) {
   __shared__ float unit_lut[kDQ ? 256 : 1];
@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(kWarps * 32, NT >= 4 ? 1 : 2)
 #pragma unroll
     for (int k = 0; k < kPairTableBytes / 16 / (kWarps * 32); ++k) {
       const int idx = threadIdx.x + k * kWarps * 32;  // 16-byte pieces: two lanes' copies of one entry
-      const float hi = c_code_gemv[(idx >> 4) >> 4], lo = c_code_gemv[(idx >> 4) & 15];
+      const float hi = c_code_gemv[kBook][(idx >> 4) >> 4], lo = c_code_gemv[kBook][(idx >> 4) & 15];
       *reinterpret_cast<float4*>(pair_table + idx * 16) = make_float4(hi, lo, hi, lo);
     }
   }
@@ -169,9 +169,9 @@ __global__ void __launch_bounds__(kWarps * 32, NT >= 4 ? 1 : 2)
       a0 = dq_absmax(unit_lut[cur.q0], cur.s0, mu);
       a1 = dq_absmax(unit_lut[cur.q1], cur.s1, mu);
     }
-    const Table T0 = make_table(a0);
+    const Table T0 = make_table<kBook>(a0);
     Table T1;
-    if (!kTable) T1 = make_table(a1);
+    if (!kTable) T1 = make_table<kBook>(a1);
     const uint32_t w0[8] = {cur.w0[0].x, cur.w0[0].y, cur.w0[0].z, cur.w0[0].w,
                             cur.w0[1].x, cur.w0[1].y, cur.w0[1].z, cur.w0[1].w};
     const uint32_t w1[8] = {cur.w1[0].x, cur.w1[0].y, cur.w1[0].z, cur.w1[0].w,
@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(kWarps * 32, NT >= 4 ? 1 : 2)
   }
 }
 
-template <int NT>
+template <int NT, int kBook>
 cudaError_t launch_nt(const GemvGroup& grp, int64_t cols, const void* x, int batch, bool dq, cudaStream_t stream) {
   const unsigned grid = (unsigned)grp.tile_end[grp.count - 1];
   const auto* xb = static_cast<const __nv_bfloat16*>(x);
@@ -243,37 +243,46 @@ cudaError_t launch_nt(const GemvGroup& grp, int64_t cols, const void* x, int bat
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!(attr_done[dq].load() & (1ull << dev))) {
-      e = cudaFuncSetAttribute(dq ? (const void*)gemv_kernel<NT, true, true> : (const void*)gemv_kernel<NT, false, true>,
+      e = cudaFuncSetAttribute(dq ? (const void*)gemv_kernel<NT, true, true, kBook> : (const void*)gemv_kernel<NT, false, true, kBook>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, kPairTableBytes);
       if (e != cudaSuccess) return e;
       attr_done[dq].fetch_or(1ull << dev);
     }
-    e = dq ? launch_pdl(gemv_kernel<NT, true, true>, dim3(grid), dim3(kWarps * 32), kPairTableBytes, stream, grp,
+    e = dq ? launch_pdl(gemv_kernel<NT, true, true, kBook>, dim3(grid), dim3(kWarps * 32), kPairTableBytes, stream, grp,
                         cols, xb, batch)
-           : launch_pdl(gemv_kernel<NT, false, true>, dim3(grid), dim3(kWarps * 32), kPairTableBytes, stream, grp,
+           : launch_pdl(gemv_kernel<NT, false, true, kBook>, dim3(grid), dim3(kWarps * 32), kPairTableBytes, stream, grp,
                         cols, xb, batch);
   } else {
-    e = dq ? launch_pdl(gemv_kernel<NT, true, false>, dim3(grid), dim3(kWarps * 32), 0, stream, grp, cols, xb, batch)
-           : launch_pdl(gemv_kernel<NT, false, false>, dim3(grid), dim3(kWarps * 32), 0, stream, grp, cols, xb,
+    e = dq ? launch_pdl(gemv_kernel<NT, true, false, kBook>, dim3(grid), dim3(kWarps * 32), 0, stream, grp, cols, xb, batch)
+           : launch_pdl(gemv_kernel<NT, false, false, kBook>, dim3(grid), dim3(kWarps * 32), 0, stream, grp, cols, xb,
                         batch);
   }
   count_launches(1);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
+template <int kBook>
+cudaError_t launch_book(const GemvGroup& grp, int64_t cols, const void* x, int batch, bool dq, cudaStream_t stream) {
+  if (batch <= 8) return launch_nt<1, kBook>(grp, cols, x, batch, dq, stream);
+  if (batch <= 16) return launch_nt<2, kBook>(grp, cols, x, batch, dq, stream);
+  if (batch <= 32) return launch_nt<4, kBook>(grp, cols, x, batch, dq, stream);
+  return launch_nt<8, kBook>(grp, cols, x, batch, dq, stream);
+}
+
 cudaError_t launch_group(const GemvGroup& grp, int64_t cols, const void* x, int batch, bool dq,
                          cudaStream_t stream) {
-  if (batch <= 8) return launch_nt<1>(grp, cols, x, batch, dq, stream);
-  if (batch <= 16) return launch_nt<2>(grp, cols, x, batch, dq, stream);
-  if (batch <= 32) return launch_nt<4>(grp, cols, x, batch, dq, stream);
-  return launch_nt<8>(grp, cols, x, batch, dq, stream);
+  return grp.s[0].book ? launch_book<1>(grp, cols, x, batch, dq, stream) : launch_book<0>(grp, cols, x, batch, dq, stream);
 }
 
 }  // namespace
 
 // batch <= 64: the activation rows are spread over ceil(batch / 8) n-tiles
 cudaError_t launch_gemv(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x, int batch,
-                        void* y, cudaStream_t stream, int /*num_sms*/) {
+                        void* y, unsigned* err, cudaStream_t stream, int num_sms) {
+  if (batch <= 8) {
+    const GemvItem item = {packed, s, x, y, rows, cols};
+    return launch_gemv_items(&item, 1, batch, err, stream, num_sms);
+  }
   if (rows / 16 > INT32_MAX) return cudaErrorInvalidValue;
   GemvGroup grp = {};
   grp.packed[0] = packed;
@@ -287,8 +296,14 @@ cudaError_t launch_gemv(const uint8_t* packed, const Scales& s, int64_t rows, in
 // several weights with the same cols and scale kind, one input x: one launch whose CTAs cover the 16-row
 // tiles of every weight in turn
 cudaError_t launch_gemv_group(const uint8_t* const* packed, const Scales* s, const int64_t* rows, int count,
-                              int64_t cols, const void* x, int batch, void* const* y, cudaStream_t stream) {
+                              int64_t cols, const void* x, int batch, void* const* y, unsigned* err,
+                              cudaStream_t stream, int num_sms) {
   if (count < 1 || count > kMaxGroup) return cudaErrorInvalidValue;
+  if (batch <= 8) {
+    GemvItem items[kMaxGroup];
+    for (int i = 0; i < count; ++i) items[i] = GemvItem{packed[i], s[i], x, y[i], rows[i], cols};
+    return launch_gemv_items(items, count, batch, err, stream, num_sms);
+  }
   GemvGroup grp = {};
   int64_t tiles = 0;
   for (int i = 0; i < count; ++i) {

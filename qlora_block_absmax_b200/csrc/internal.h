@@ -39,9 +39,10 @@ struct Scales {
   const float* scale;    // second-level block absmax
   const float* mean;     // device pointer to the removed mean
   int dq_code;           // 0 = E4M3, 1 = int8
+  int book;              // 4-bit code book: 0 = NF4, 1 = FP4 (E2M1 / 6)
 };
 
-cudaError_t launch_quantize(const void* src, bool bf16, int64_t n, uint8_t* packed, float* absmax,
+cudaError_t launch_quantize(const void* src, bool bf16, int64_t n, uint8_t* packed, float* absmax, int book,
                             cudaStream_t stream, int num_sms);
 
 // workspace: zero before its first use, left ready by every completed call; `clear` zeroes it first
@@ -53,13 +54,28 @@ constexpr size_t kDoubleQuantWorkspace = 256;
 cudaError_t launch_dequantize(const uint8_t* packed, const Scales& s, int64_t n, void* out, bool out_bf16,
                               cudaStream_t stream, int num_sms);
 
+// batch <= 8 runs on the persistent stream kernel (gemv_stream.cu), 9..64 on the per-tile kernel (gemv.cu)
 cudaError_t launch_gemv(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x,
-                        int batch, void* y, cudaStream_t stream, int num_sms);
+                        int batch, void* y, unsigned* err, cudaStream_t stream, int num_sms);
 
 // several weights (same cols and scale kind) on one input in one launch, count <= kMaxGroup
 constexpr int kMaxGroup = 4;
 cudaError_t launch_gemv_group(const uint8_t* const* packed, const Scales* s, const int64_t* rows, int count,
-                              int64_t cols, const void* x, int batch, void* const* y, cudaStream_t stream);
+                              int64_t cols, const void* x, int batch, void* const* y, unsigned* err,
+                              cudaStream_t stream, int num_sms);
+
+// one GEMV of the persistent stream: weight [rows, cols] (rows % 16 == 0, cols % 64 == 0), its input x [batch, cols]
+// and output y [batch, rows]; up to kMaxStreamItems of them in one launch, batch 1..8
+struct GemvItem {
+  const uint8_t* packed;
+  Scales s;
+  const void* x;
+  void* y;
+  int64_t rows, cols;
+};
+constexpr int kMaxStreamItems = 256;
+cudaError_t launch_gemv_items(const GemvItem* items, int count, int batch, unsigned* err, cudaStream_t stream,
+                              int num_sms);
 
 size_t gemm_workspace_bytes(int64_t rows, int64_t cols, int64_t m);
 cudaError_t launch_gemm(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x,

@@ -18,11 +18,16 @@ struct Table {  // byte pools: low/high bytes of bf16(code[i] * a), i in 0..7 (A
   uint32_t la0, la1, lb0, lb1, ha0, ha1, hb0, hb1;
 };
 
+// kBook: the code book, 0 = NF4, 1 = FP4 (E2M1 / 6 by bit pattern; "bitsandbytes", "Glossary")
+template <int kBook = 0>
 __device__ __forceinline__ Table make_table(float a) {
-  constexpr float code[16] = NF4_CODE_INIT;
+  constexpr float nf4[16] = NF4_CODE_INIT;
+  constexpr float fp4[16] = FP4_CODE_INIT;
   uint32_t r[8];
 #pragma unroll
-  for (int m = 0; m < 8; ++m) r[m] = pack_bf16x2(__fmul_rn(code[2 * m], a), __fmul_rn(code[2 * m + 1], a));
+  for (int m = 0; m < 8; ++m)
+    r[m] = pack_bf16x2(__fmul_rn(kBook ? fp4[2 * m] : nf4[2 * m], a),
+                       __fmul_rn(kBook ? fp4[2 * m + 1] : nf4[2 * m + 1], a));
   Table T;
   T.la0 = prmt(r[0], r[1], 0x6420);
   T.la1 = prmt(r[2], r[3], 0x6420);

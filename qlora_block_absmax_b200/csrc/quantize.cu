@@ -18,6 +18,7 @@
 // bits.  x is first estimated as q = w * RN(1/a) (within 3 * 2^-24 of x); one
 // fused multiply-add rounded down puts q's bucket in the low 5 mantissa bits
 // of its result, a shuffle fetches the entry, and code = base + (q > entry).
+// Elements are decided in pairs with paired fp32 arithmetic (f32x2).
 // When q lies within 2^-19 of the entry -- where the estimate, or the 4 bits
 // stored in the entry, could change the decision -- the exact quotient
 // __fdiv_rn(w, a) is compared with the exact threshold instead.  Every code is
@@ -30,6 +31,9 @@ namespace {
 
 __constant__ uint32_t c_q32[32] = NF4_Q32_INIT;
 __constant__ float c_threshold[15] = NF4_THRESHOLD_INIT;
+// FP4 (E2M1 / 6): 16 buckets over [0, 1] of |x| and the 7 magnitude thresholds
+__constant__ uint32_t c_q16[16] = FP4_Q16_INIT;
+__constant__ float c_f4threshold[7] = FP4_THRESHOLD_INIT;
 
 constexpr float kNearThreshold = 0x1p-19f;
 constexpr float kTinyScale = 0x1p-120f;  // below this 1/a may overflow: divide exactly
@@ -45,6 +49,28 @@ __device__ __noinline__ int code_exact(float w, float a) {
   return code;
 }
 
+// FP4: the magnitude code of |x| against the exact magnitude thresholds, with the sign of x in bit 3 (a zero
+// result keeps the sign: -0 is pattern 8)
+__device__ __noinline__ int code_exact_fp4(float w, float a) {
+  const float x = __fdiv_rn(w, a);
+  const float ax = fabsf(x);
+  int code = 0;
+#pragma unroll
+  for (int i = 0; i < 7; ++i) code += (ax > c_f4threshold[i]) ? 1 : 0;
+  return code | ((__float_as_uint(x) >> 31) << 3);
+}
+
+// FP4 fast path: 16 magnitude buckets (lanes 0..15 of the warp hold them; lanes 16..31 repeat them); q estimates
+// w / a within 3 * 2^-24 and has the sign of w
+__device__ __forceinline__ uint32_t code_fast_fp4(uint32_t entry, float q, float& gap) {
+  const float aq = fabsf(q);
+  const float v = __fmaf_rd(aq, 16.0f * NF4_Q32_SCALE, 0x1p23f);  // low 4 mantissa bits: the bucket
+  const uint32_t e = __shfl_sync(0xffffffffu, entry, __float_as_int(v));
+  const float thr = __uint_as_float(e);
+  gap = fminf(gap, fabsf(aq - thr));
+  return (e & 15u) + (aq > thr ? 1u : 0u) + ((__float_as_uint(q) >> 31) << 3);
+}
+
 // `entry` is this lane's bucket word; every lane of the warp must call this
 // (the lookup is a shuffle).  q estimates w / a within 3 * 2^-24.  `gap`
 // tracks the smallest distance between an estimate and its entry.
@@ -56,6 +82,35 @@ __device__ __forceinline__ uint32_t code_fast(uint32_t entry, float q, float& ga
   const float thr = __uint_as_float(e);
   gap = fminf(gap, fabsf(q - thr));
   return (e & 15u) + (q > thr ? 1u : 0u);
+}
+
+// Two elements of NF4 at once: q = w * r and the bucket value v = RD(16 S q + 2^23 + 16) as paired fp32
+// operations (each half rounded as its scalar form), two shuffles fetch the bucket entries, and d = thr - q (also
+// paired, exact in sign: the difference of two fp32 values is never rounded to zero) gives both the decision
+// (q > thr iff d's sign bit is set) and the distance to the threshold.
+__device__ __forceinline__ void code_fast_pair(uint32_t entry, float w0, float w1, float r, float& gap,
+                                               uint32_t& c0, uint32_t& c1) {
+  unsigned long long wq, rr, q, v, d, t;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(wq) : "f"(w0), "f"(w1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(rr) : "f"(r));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(q) : "l"(wq), "l"(rr));
+  {
+    unsigned long long sc, of;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(sc) : "f"(16.0f * NF4_Q32_SCALE));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(of) : "f"(0x1p23f + 16.0f));
+    asm("fma.rm.f32x2 %0, %1, %2, %3;" : "=l"(v) : "l"(q), "l"(sc), "l"(of));
+  }
+  uint32_t v0, v1;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(v0), "=r"(v1) : "l"(v));
+  const uint32_t e0 = __shfl_sync(0xffffffffu, entry, (int)v0);
+  const uint32_t e1 = __shfl_sync(0xffffffffu, entry, (int)v1);
+  asm("mov.b64 %0, {%1, %2};" : "=l"(t) : "r"(e0), "r"(e1));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(t), "l"(q));
+  uint32_t d0, d1;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(d0), "=r"(d1) : "l"(d));
+  gap = fminf(gap, fminf(fabsf(__uint_as_float(d0)), fabsf(__uint_as_float(d1))));
+  c0 = (e0 & 15u) + (d0 >> 31);
+  c1 = (e1 & 15u) + (d1 >> 31);
 }
 
 // two codes -> one byte (first in the high nibble); four bytes -> one word
@@ -71,13 +126,13 @@ __device__ __forceinline__ float load1(const void* src, int64_t i) {
   return static_cast<const float*>(src)[i];
 }
 
-template <bool kBF16>
+template <bool kBF16, bool kFp4>
 __global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ src, int64_t n,
                                                        uint8_t* __restrict__ packed,
                                                        float* __restrict__ absmax) {
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
-  const uint32_t entry = c_q32[lane];
+  const uint32_t entry = kFp4 ? c_q16[lane & 15] : c_q32[lane];
   const int sub = lane & 3;                                  // which 16 of the block's 64
   const unsigned gmask = 0xfu << (lane & ~3);                // the 4 lanes of this block
   const int64_t nfull = n / kBlock;
@@ -142,15 +197,20 @@ __global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ 
     const float r = __frcp_rn(zero ? 1.0f : a);
     uint32_t c[16];
     float gap = 1.0f;
+    if (kFp4) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) c[i] = code_fast(entry, __fmul_rn(w[i], r), gap);
+      for (int i = 0; i < 16; ++i) c[i] = code_fast_fp4(entry, __fmul_rn(w[i], r), gap);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; i += 2) code_fast_pair(entry, w[i], w[i + 1], r, gap, c[i], c[i + 1]);
+    }
     if (exact || gap <= kNearThreshold) {  // rare: redo this lane's 16 elements with exact quotients
 #pragma unroll
-      for (int i = 0; i < 16; ++i) c[i] = (uint32_t)code_exact(w[i], a);
+      for (int i = 0; i < 16; ++i) c[i] = (uint32_t)(kFp4 ? code_exact_fp4(w[i], a) : code_exact(w[i], a));
     }
-    // Step 4: element 2j -> high nibble of byte j
+    // Step 4: element 2j -> high nibble of byte j; an all-zero block is all zero codes (NF4 7, FP4 +0)
     uint32_t lo = pack8(c, 0), hi = pack8(c, 8);
-    if (zero) lo = hi = 0x77777777u;
+    if (zero) lo = hi = kFp4 ? 0u : 0x77777777u;
 #pragma unroll
     for (int i = 0; i < (kBF16 ? 2 : 4); ++i) cur[i] = nxt[i];
     if (!live) continue;
@@ -158,13 +218,13 @@ __global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ 
       *reinterpret_cast<uint2*>(packed + first / 2) = make_uint2(lo, hi);
     } else {
       // short block: write only bytes holding real elements; an odd tail keeps
-      // the zero code (7) in its low nibble
+      // the zero code (NF4 7, FP4 +0) in its low nibble
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int64_t e = first + 2 * j;  // element in the high nibble
         if (e < n) {
           uint8_t v = (uint8_t)((j < 4 ? lo : hi) >> (8 * (j & 3)));
-          if (e + 1 >= n) v = (uint8_t)((v & 0xf0u) | 0x7u);
+          if (e + 1 >= n) v = (uint8_t)((v & 0xf0u) | (kFp4 ? 0x0u : 0x7u));
           packed[first / 2 + j] = v;
         }
       }
@@ -176,23 +236,26 @@ __global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ 
 
 }  // namespace
 
-cudaError_t launch_quantize(const void* src, bool bf16, int64_t n, uint8_t* packed, float* absmax,
+cudaError_t launch_quantize(const void* src, bool bf16, int64_t n, uint8_t* packed, float* absmax, int book,
                             cudaStream_t stream, int num_sms) {
   const int64_t nblocks = (n + kBlock - 1) / kBlock;
   const int per_cta = 256 / 4;
   int64_t grid = (nblocks + per_cta - 1) / per_cta;
+  const void* fn = bf16 ? (book ? (const void*)quantize_kernel<true, true> : (const void*)quantize_kernel<true, false>)
+                        : (book ? (const void*)quantize_kernel<false, true> : (const void*)quantize_kernel<false, false>);
   int occ = 0;  // one wave: as many CTAs as fit on the SMs at once
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, bf16 ? (const void*)quantize_kernel<true>
-                                                                : (const void*)quantize_kernel<false>,
-                                                    256, 0) != cudaSuccess || occ < 1)
-    occ = 1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, 256, 0) != cudaSuccess || occ < 1) occ = 1;
   const int64_t cap = (int64_t)num_sms * occ;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
-  const cudaError_t e = bf16 ? launch_pdl(quantize_kernel<true>, dim3((unsigned)grid), dim3(256), 0, stream, src, n,
-                                           packed, absmax)
-                              : launch_pdl(quantize_kernel<false>, dim3((unsigned)grid), dim3(256), 0, stream, src, n,
-                                           packed, absmax);
+  const dim3 g((unsigned)grid), b(256);
+  cudaError_t e;
+  if (bf16)
+    e = book ? launch_pdl(quantize_kernel<true, true>, g, b, 0, stream, src, n, packed, absmax)
+             : launch_pdl(quantize_kernel<true, false>, g, b, 0, stream, src, n, packed, absmax);
+  else
+    e = book ? launch_pdl(quantize_kernel<false, true>, g, b, 0, stream, src, n, packed, absmax)
+             : launch_pdl(quantize_kernel<false, false>, g, b, 0, stream, src, n, packed, absmax);
   count_launches(1);
   return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -54,6 +54,19 @@ int main(void) {
   const nf4_weight *group[5] = {&w, &w, &w, &w, &w};
   void *ys[5] = {(void *)0x40000, (void *)0x40000, (void *)0x40000, (void *)0x40000, (void *)0x40000};
   CHECK(nf4_gemv_grouped(group, 5, (const void *)0x30000, 1, ys, s) == NF4_ERR_INVALID_ARG); /* more than 4 */
+  /* the multi-weight GEMV: 1..NF4_GEMV_STREAM_MAX weights, batch 1..8 */
+  const void *xs[2] = {(const void *)0x30000, (const void *)0x30000};
+  CHECK(nf4_gemv_stream(&w, xs, ys, 0, 1, s) == NF4_ERR_INVALID_ARG);
+  CHECK(nf4_gemv_stream(&w, xs, ys, NF4_GEMV_STREAM_MAX + 1, 1, s) == NF4_ERR_INVALID_ARG);
+  CHECK(nf4_gemv_stream(&w, xs, ys, 1, 9, s) == NF4_ERR_INVALID_ARG);
+  /* the code book: NF4 or FP4 only */
+  CHECK(nf4_quantize_typed((const void *)0x1000, NF4_F32, 10, 64, 2, (uint8_t *)0x2000, (float *)0x3000, s) ==
+        NF4_ERR_INVALID_ARG);
+  CHECK(nf4_quantize_typed((const void *)0x1000, NF4_F32, 0, 64, NF4_QUANT_FP4, (uint8_t *)0x2000, (float *)0x3000,
+                           s) == NF4_OK);
+  w.quant_type = 7;
+  CHECK(nf4_dequantize(&w, (void *)0x40000, NF4_BF16, s) == NF4_ERR_INVALID_ARG);
+  w.quant_type = NF4_QUANT_NF4;
   w.blocksize = 32;
   CHECK(nf4_dequantize(&w, (void *)0x40000, NF4_BF16, s) == NF4_ERR_UNSUPPORTED);
   if (failures) return 1;

@@ -73,6 +73,11 @@ def test_host_validation_before_cuda(lib):
     assert lib.nf4_double_quant(0x1000, 10, 256, 5, 0x2000, 0x3000, 0x4000, 0x5000, 256, s) == E["NF4_ERR_INVALID_ARG"]
     assert lib.nf4_double_quant(0x1000, 10, 256, 0, 0x2000, 0x3000, 0x4000, 0x5000, 8, s) == E["NF4_ERR_INVALID_ARG"]
     assert lib.nf4_double_quant(0x1000, 0, 256, 0, 0x2000, 0x3000, 0x4000, 0x5000, 256, s) == E["NF4_OK"]
+    too_many = 2 ** 31  # one past NF4_DQ_MAX_NB: the exact-sum limbs would no longer be exact
+    assert lib.nf4_double_quant(0x1000, too_many, 256, 0, 0x2000, 0x3000, 0x4000, 0x5000, 256, s) == \
+        E["NF4_ERR_INVALID_ARG"]
+    assert lib.nf4_double_quant_noalloc(0x1000, too_many, 256, 0, 0x2000, 0x3000, 0x4000, s) == \
+        E["NF4_ERR_INVALID_ARG"]
     assert lib.nf4_double_quant_workspace_bytes(1 << 20) >= 128
     # weight descriptor checks
     w = weight(bs=32)
@@ -168,3 +173,37 @@ def test_plain_c_client(tmp_path):
                     "-Wl,-rpath," + libdir, "-lm", "-o", exe], check=True)
     r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0 and r.stdout.strip() == "ok", r.stderr
+
+
+def test_host_validation_gemv_stream(lib):
+    """nf4_gemv_stream rejects bad arguments on the host, before any CUDA call: count 1..256, batch 1..8,
+    per-weight shape rules, null and misaligned pointers; a list of empty weights launches nothing"""
+    E = {v: k for k, v in _lib.STATUS_NAMES.items()}
+    s = None
+    n = 257
+    ws = (_lib.NF4Weight * n)(*[weight() for _ in range(n)])
+    xs = (ctypes.c_void_p * n)(*[0x9000] * n)
+    ys = (ctypes.c_void_p * n)(*[0xa000] * n)
+    assert lib.nf4_gemv_stream(ws, xs, ys, 0, 1, s) == E["NF4_ERR_INVALID_ARG"]
+    assert lib.nf4_gemv_stream(ws, xs, ys, 257, 1, s) == E["NF4_ERR_INVALID_ARG"]
+    assert lib.nf4_gemv_stream(ws, xs, ys, 2, 0, s) == E["NF4_ERR_INVALID_ARG"]
+    assert lib.nf4_gemv_stream(ws, xs, ys, 2, 9, s) == E["NF4_ERR_INVALID_ARG"]
+    assert lib.nf4_gemv_stream(None, xs, ys, 2, 1, s) == E["NF4_ERR_INVALID_ARG"]
+    assert lib.nf4_gemv_stream(ws, None, ys, 2, 1, s) == E["NF4_ERR_INVALID_ARG"]
+    assert lib.nf4_gemv_stream(ws, xs, None, 2, 1, s) == E["NF4_ERR_INVALID_ARG"]
+    mixed = (_lib.NF4Weight * 3)(weight(), weight(cols=96), weight())
+    assert lib.nf4_gemv_stream(mixed, xs, ys, 3, 1, s) == E["NF4_ERR_UNSUPPORTED"]
+    mixed = (_lib.NF4Weight * 2)(weight(), weight(rows=40))
+    assert lib.nf4_gemv_stream(mixed, xs, ys, 2, 1, s) == E["NF4_ERR_UNSUPPORTED"]
+    mixed = (_lib.NF4Weight * 2)(weight(), weight(bs=128))
+    assert lib.nf4_gemv_stream(mixed, xs, ys, 2, 1, s) == E["NF4_ERR_UNSUPPORTED"]
+    mixed = (_lib.NF4Weight * 2)(weight(), weight(absmax=0))
+    assert lib.nf4_gemv_stream(mixed, xs, ys, 2, 1, s) == E["NF4_ERR_INVALID_ARG"]
+    xs_bad = (ctypes.c_void_p * 2)(0x9000, 0x9008)
+    assert lib.nf4_gemv_stream(ws, xs_bad, ys, 2, 1, s) == E["NF4_ERR_MISALIGNED"]
+    ys_bad = (ctypes.c_void_p * 2)(0xa000, 0xa002)
+    assert lib.nf4_gemv_stream(ws, xs, ys_bad, 2, 1, s) == E["NF4_ERR_MISALIGNED"]
+    xs_null = (ctypes.c_void_p * 2)(0x9000, None)
+    assert lib.nf4_gemv_stream(ws, xs_null, ys, 2, 1, s) == E["NF4_ERR_INVALID_ARG"]
+    empty = (_lib.NF4Weight * 2)(weight(rows=0), weight(cols=0))
+    assert lib.nf4_gemv_stream(empty, xs_null, ys, 2, 1, s) == E["NF4_OK"]  # nothing to compute, nothing launched

@@ -3,8 +3,9 @@ allocate device memory (a fixed memory budget, or a host framework that owns
 the allocator), with its scratch in a static array inside the library.
 
 Called through the C ABI and compared with nf4_double_quant (caller-provided
-workspace) bit for bit -- the tolerance every double-quant test uses -- on two
-calls in a row, so a second call also shows the shared scratch is cleared.
+workspace) bit for bit -- the tolerance every double-quant test uses: two calls
+in a row on the shared array, with different sizes, each match the workspace
+entry point exactly.
 """
 import ctypes
 
