@@ -91,7 +91,10 @@ typedef enum { NF4_QUANT_NF4 = 0, NF4_QUANT_FP4 = 1 } nf4_quant_type;
  *   absmax_q      nb 8-bit codes of the mean-removed scales (double quant)
  *   absmax_scale  ceil(nb/dq_blocksize) fp32 second-level block absmax values
  *   absmax_mean   1 fp32: the mean removed before second-level quantization
- *   blocksize     64 (only value implemented); dq_blocksize 256; dq_code nf4_dq_code
+ *   blocksize     level-1 block size: 32, 64, 128 or 256 for nf4_dequantize;
+ *                 the matmuls (GEMV, GEMM and their variants) take 64 only
+ *                 and return NF4_ERR_UNSUPPORTED for the others
+ *   dq_blocksize  256; dq_code nf4_dq_code
  *   quant_type    nf4_quant_type of the codes (0 = NF4: a zero-initialised
  *                 descriptor describes NF4 codes) */
 typedef struct {
@@ -112,7 +115,8 @@ typedef struct {
  *   src         device, n elements of src_dtype (NF4_F32 or NF4_BF16); 16-byte aligned
  *   packed_out  device, ceil(n/2) bytes; an odd tail's low nibble is 7 (zero code)
  *   absmax_out  device, ceil(n/blocksize) fp32 (the level-1 scales a)
- * blocksize must be 64 (else NF4_ERR_UNSUPPORTED). */
+ * blocksize is 32, 64, 128 or 256 (else NF4_ERR_UNSUPPORTED); 64 is the size
+ * the matmuls take. */
 NF4_API nf4_status nf4_quantize(const void *src, int32_t src_dtype, int64_t n, int32_t blocksize,
                         uint8_t *packed_out, float *absmax_out, nf4_stream_t stream);
 
@@ -175,7 +179,8 @@ NF4_API nf4_status nf4_double_quant_noalloc(const float *absmax, int64_t nb, int
  * precision with the scale and the code book).  With double quantization the
  * scale is first reconstructed: a^ = fp32(fp32(fp32(dec(q)/Q) * m) + mu).
  * w^ = fp32(code[idx] * a^); out = w^ (NF4_F32) or bf16_rn(w^) (NF4_BF16).
- *   w    weight descriptor (rows*cols elements; rows/cols need no alignment)
+ *   w    weight descriptor (rows*cols elements; rows/cols need no alignment;
+ *        blocksize 32, 64, 128 or 256, else NF4_ERR_UNSUPPORTED)
  *   out  device, rows*cols elements of out_dtype, 16-byte aligned */
 NF4_API nf4_status nf4_dequantize(const nf4_weight *w, void *out, int32_t out_dtype, nf4_stream_t stream);
 

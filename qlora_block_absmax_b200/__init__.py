@@ -124,17 +124,20 @@ def double_quant(absmax: torch.Tensor, code: str = "e4m3", dq_blocksize: int = D
 
 
 def quantize_weight(w: torch.Tensor, use_double_quant: bool = True, code: str = "e4m3",
-                    stream=None, quant_type: str = "nf4") -> QuantizedWeight:
-    """Quantize a 2-D weight [rows, cols] (nn.Linear layout: out x in) to NF4 (or FP4: quant_type="fp4")."""
+                    stream=None, quant_type: str = "nf4", blocksize: int = BLOCKSIZE) -> QuantizedWeight:
+    """Quantize a 2-D weight [rows, cols] (nn.Linear layout: out x in) to NF4 (or FP4: quant_type="fp4").
+
+    blocksize is 32, 64, 128 or 256; the matmuls take 64-element blocks only (dequantize takes all four)."""
     if w.dim() != 2:
         raise ValueError("quantize_weight takes a 2-D [rows, cols] tensor")
-    packed, absmax = quantize(w, stream=stream, quant_type=quant_type)
+    packed, absmax = quantize(w, blocksize=blocksize, stream=stream, quant_type=quant_type)
     qt = _QUANT_TYPES[quant_type]
-    qw = QuantizedWeight(packed=packed, rows=w.shape[0], cols=w.shape[1], absmax=absmax, quant_type=qt)
+    qw = QuantizedWeight(packed=packed, rows=w.shape[0], cols=w.shape[1], absmax=absmax, blocksize=blocksize,
+                         quant_type=qt)
     if use_double_quant:
         q, scale, mean = double_quant(absmax, code, stream=stream)
         qw = QuantizedWeight(packed=packed, rows=w.shape[0], cols=w.shape[1], absmax_q=q, absmax_scale=scale,
-                             absmax_mean=mean, dq_code=_DQ_CODES[code], quant_type=qt)
+                             absmax_mean=mean, dq_code=_DQ_CODES[code], blocksize=blocksize, quant_type=qt)
     return qw
 
 

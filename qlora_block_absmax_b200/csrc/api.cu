@@ -49,11 +49,14 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 nf4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? NF4_OK : NF4_ERR_CUDA; }
 
-// Common checks of a weight descriptor; fills the kernel-side scale view.
-nf4_status check_weight(const nf4_weight* w, nf4::Scales* s) {
+bool level1_blocksize(int32_t b) { return b == 32 || b == 64 || b == 128 || b == 256; }
+
+// Common checks of a weight descriptor; fills the kernel-side scale view.  The
+// matmuls take 64-element blocks only; dequantization takes every level-1 size.
+nf4_status check_weight(const nf4_weight* w, nf4::Scales* s, bool any_blocksize = false) {
   if (w == nullptr || w->packed == nullptr) return NF4_ERR_INVALID_ARG;
   if (w->rows < 0 || w->cols < 0) return NF4_ERR_INVALID_ARG;
-  if (w->blocksize != nf4::kBlock) return NF4_ERR_UNSUPPORTED;
+  if (any_blocksize ? !level1_blocksize(w->blocksize) : w->blocksize != nf4::kBlock) return NF4_ERR_UNSUPPORTED;
   if (w->quant_type != NF4_QUANT_NF4 && w->quant_type != NF4_QUANT_FP4) return NF4_ERR_INVALID_ARG;
   if (!aligned(w->packed, 16)) return NF4_ERR_MISALIGNED;
   if (w->absmax != nullptr) {
@@ -139,14 +142,14 @@ nf4_status nf4_quantize_typed(const void* src, int32_t src_dtype, int64_t n, int
   if (n < 0) return NF4_ERR_INVALID_ARG;
   if (quant_type != NF4_QUANT_NF4 && quant_type != NF4_QUANT_FP4) return NF4_ERR_INVALID_ARG;
   if (src_dtype != NF4_F32 && src_dtype != NF4_BF16) return NF4_ERR_INVALID_ARG;
-  if (blocksize != nf4::kBlock) return NF4_ERR_UNSUPPORTED;
+  if (!level1_blocksize(blocksize)) return NF4_ERR_UNSUPPORTED;
   if (n == 0) return NF4_OK;
   if (src == nullptr || packed_out == nullptr || absmax_out == nullptr) return NF4_ERR_INVALID_ARG;
   if (!aligned(src, 16) || !aligned(packed_out, 16) || !aligned(absmax_out, 4)) return NF4_ERR_MISALIGNED;
   DeviceInfo d;
   nf4_status st = device_info(&d);
   if (st != NF4_OK) return st;
-  return from_cuda(nf4::launch_quantize(src, src_dtype == NF4_BF16, n, packed_out, absmax_out, quant_type,
+  return from_cuda(nf4::launch_quantize(src, src_dtype == NF4_BF16, n, blocksize, packed_out, absmax_out, quant_type,
                                         reinterpret_cast<cudaStream_t>(stream), d.num_sms));
 }
 
@@ -227,7 +230,7 @@ nf4_status nf4_double_quant_noalloc(const float* absmax, int64_t nb, int32_t dq_
 
 nf4_status nf4_dequantize(const nf4_weight* w, void* out, int32_t out_dtype, nf4_stream_t stream) {
   nf4::Scales s;
-  nf4_status st = check_weight(w, &s);
+  nf4_status st = check_weight(w, &s, true);
   if (st != NF4_OK) return st;
   if (out_dtype != NF4_F32 && out_dtype != NF4_BF16) return NF4_ERR_INVALID_ARG;
   const int64_t n = w->rows * w->cols;
@@ -236,7 +239,7 @@ nf4_status nf4_dequantize(const nf4_weight* w, void* out, int32_t out_dtype, nf4
   if (!aligned(out, 16)) return NF4_ERR_MISALIGNED;
   DeviceInfo d;
   if ((st = device_info(&d)) != NF4_OK) return st;
-  return from_cuda(nf4::launch_dequantize(w->packed, s, n, out, out_dtype == NF4_BF16,
+  return from_cuda(nf4::launch_dequantize(w->packed, s, n, w->blocksize, out, out_dtype == NF4_BF16,
                                           reinterpret_cast<cudaStream_t>(stream), d.num_sms));
 }
 

@@ -1,4 +1,4 @@
-// gemv.cu -- decode GEMV (and skinny GEMM, m <= 64) with on-the-fly NF4 dequantization.
+// gemv.cu -- decode GEMV (batch 1..8) with on-the-fly 4-bit dequantization, one CTA per 16-row tile.
 //
 // "bitsandbytes" (ozercemkelahmet.com/tools), "How it works" Step 5: each block
 // is expanded back to 16-bit with its scale and the code book, then
@@ -127,10 +127,15 @@ __global__ void __launch_bounds__(kWarps * 32, NT >= 4 ? 1 : 2)
   const int64_t rows = (int64_t)(tile1 - tile0) * 16;
   if (kDQ) unit_lut[threadIdx.x & 255] = dq_unit(threadIdx.x & 255, s.dq_code);
   if (kTable) {
+    // the 16 levels through shared memory first: the table's lanes read them at different indices, which a
+    // constant-memory read would serialise
+    __shared__ float code_s[16];
+    if (threadIdx.x < 16) code_s[threadIdx.x] = c_code_gemv[kBook][threadIdx.x];
+    __syncthreads();
 #pragma unroll
     for (int k = 0; k < kPairTableBytes / 16 / (kWarps * 32); ++k) {
       const int idx = threadIdx.x + k * kWarps * 32;  // 16-byte pieces: two lanes' copies of one entry
-      const float hi = c_code_gemv[kBook][(idx >> 4) >> 4], lo = c_code_gemv[kBook][(idx >> 4) & 15];
+      const float hi = code_s[idx >> 8], lo = code_s[(idx >> 4) & 15];
       *reinterpret_cast<float4*>(pair_table + idx * 16) = make_float4(hi, lo, hi, lo);
     }
   }
@@ -263,10 +268,8 @@ cudaError_t launch_nt(const GemvGroup& grp, int64_t cols, const void* x, int bat
 
 template <int kBook>
 cudaError_t launch_book(const GemvGroup& grp, int64_t cols, const void* x, int batch, bool dq, cudaStream_t stream) {
-  if (batch <= 8) return launch_nt<1, kBook>(grp, cols, x, batch, dq, stream);
-  if (batch <= 16) return launch_nt<2, kBook>(grp, cols, x, batch, dq, stream);
-  if (batch <= 32) return launch_nt<4, kBook>(grp, cols, x, batch, dq, stream);
-  return launch_nt<8, kBook>(grp, cols, x, batch, dq, stream);
+  if (batch > 8) return cudaErrorInvalidValue;  // one n-tile of 8 activation rows
+  return launch_nt<1, kBook>(grp, cols, x, batch, dq, stream);
 }
 
 cudaError_t launch_group(const GemvGroup& grp, int64_t cols, const void* x, int batch, bool dq,
@@ -276,13 +279,11 @@ cudaError_t launch_group(const GemvGroup& grp, int64_t cols, const void* x, int 
 
 }  // namespace
 
-// batch <= 64: the activation rows are spread over ceil(batch / 8) n-tiles
+// batch <= 8: one n-tile of the mma holds every activation row
 cudaError_t launch_gemv(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x, int batch,
                         void* y, unsigned* err, cudaStream_t stream, int num_sms) {
-  if (batch <= 8) {
-    const GemvItem item = {packed, s, x, y, rows, cols};
-    return launch_gemv_items(&item, 1, batch, err, stream, num_sms);
-  }
+  (void)err;
+  (void)num_sms;
   if (rows / 16 > INT32_MAX) return cudaErrorInvalidValue;
   GemvGroup grp = {};
   grp.packed[0] = packed;
@@ -299,11 +300,8 @@ cudaError_t launch_gemv_group(const uint8_t* const* packed, const Scales* s, con
                               int64_t cols, const void* x, int batch, void* const* y, unsigned* err,
                               cudaStream_t stream, int num_sms) {
   if (count < 1 || count > kMaxGroup) return cudaErrorInvalidValue;
-  if (batch <= 8) {
-    GemvItem items[kMaxGroup];
-    for (int i = 0; i < count; ++i) items[i] = GemvItem{packed[i], s[i], x, y[i], rows[i], cols};
-    return launch_gemv_items(items, count, batch, err, stream, num_sms);
-  }
+  (void)err;
+  (void)num_sms;
   GemvGroup grp = {};
   int64_t tiles = 0;
   for (int i = 0; i < count; ++i) {

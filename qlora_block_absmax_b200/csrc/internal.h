@@ -42,8 +42,9 @@ struct Scales {
   int book;              // 4-bit code book: 0 = NF4, 1 = FP4 (E2M1 / 6)
 };
 
-cudaError_t launch_quantize(const void* src, bool bf16, int64_t n, uint8_t* packed, float* absmax, int book,
-                            cudaStream_t stream, int num_sms);
+// blocksize 32, 64, 128 or 256
+cudaError_t launch_quantize(const void* src, bool bf16, int64_t n, int blocksize, uint8_t* packed, float* absmax,
+                            int book, cudaStream_t stream, int num_sms);
 
 // workspace: zero before its first use, left ready by every completed call; `clear` zeroes it first
 cudaError_t launch_double_quant(const float* absmax, int64_t nb, int dq_code, uint8_t* q, float* scale,
@@ -51,10 +52,11 @@ cudaError_t launch_double_quant(const float* absmax, int64_t nb, int dq_code, ui
                                 int num_sms);
 constexpr size_t kDoubleQuantWorkspace = 256;
 
-cudaError_t launch_dequantize(const uint8_t* packed, const Scales& s, int64_t n, void* out, bool out_bf16,
-                              cudaStream_t stream, int num_sms);
+// blocksize 32, 64, 128 or 256
+cudaError_t launch_dequantize(const uint8_t* packed, const Scales& s, int64_t n, int blocksize, void* out,
+                              bool out_bf16, cudaStream_t stream, int num_sms);
 
-// batch <= 8 runs on the persistent stream kernel (gemv_stream.cu), 9..64 on the per-tile kernel (gemv.cu)
+// one CTA per 16-row tile (gemv.cu); batch up to 64
 cudaError_t launch_gemv(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x,
                         int batch, void* y, unsigned* err, cudaStream_t stream, int num_sms);
 

@@ -6,10 +6,11 @@
 //   Step 3  each scaled value takes the nearest NF4 code ("How NF4 works"),
 //   Step 4  two 4-bit codes share one byte; the scales are stored beside them.
 //
-// Layout: four lanes own one 64-element block, 16 consecutive elements each
-// (two 16-byte loads for bf16, four for fp32); a warp covers 8 consecutive
+// Layout: B/16 lanes own one block of B elements (B = 32, 64, 128 or 256; 64
+// is the pages' example and the default), 16 consecutive elements each (two
+// 16-byte loads for bf16, four for fp32); a warp covers 32/(B/16) consecutive
 // blocks per iteration and iterates uniformly (the lookup is a warp shuffle).
-// The block absmax is a 4-lane shuffle reduction.
+// The block absmax is a shuffle reduction over the block's lanes.
 //
 // Nearest code of x = RN(w / a): the number of thresholds (exact code
 // midpoints rounded down to fp32) below x.  A 32-bucket table covers [-1, 1];
@@ -126,17 +127,19 @@ __device__ __forceinline__ float load1(const void* src, int64_t i) {
   return static_cast<const float*>(src)[i];
 }
 
-template <bool kBF16, bool kFp4>
+template <bool kBF16, bool kFp4, int kL>
 __global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ src, int64_t n,
                                                        uint8_t* __restrict__ packed,
                                                        float* __restrict__ absmax) {
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const uint32_t entry = kFp4 ? c_q16[lane & 15] : c_q32[lane];
-  const int sub = lane & 3;                                  // which 16 of the block's 64
-  const unsigned gmask = 0xfu << (lane & ~3);                // the 4 lanes of this block
-  const int64_t nfull = n / kBlock;
-  const int64_t nblocks = (n + kBlock - 1) / kBlock;
+  // kL lanes own one block of kB = 16 kL elements, 16 consecutive elements each
+  constexpr int kB = 16 * kL;
+  constexpr int kPerWarp = 32 / kL;                          // blocks per warp and iteration
+  const int sub = lane & (kL - 1);                           // which 16 of the block
+  const int64_t nfull = n / kB;
+  const int64_t nblocks = (n + kB - 1) / kB;
   const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
   const int64_t warp_id = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
 
@@ -144,23 +147,23 @@ __global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ 
   // flight while this one is coded
   using Raw = uint4[kBF16 ? 2 : 4];
   auto fetch = [&](int64_t wb, Raw& raw) {
-    const int64_t b = wb + (lane >> 2);
+    const int64_t b = wb + lane / kL;
     if (b < nfull) {
       const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(src) +
-                                                      (b * kBlock + sub * 16) * (kBF16 ? 2 : 4));
+                                                      (b * kB + sub * 16) * (kBF16 ? 2 : 4));
 #pragma unroll
       for (int i = 0; i < (kBF16 ? 2 : 4); ++i) raw[i] = __ldcs(p + i);
     }
   };
   Raw cur, nxt;
-  int64_t wb = warp_id * 8;
+  int64_t wb = warp_id * kPerWarp;
   pdl_wait();
   if (wb < nblocks) fetch(wb, cur);
-  for (; wb < nblocks; wb += warps_total * 8) {  // uniform per warp
-    if (wb + warps_total * 8 < nblocks) fetch(wb + warps_total * 8, nxt);
-    const int64_t b = wb + (lane >> 2);
+  for (; wb < nblocks; wb += warps_total * kPerWarp) {  // uniform per warp
+    if (wb + warps_total * kPerWarp < nblocks) fetch(wb + warps_total * kPerWarp, nxt);
+    const int64_t b = wb + lane / kL;
     const bool live = b < nblocks;
-    const int64_t first = b * kBlock + sub * 16;
+    const int64_t first = b * kB + sub * 16;
     float w[16];
     if (live && b < nfull) {
       if (kBF16) {
@@ -188,8 +191,8 @@ __global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ 
     float a = 0.0f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(w[i]));
-    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
-    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+#pragma unroll
+    for (int off = 1; off < kL; off <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
 
     // Step 3: nearest code of RN(w / a); an all-zero block takes the zero code (7)
     const bool zero = !(a > 0.0f);
@@ -231,33 +234,47 @@ __global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ 
     }
     if (sub == 0) absmax[b] = a;
   }
-  (void)gmask;
+}
+
+template <bool kBF16, bool kFp4, int kL>
+cudaError_t launch_one(const void* src, int64_t n, uint8_t* packed, float* absmax, cudaStream_t stream, int num_sms) {
+  const int64_t nblocks = (n + 16 * kL - 1) / (16 * kL);
+  const int per_cta = 256 / kL;
+  int64_t grid = (nblocks + per_cta - 1) / per_cta;
+  int occ = 0;  // one wave: as many CTAs as fit on the SMs at once
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_kernel<kBF16, kFp4, kL>, 256, 0) != cudaSuccess ||
+      occ < 1)
+    occ = 1;
+  const int64_t cap = (int64_t)num_sms * occ;
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  const cudaError_t e =
+      launch_pdl(quantize_kernel<kBF16, kFp4, kL>, dim3((unsigned)grid), dim3(256), 0, stream, src, n, packed, absmax);
+  count_launches(1);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+template <bool kBF16, bool kFp4>
+cudaError_t launch_blocks(const void* src, int64_t n, int blocksize, uint8_t* packed, float* absmax,
+                          cudaStream_t stream, int num_sms) {
+  switch (blocksize) {
+    case 32: return launch_one<kBF16, kFp4, 2>(src, n, packed, absmax, stream, num_sms);
+    case 64: return launch_one<kBF16, kFp4, 4>(src, n, packed, absmax, stream, num_sms);
+    case 128: return launch_one<kBF16, kFp4, 8>(src, n, packed, absmax, stream, num_sms);
+    case 256: return launch_one<kBF16, kFp4, 16>(src, n, packed, absmax, stream, num_sms);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace
 
-cudaError_t launch_quantize(const void* src, bool bf16, int64_t n, uint8_t* packed, float* absmax, int book,
-                            cudaStream_t stream, int num_sms) {
-  const int64_t nblocks = (n + kBlock - 1) / kBlock;
-  const int per_cta = 256 / 4;
-  int64_t grid = (nblocks + per_cta - 1) / per_cta;
-  const void* fn = bf16 ? (book ? (const void*)quantize_kernel<true, true> : (const void*)quantize_kernel<true, false>)
-                        : (book ? (const void*)quantize_kernel<false, true> : (const void*)quantize_kernel<false, false>);
-  int occ = 0;  // one wave: as many CTAs as fit on the SMs at once
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, 256, 0) != cudaSuccess || occ < 1) occ = 1;
-  const int64_t cap = (int64_t)num_sms * occ;
-  if (grid > cap) grid = cap;
-  if (grid < 1) grid = 1;
-  const dim3 g((unsigned)grid), b(256);
-  cudaError_t e;
+cudaError_t launch_quantize(const void* src, bool bf16, int64_t n, int blocksize, uint8_t* packed, float* absmax,
+                            int book, cudaStream_t stream, int num_sms) {
   if (bf16)
-    e = book ? launch_pdl(quantize_kernel<true, true>, g, b, 0, stream, src, n, packed, absmax)
-             : launch_pdl(quantize_kernel<true, false>, g, b, 0, stream, src, n, packed, absmax);
-  else
-    e = book ? launch_pdl(quantize_kernel<false, true>, g, b, 0, stream, src, n, packed, absmax)
-             : launch_pdl(quantize_kernel<false, false>, g, b, 0, stream, src, n, packed, absmax);
-  count_launches(1);
-  return e != cudaSuccess ? e : cudaGetLastError();
+    return book ? launch_blocks<true, true>(src, n, blocksize, packed, absmax, stream, num_sms)
+                : launch_blocks<true, false>(src, n, blocksize, packed, absmax, stream, num_sms);
+  return book ? launch_blocks<false, true>(src, n, blocksize, packed, absmax, stream, num_sms)
+              : launch_blocks<false, false>(src, n, blocksize, packed, absmax, stream, num_sms);
 }
 
 }  // namespace nf4

@@ -27,7 +27,7 @@ int main(void) {
   /* quantize: bad sizes, block size, alignment -- all rejected on the host */
   CHECK(nf4_quantize((const void *)0x1000, NF4_F32, -1, 64, (uint8_t *)0x2000, (float *)0x3000, s) ==
         NF4_ERR_INVALID_ARG);
-  CHECK(nf4_quantize((const void *)0x1000, NF4_F32, 10, 128, (uint8_t *)0x2000, (float *)0x3000, s) ==
+  CHECK(nf4_quantize((const void *)0x1000, NF4_F32, 10, 512, (uint8_t *)0x2000, (float *)0x3000, s) ==
         NF4_ERR_UNSUPPORTED);
   CHECK(nf4_quantize((const void *)0x1004, NF4_F32, 10, 64, (uint8_t *)0x2000, (float *)0x3000, s) ==
         NF4_ERR_MISALIGNED);
@@ -67,8 +67,10 @@ int main(void) {
   w.quant_type = 7;
   CHECK(nf4_dequantize(&w, (void *)0x40000, NF4_BF16, s) == NF4_ERR_INVALID_ARG);
   w.quant_type = NF4_QUANT_NF4;
-  w.blocksize = 32;
+  w.blocksize = 48; /* level-1 sizes: 32, 64, 128, 256 */
   CHECK(nf4_dequantize(&w, (void *)0x40000, NF4_BF16, s) == NF4_ERR_UNSUPPORTED);
+  w.blocksize = 128; /* dequantize takes it; the matmuls take 64 only */
+  CHECK(nf4_gemv(&w, (const void *)0x30000, 1, (void *)0x40000, s) == NF4_ERR_UNSUPPORTED);
   if (failures) return 1;
   printf("ok\n");
   return 0;

@@ -64,7 +64,8 @@ def test_host_validation_before_cuda(lib):
     # quantize
     assert lib.nf4_quantize(0x1000, 0, -1, 64, 0x2000, 0x3000, s) == E["NF4_ERR_INVALID_ARG"]
     assert lib.nf4_quantize(0x1000, 7, 10, 64, 0x2000, 0x3000, s) == E["NF4_ERR_INVALID_ARG"]
-    assert lib.nf4_quantize(0x1000, 0, 10, 32, 0x2000, 0x3000, s) == E["NF4_ERR_UNSUPPORTED"]
+    for bs in (16, 48, 512):  # level-1 sizes are 32, 64, 128 and 256
+        assert lib.nf4_quantize(0x1000, 0, 10, bs, 0x2000, 0x3000, s) == E["NF4_ERR_UNSUPPORTED"]
     assert lib.nf4_quantize(0x1000, 0, 0, 64, 0x2000, 0x3000, s) == E["NF4_OK"]  # empty: nothing launched
     assert lib.nf4_quantize(None, 0, 10, 64, 0x2000, 0x3000, s) == E["NF4_ERR_INVALID_ARG"]
     assert lib.nf4_quantize(0x1008, 0, 10, 64, 0x2000, 0x3000, s) == E["NF4_ERR_MISALIGNED"]
@@ -80,7 +81,7 @@ def test_host_validation_before_cuda(lib):
         E["NF4_ERR_INVALID_ARG"]
     assert lib.nf4_double_quant_workspace_bytes(1 << 20) >= 128
     # weight descriptor checks
-    w = weight(bs=32)
+    w = weight(bs=48)
     assert lib.nf4_dequantize(ctypes.byref(w), 0x9000, 0, s) == E["NF4_ERR_UNSUPPORTED"]
     w = weight(packed=0x1001)
     assert lib.nf4_dequantize(ctypes.byref(w), 0x9000, 0, s) == E["NF4_ERR_MISALIGNED"]
