@@ -85,7 +85,7 @@ class QuantizedWeight:
 
 def quantize(w: torch.Tensor, blocksize: int = BLOCKSIZE, out=None, stream=None, quant_type: str = "nf4"):
     """Level-1 4-bit quantization (NF4, or FP4 with quant_type="fp4") of a flattened fp32/bf16 tensor.
-    Returns (packed uint8 [ceil(n/2)], absmax fp32 [ceil(n/64)])."""
+    Returns (packed uint8 [ceil(n/2)], absmax fp32 [ceil(n/blocksize)])."""
     _need_cuda(w, "w")
     if w.dtype not in (torch.float32, torch.bfloat16):
         raise TypeError("quantize takes float32 or bfloat16")

@@ -10,17 +10,21 @@
 // (one fp32 per tensor): mu = fp32(fp64(exact sum) / nb).
 //
 // Two kernels, chained with programmatic dependent launch (no grid barrier):
-//   sum     every fp32 value is an integer multiple of 2^-149, so each thread
-//           adds its values into ten signed 64-bit limbs holding 32 bits each
-//           of a 320-bit fixed-point number; integer addition makes the total
-//           exact and independent of order.  Warp shuffles and shared memory
-//           combine threads, 64-bit atomics combine CTAs.  The CTA that
+//   sum     every fp32 value is an integer multiple of 2^-149: a 56-bit chunk
+//           at one of ten 32-bit limbs of a 320-bit fixed-point number.  Each
+//           thread adds its chunks into two 64-bit registers (the limb of its
+//           first value and the next one; others go straight to shared
+//           memory), then hands 32-bit digits on; integer addition makes the
+//           total exact and independent of order.  Warp shuffles and shared
+//           memory combine threads, 64-bit atomics combine CTAs.  The CTA that
 //           arrives last (a counter in the workspace) normalises the limbs,
 //           rounds the sum once to fp64, writes mu and resets the limbs and
 //           the counter, so the workspace is ready for the next call (only the
 //           first call needs a zeroed buffer).
-//   encode  one warp per 256-value block: residuals, block absmax, codes; it
-//           reads mu after waiting for the sum kernel.
+//   encode  one warp per 256-value block: residuals, block absmax, codes.  It
+//           loads its absmax values while the sum kernel still runs (that
+//           kernel lets it start only once the array is complete) and waits
+//           for the sum kernel only before reading mu.
 #include "nf4_common.cuh"
 #include "internal.h"
 
@@ -35,20 +39,70 @@ struct SumWorkspace {
 };
 static_assert(sizeof(SumWorkspace) <= kDoubleQuantWorkspace, "workspace");
 
-__device__ __forceinline__ void add_value(long long (&acc)[kLimbs], float x) {
+// An fp32 value x is +-mant * 2^(sh - 149) with mant < 2^24 and 0 <= sh <= 253: the
+// 56-bit chunk mant << (sh mod 32) placed at limb sh / 32.
+struct Chunk {
+  long long v;  // signed chunk, |v| < 2^56
+  int li;       // limb of its lowest bit
+};
+__device__ __forceinline__ Chunk chunk_of(float x) {
   const uint32_t u = __float_as_uint(x);
   const uint32_t e = (u >> 23) & 0xffu, f = u & 0x7fffffu;
-  const uint32_t mant = e ? (f | 0x800000u) : f;  // value = mant * 2^(sh - 149)
+  const uint32_t mant = e ? (f | 0x800000u) : f;
   const int sh = e ? (int)e - 1 : 0;
-  const int li = sh >> 5;
-  const uint64_t v = (uint64_t)mant << (sh & 31);
-  long long lo = (long long)(v & 0xffffffffull), hi = (long long)(v >> 32);
-  if (u >> 31) {
-    lo = -lo;
-    hi = -hi;
+  const long long v = (long long)((uint64_t)mant << (sh & 31));
+  return Chunk{(u >> 31) ? -v : v, sh >> 5};
+}
+
+// Per-thread running sum: chunks at limb `base` and `base + 1` add into two 64-bit
+// registers (exact while fewer than 2^7 chunks have been added); any other limb, and
+// every 64 values, goes to the CTA's shared limbs as balanced 32-bit digits
+// (|digit| <= 2^31, so no limb total over 2^31 values leaves the signed 64-bit range).
+struct Runner {
+  int base = -1;
+  long long a0 = 0, a1 = 0;
+  int n = 0;
+};
+
+__device__ __forceinline__ void shared_add(long long* limbs, int li, long long v) {
+  atomicAdd(reinterpret_cast<unsigned long long*>(limbs + li), (unsigned long long)v);  // wraps: signed add
+}
+
+// the low 32 bits of v as a signed digit in [-2^31, 2^31): v - low(v) is a multiple of 2^32
+__device__ __forceinline__ long long low_digit(long long v) { return (long long)(int32_t)(uint32_t)v; }
+
+// digits of a0 (at base) and a1 (at base + 1): a = lo + 2^32 hi with balanced lo
+__device__ __forceinline__ void runner_digits(const Runner& r, long long& d0, long long& d1, long long& d2) {
+  const long long l0 = low_digit(r.a0), l1 = low_digit(r.a1);
+  d0 = l0;
+  d1 = ((r.a0 - l0) >> 32) + l1;
+  d2 = (r.a1 - l1) >> 32;
+}
+
+__device__ __forceinline__ void runner_flush(Runner& r, long long* limbs) {
+  if (r.base < 0) return;
+  long long d0, d1, d2;
+  runner_digits(r, d0, d1, d2);
+  if (d0) shared_add(limbs, r.base, d0);
+  if (d1) shared_add(limbs, r.base + 1, d1);
+  if (d2) shared_add(limbs, r.base + 2, d2);
+  r.a0 = r.a1 = 0;
+  r.n = 0;
+}
+
+__device__ __forceinline__ void runner_add(Runner& r, float x, long long* limbs) {
+  const Chunk c = chunk_of(x);
+  if (r.base < 0) r.base = c.li;
+  if (c.li == r.base) {
+    r.a0 += c.v;
+  } else if (c.li == r.base + 1) {
+    r.a1 += c.v;
+  } else {  // rare: a value more than 2^32 away in magnitude from this thread's first
+    const long long lo = low_digit(c.v);
+    shared_add(limbs, c.li, lo);
+    shared_add(limbs, c.li + 1, (c.v - lo) >> 32);
   }
-#pragma unroll
-  for (int L = 0; L < kLimbs; ++L) acc[L] += (L == li) ? lo : ((L == li + 1) ? hi : 0);
+  if (++r.n == 64) runner_flush(r, limbs);
 }
 
 // limb i of d (0 <= i < kLimbs), else 0; unrolled so d stays in registers
@@ -133,38 +187,48 @@ __device__ float finish_mean(const long long (&limb_in)[kLimbs], int64_t nb) {
 }
 
 // Exact sum of the absmax values; the last CTA derives mu, writes it and resets the workspace.
-__global__ void __launch_bounds__(256) dq_sum_kernel(const float* __restrict__ a, int64_t nb,
+__global__ void __launch_bounds__(512) dq_sum_kernel(const float* __restrict__ a, int64_t nb,
                                                      float* __restrict__ mean_out, SumWorkspace* __restrict__ ws) {
-  pdl_launch_dependents();  // the encode kernel may set itself up; it waits for this one to finish
+  __shared__ long long limbs[kLimbs];
+  __shared__ int s_last;
+  if (threadIdx.x < kLimbs) limbs[threadIdx.x] = 0;
+  __syncthreads();
   pdl_wait();
-  long long acc[kLimbs];
-#pragma unroll
-  for (int L = 0; L < kLimbs; ++L) acc[L] = 0;
+  // Signalled only now that the grid before this one (the producer of `a`) has finished: the encode kernel may
+  // then read `a` before its own wait, which only has to cover mu.
+  pdl_launch_dependents();
+  Runner r;
   const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t n4 = nb / 4;  // absmax is 16-byte aligned: float4 loads for the body
   for (int64_t i = tid; i < n4; i += nthreads) {
-    const float4 v = reinterpret_cast<const float4*>(a)[i];
-    add_value(acc, v.x);
-    add_value(acc, v.y);
-    add_value(acc, v.z);
-    add_value(acc, v.w);
+    const float4 v = __ldcs(reinterpret_cast<const float4*>(a) + i);
+    runner_add(r, v.x, limbs);
+    runner_add(r, v.y, limbs);
+    runner_add(r, v.z, limbs);
+    runner_add(r, v.w, limbs);
   }
-  for (int64_t i = 4 * n4 + tid; i < nb; i += nthreads) add_value(acc, a[i]);
+  for (int64_t i = 4 * n4 + tid; i < nb; i += nthreads) runner_add(r, a[i], limbs);
+  // combine the warp's runners: one set of digits when every lane has the same base (the usual case)
+  const int wbase = __reduce_max_sync(0xffffffffu, r.base);
+  if (r.base < 0) r.base = wbase;  // lanes without values hold zeros
+  if (__all_sync(0xffffffffu, r.base == wbase)) {
+    long long d[3];
+    runner_digits(r, d[0], d[1], d[2]);
 #pragma unroll
-  for (int L = 0; L < kLimbs; ++L)
+    for (int k = 0; k < 3; ++k)
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc[L] += __shfl_xor_sync(0xffffffffu, acc[L], off);
-  __shared__ long long red[8][kLimbs];
-  __shared__ int s_last;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (lane == 0)
+      for (int off = 16; off > 0; off >>= 1) d[k] += __shfl_xor_sync(0xffffffffu, d[k], off);
+    if ((threadIdx.x & 31) == 0 && wbase >= 0)
 #pragma unroll
-    for (int L = 0; L < kLimbs; ++L) red[warp][L] = acc[L];
+      for (int k = 0; k < 3; ++k)
+        if (d[k]) shared_add(limbs, wbase + k, d[k]);
+  } else {
+    runner_flush(r, limbs);
+  }
   __syncthreads();
   if (threadIdx.x < kLimbs) {
-    long long t = 0;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w][threadIdx.x];
+    const long long t = limbs[threadIdx.x];
     // values of similar magnitude touch two or three limbs: skip the zero ones (all limbs share one cache line)
     if (t != 0) atomicAdd(&ws->limb[threadIdx.x], (unsigned long long)t);  // wraps mod 2^64 = signed add
   }
@@ -182,29 +246,37 @@ __global__ void __launch_bounds__(256) dq_sum_kernel(const float* __restrict__ a
   }
 }
 
-// Codes: one warp per block of kDqBlock residuals.
+// Codes: one warp per block of kDqBlock residuals.  The sum kernel signals its dependents only after its own
+// wait, so by the time this grid starts the absmax array is complete: its values are loaded (at L2, not through
+// a possibly older L1 line) before the wait, which then covers only mu.
 __global__ void __launch_bounds__(256) dq_encode_kernel(const float* __restrict__ a, int64_t nb, int dq_code,
                                                         uint8_t* __restrict__ q, float* __restrict__ scale,
                                                         const float* __restrict__ mean) {
   pdl_launch_dependents();
-  pdl_wait();  // the sum kernel has finished: mu is in memory
-  const float mu = *mean;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t ngroups = (nb + kDqBlock - 1) / kDqBlock;
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
   const float Q = dq_code == 0 ? kE4M3Top : kInt8Top;
+  bool waited = false;
+  float mu = 0.0f;
   for (int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp; g < ngroups; g += nwarps) {
     const int64_t first = g * kDqBlock + lane * 8;
     const bool full = (g + 1) * kDqBlock <= nb;
     float r[8];
     if (full) {
       const float4* p = reinterpret_cast<const float4*>(a + first);
-      const float4 v0 = p[0], v1 = p[1];
+      const float4 v0 = __ldcg(p), v1 = __ldcg(p + 1);
       r[0] = v0.x; r[1] = v0.y; r[2] = v0.z; r[3] = v0.w;
       r[4] = v1.x; r[5] = v1.y; r[6] = v1.z; r[7] = v1.w;
-    } else {
+    }
+    if (!waited) {  // the sum kernel has finished: mu is in memory
+      pdl_wait();
+      mu = __ldcg(mean);
+      waited = true;
+    }
+    if (!full) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) r[i] = (first + i < nb) ? a[first + i] : mu;  // mu -> residual 0
+      for (int i = 0; i < 8; ++i) r[i] = (first + i < nb) ? __ldcg(a + first + i) : mu;  // mu -> residual 0
     }
     float m = 0.0f;
 #pragma unroll
@@ -240,6 +312,7 @@ __global__ void __launch_bounds__(256) dq_encode_kernel(const float* __restrict_
         if (first + i < nb) q[first + i] = (uint8_t)((i < 4 ? lo : hi) >> (8 * (i & 3)));
     }
   }
+  if (!waited) pdl_wait();  // a warp without a block still orders itself after the sum kernel
 }
 
 }  // namespace
@@ -250,10 +323,10 @@ cudaError_t launch_double_quant(const float* absmax, int64_t nb, int dq_code, ui
   cudaError_t e = cudaSuccess;
   if (clear && (e = cudaMemsetAsync(workspace, 0, sizeof(SumWorkspace), stream)) != cudaSuccess) return e;
   auto* ws = static_cast<SumWorkspace*>(workspace);
-  // sum: each thread at least 16 values (fewer CTAs, fewer atomics on the limbs), at most one CTA per SM
-  int64_t grid = (nb + 256 * 16 - 1) / (256 * 16);
+  // sum: one CTA of 512 threads per SM at most (one set of global limb atomics per CTA), at least 4 values a thread
+  int64_t grid = (nb + 512 * 4 - 1) / (512 * 4);
   grid = grid < 1 ? 1 : (grid > num_sms ? num_sms : grid);
-  e = launch_pdl(dq_sum_kernel, dim3((unsigned)grid), dim3(256), 0, stream, absmax, nb, mean, ws);
+  e = launch_pdl(dq_sum_kernel, dim3((unsigned)grid), dim3(512), 0, stream, absmax, nb, mean, ws);
   count_launches(1);
   if (e != cudaSuccess) return e;
   // encode: one warp per 256-value block, up to 8 CTAs of 8 warps per SM

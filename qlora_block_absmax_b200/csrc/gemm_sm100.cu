@@ -15,12 +15,14 @@
 // so the MMA reads only the activation tile from shared memory.  One
 // persistent CTA per SM walks the tiles; warp roles:
 //   warps 0-3   epilogue: tcgen05.ld -> bf16 -> Y (warp w reads TMEM lanes 32w..)
-//   warps 4-11  dequant producers, two groups of four taking alternate stages:
-//               thread p decodes weight row p of the stage (64 codes) with the
-//               byte-permute tables and stores it to its TMEM lane (tcgen05.st)
-//   warp 12     TMA producer: activation tile (256 x 64 bf16, 128B swizzle)
-//   warp 13     TMEM allocator and MMA issuer (one elected thread)
-//   warp 14     TMA producer: packed codes and 16-byte scale chunks
+//   warps 4..4+4G-1  dequant producers, G groups of four taking stages in
+//               turn: thread p decodes weight row p of the stage (64 codes)
+//               with the byte-permute tables and stores it to its TMEM lane
+//               (tcgen05.st); a decode is a long dependent chain per thread,
+//               so the groups in flight are what keep the issue slots busy
+//   next warp   TMA producer: activation tile (256 x 64 bf16, 128B swizzle)
+//   next warp   TMEM allocator and MMA issuer (one elected thread)
+//   last warp   TMA producer: packed codes and 16-byte scale chunks
 // With a low-rank adapter (QLoRA: "bitsandbytes quantization tutorial",
 // "QLoRA: Fine-Tuning a 4-bit Model") each output tile runs one more stage:
 // the producers put [B | B] rows of the up map in the TMEM slot, the TMA warp
@@ -46,18 +48,22 @@ using namespace umma;
 
 constexpr int kTileK = 64;        // k per stage (128 bytes of bf16: one swizzle atom)
 constexpr int kXStages = 5;  // activation-tile ring (TMA from L2/HBM)
-constexpr int kAStages = 3;  // decoded weight-tile ring in TMEM (written by the producer warps)
+// producer groups of four warps, one stage each in turn (3 or 4 groups -- more warps with fewer registers each --
+// measured 3 to 25 % slower at every shape)
+constexpr int kGroups = 2;
+constexpr int kAStages = 2 * kGroups;     // decoded weight-tile ring in TMEM (written by the producer warps)
 constexpr int kWStages = 6;  // packed-code + scale ring (TMA from HBM), deeper to hide its latency
 constexpr int kBBytes = kTileM * kTileK * 2;  // 32 KB: activation tile (operand B)
 constexpr int kWBytes = kTileN * kTileK / 2;  // 4 KB: packed codes of the weight tile
 constexpr int kSBytes = kTileN * 16;          // 2 KB: 16-byte scale chunk per weight row
 constexpr int kRingBytes = kXStages * kBBytes + kWStages * (kWBytes + kSBytes);  // A lives in TMEM
-constexpr int kTmemCols = 512;               // accumulator (256 columns) + 3 A stages of 32 columns
-constexpr int kThreads = 15 * 32;
-constexpr int kProdWarp0 = 4;                 // producers: warps 4..11
-constexpr int kTmaWarp = 12;                  // activation tiles
-constexpr int kMmaWarp = 13;
-constexpr int kTmaWWarp = 14;                 // packed codes and scales
+constexpr int kTmemCols = 512;               // accumulator (256 columns) + the A ring of 32-column stages
+constexpr int kProdWarp0 = 4;                 // producers: warps 4 .. 4 + 4 kGroups - 1
+constexpr int kTmaWarp = kProdWarp0 + 4 * kGroups;  // activation tiles
+constexpr int kMmaWarp = kTmaWarp + 1;
+constexpr int kTmaWWarp = kTmaWarp + 2;             // packed codes and scales
+constexpr int kThreads = (kTmaWWarp + 1) * 32;
+static_assert(kAccCols + kAStages * 32 <= 512, "TMEM: accumulator + A ring");
 constexpr size_t kSmemBytes = (size_t)kRingBytes + kEpiWarps * kStageOutBytes + 1024 /*align*/ +
                               2048 /*barriers, lut*/;
 
@@ -150,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp >= kProdWarp0 && warp < kTmaWarp) {
     // ------------------------------------------------ dequant producers
-    const int group = (warp - kProdWarp0) >> 2;          // 0 or 1: alternate stages
+    const int group = (warp - kProdWarp0) >> 2;          // 0 .. kGroups - 1: stages in turn
     const int p = ((warp - kProdWarp0) & 3) * 32 + lane;  // weight row within the tile
     const float mu = kDQ ? *s.mean : 0.0f;
     const int64_t rb = cols / kBlock;
@@ -163,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int ks = ks0; ks < ks1; ++ks, ++it) {
         const bool adapter = ks == ks0 + wk.kps;
         if (!adapter) ++wit;
-        if ((int)(it & 1) != group) continue;
+        if ((int)(it % kGroups) != group) continue;
         const int as = it % kAStages;
         const uint32_t aph = (it / kAStages) & 1;
         if (adapter) {

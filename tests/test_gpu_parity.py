@@ -145,6 +145,9 @@ def dq_cases():
         "wide": (np.abs(r.standard_normal(3000)) * np.exp(r.uniform(-80, 80, 3000))).astype(np.float32),
         "signed": r.standard_normal(1000).astype(np.float32),
         "zeros_and_tiny": np.concatenate([np.zeros(300, np.float32), np.full(212, 1e-40, np.float32)]),
+        # more than 64 values per thread of the sum kernel, magnitudes spread over ~90 binades, some negative
+        "big_mixed": (np.abs(r.standard_normal(6_000_001)) * np.exp(r.uniform(-30, 30, 6_000_001))
+                      * np.where(r.uniform(0, 1, 6_000_001) < 0.05, -1, 1)).astype(np.float32),
     }
 
 
