@@ -57,6 +57,7 @@ constexpr int kBBytes = kTileM * kTileK * 2;  // 32 KB: activation tile (operand
 constexpr int kWBytes = kTileN * kTileK / 2;  // 4 KB: packed codes of the weight tile
 constexpr int kSBytes = kTileN * 16;          // 2 KB: 16-byte scale chunk per weight row
 constexpr int kRingBytes = kXStages * kBBytes + kWStages * (kWBytes + kSBytes);  // A lives in TMEM
+static_assert(kXStages * kBBytes >= kSplitStageBytes, "split reduction staging fits in the operand ring");
 constexpr int kTmemCols = 512;               // accumulator (256 columns) + the A ring of 32-column stages
 constexpr int kProdWarp0 = 4;                 // producers: warps 4 .. 4 + 4 kGroups - 1
 constexpr int kTmaWarp = kProdWarp0 + 4 * kGroups;  // activation tiles
@@ -326,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       if (threadIdx.x == 0) NF4_STAMP(4);
       const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + acc * kAccCols;
-      epilogue_unit(wk, u, taddr, out_stage, sm, &sm->acc_empty[acc], o);
+      epilogue_unit(wk, u, taddr, out_stage, sm, &sm->acc_empty[acc], o, gbase);
       if (threadIdx.x == 0) NF4_STAMP(6);
     }
   }

@@ -172,9 +172,22 @@ struct EpiOut {
 // One work unit's accumulator (TMEM lanes = output columns n0 .. n0+127,
 // columns = activation rows m0 .. m0+255) -> Y, run by warps 0..3.  Releases
 // the accumulator through `acc_empty` as soon as it has been read.
+// Shared memory the split reduction stages the other splits' partials in: 16 bytes per piece and epilogue
+// thread; pieces = own 32-row chunks (ceil(8 / splits)) x 2 halves x (splits - 1) other partials x 4, at most
+// 48 (32 with two splits, 48 with three or four): 96 KB with 128 epilogue threads.
+static_assert(kMaxSplits <= 4, "split staging size");
+constexpr int kSplitStagePieces = 48;
+constexpr int kSplitStageBytes = kSplitStagePieces * kEpiWarps * 32 * 16;
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+// `stage_in`: kSplitStageBytes of shared memory that is idle once the unit's MMAs have finished (the operand
+// ring; with splits > 1 a CTA has a single unit, so nothing refills it)
 template <class Sm>
 __device__ __forceinline__ void epilogue_unit(const Work& wk, int u, uint32_t taddr, uint16_t* out_stage, Sm* sm,
-                                              uint64_t* acc_empty, const EpiOut& o) {
+                                              uint64_t* acc_empty, const EpiOut& o, uint8_t* stage_in) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nl = warp * 32 + lane;  // output column within the tile
   const int64_t n = (int64_t)wk.n0(u) + nl;
@@ -228,6 +241,7 @@ __device__ __forceinline__ void epilogue_unit(const Work& wk, int u, uint32_t ta
   epi_bar();
   // every split of the tile waits for all partials (the splits of a tile are co-resident: the
   // grid holds every unit at once), then finishes its share of the 32-row chunks
+  unsigned second = 0;  // (thread 0) this split's second arrival, read only after the reduction
   if (threadIdx.x == 0) {
     atomicAdd(&o.tile_count[wk.tile(u)], 1u);
     const unsigned long long t0 = global_ns();
@@ -240,29 +254,48 @@ __device__ __forceinline__ void epilogue_unit(const Work& wk, int u, uint32_t ta
       __nanosleep(64);
     }
     // second arrival: the split that completes 2 * splits has seen every split pass the wait
-    // above, so it can reset the counter for the next call
-    if (!aborted(sm) && atomicAdd(&o.tile_count[wk.tile(u)], 1u) == 2u * (unsigned)wk.splits - 1u)
-      o.tile_count[wk.tile(u)] = 0;
+    // above, so it can reset the counter for the next call (at the end, off the critical path)
+    if (!aborted(sm)) second = atomicAdd(&o.tile_count[wk.tile(u)], 1u) + 1u;
   }
   epi_bar();
   if (!aborted(sm)) {
     __threadfence();
     const float* tp = o.part + (size_t)wk.tile(u) * wk.splits * (kTileN * kTileM);
+    // Every other split's partial of this split's chunks, copied into shared memory with all copies in flight
+    // at once (one round of L2 latency), piece p of this thread at stage_in + (p * 128 + nl) * 16.
+    const uint32_t stage = smem_u32(stage_in);
+    fence_proxy_async_smem();  // the ring was last written by TMA and read by the MMAs
+    int pc = 0;
+#pragma unroll 1
+    for (int c = my; c < kTileM / 32; c += wk.splits)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < kMaxSplits - 1; ++q) {
+          const int sp = q + (q >= my);
+          if (sp < wk.splits) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j, ++pc)
+              cp_async16(stage + (uint32_t)(pc * (kEpiWarps * 32) + nl) * 16u,
+                         tp + (size_t)sp * (kTileN * kTileM) + ((size_t)(c * 8 + h * 4 + j) * kTileN + nl) * 4);
+          }
+        }
+    asm volatile("cp.async.commit_group;\n cp.async.wait_group 0;" ::: "memory");
+    const float4* staged = reinterpret_cast<const float4*>(stage_in);
+    pc = 0;
 #pragma unroll 1
     for (int c = my; c < kTileM / 32; c += wk.splits) {
       uint32_t v[32];
       tmem_ld32(taddr + c * 32, v);  // this split's own partial of the chunk
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {  // 16 rows at a time: every other split's loads in flight together
+      for (int h = 0; h < 2; ++h) {  // 16 rows at a time
         float4 t[kMaxSplits - 1][4];
 #pragma unroll
         for (int q = 0; q < kMaxSplits - 1; ++q) {
           const int sp = q + (q >= my);
           if (sp < wk.splits) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              t[q][j] = __ldcg(reinterpret_cast<const float4*>(
-                  tp + (size_t)sp * (kTileN * kTileM) + ((size_t)(c * 8 + h * 4 + j) * kTileN + nl) * 4));
+            for (int j = 0; j < 4; ++j, ++pc) t[q][j] = staged[pc * (kEpiWarps * 32) + nl];
           }
         }
 #pragma unroll
@@ -303,6 +336,7 @@ __device__ __forceinline__ void epilogue_unit(const Work& wk, int u, uint32_t ta
       store_block(c);
     }
   }
+  if (threadIdx.x == 0 && second == 2u * (unsigned)wk.splits) o.tile_count[wk.tile(u)] = 0;
   tc_fence_before();
   __syncwarp();
   if (lane == 0) mbar_arrive(acc_empty);  // TMEM no longer needed

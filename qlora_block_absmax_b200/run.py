@@ -2,10 +2,11 @@
 
     python -m qlora_block_absmax_b200.run OP [--rows R] [--cols C] [--batch B] [--m M] [--iters N] [--fp4]
 
-OP: quantize | double_quant | dequantize | gemv | gemv_stream | gemm | gemm_dx | gemm_lora
+OP: quantize | double_quant | dequantize | gemv | gemv_grouped | gemv_stream | gemm | gemm_dx | gemm_lora
 Weights: bf16 ~N(0, 0.02) from the device generator (seed 1010), NF4 (or FP4 with --fp4) with E4M3 double quant;
 activations bf16 ~N(0, 1) (seed 1013).  gemv_stream runs one decoder layer of the 8B shape (7 weights) in one
-launch.  Useful to look at one kernel in isolation (for instance under a profiler); prints one line per call
+launch; gemv_grouped runs q, k, v of that layer (4096, 1024, 1024 x 4096) on one x in one launch.  Useful to look
+at one kernel in isolation (for instance under a profiler); prints one line per call
 with the device time of the last iteration.
 """
 from __future__ import annotations
@@ -20,8 +21,8 @@ from qlora_block_absmax_b200 import synth
 
 def main() -> None:
     ap = argparse.ArgumentParser()
-    ap.add_argument("op", choices=["quantize", "double_quant", "dequantize", "gemv", "gemv_stream", "gemm", "gemm_dx",
-                                   "gemm_lora"])
+    ap.add_argument("op", choices=["quantize", "double_quant", "dequantize", "gemv", "gemv_grouped", "gemv_stream",
+                                   "gemm", "gemm_dx", "gemm_lora"])
     ap.add_argument("--rows", type=int, default=4096)
     ap.add_argument("--cols", type=int, default=4096)
     ap.add_argument("--batch", type=int, default=1)
@@ -48,6 +49,11 @@ def main() -> None:
     elif a.op == "gemv":
         x = synth.activations_device((a.batch, a.cols), 1013, device=dev)
         call = lambda: nf4.gemv(qw, x)  # noqa: E731
+    elif a.op == "gemv_grouped":
+        x = synth.activations_device((a.batch, 4096), 1013, device=dev)
+        qkv = [nf4.quantize_weight(synth.normal_weights_device((r, 4096), synth.layer_seed(0, p), device=dev),
+                                   quant_type=qt) for p, (_, r, _) in enumerate(synth.LLAMA8B_LAYER[:3])]
+        call = lambda: nf4.gemv_grouped(qkv, x)  # noqa: E731
     elif a.op == "gemv_stream":
         ws, xs = [], []
         acts = [synth.activations_device((a.batch, c), 3300 + j, device=dev) for j, c in enumerate((4096, 14336))]
