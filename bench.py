@@ -628,6 +628,7 @@ def run_ours(args):
             d["frac_bf16"] = round(work[k]["flops"] / t / 1e12 / peaks["bf16_tflops"], 4)
         if "elems" in work[k]:
             d["gelem_s"] = round(work[k]["elems"] / t / 1e9, 2)
+        d["traffic"] = TRAFFIC.get(k)  # ncu DRAM bytes per launch (cold), or None
         breakdown[k] = d
     nexts = {}
     for k in NEXT_KERNELS:
@@ -732,9 +733,12 @@ def model_config(args, nf4, synth, dev, time_calls, peaks):
     return out
 
 
-# ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of each kernel at this workload, from the captures
-# summarised in profiles/; an entry is removed whenever its kernel changes after the capture
-TRAFFIC = {"quantize": 33576192, "double_quant": 1084928, "dequantize": 8679680}
+# ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of each kernel at this workload (double quant: its two
+# kernels; gemm_lora: the down map and the GEMM), from the captures summarised in profiles/ (ncu flushes the caches
+# before each replayed launch, so these are cold-read figures); an entry is removed whenever its kernel changes
+# after the capture
+TRAFFIC = {"quantize": 33573632, "double_quant": 2137088, "dequantize": 8678400, "gemv": 8681984, "gemm": 10825728,
+           "gemm_dx": 10822144, "gemm_lora": 13229824, "gemv_grouped": 13009664}
 
 
 def oracle_table(args):

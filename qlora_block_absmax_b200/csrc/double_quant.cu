@@ -190,7 +190,6 @@ __device__ float finish_mean(const long long (&limb_in)[kLimbs], int64_t nb) {
 __global__ void __launch_bounds__(512) dq_sum_kernel(const float* __restrict__ a, int64_t nb,
                                                      float* __restrict__ mean_out, SumWorkspace* __restrict__ ws) {
   __shared__ long long limbs[kLimbs];
-  __shared__ int s_last;
   if (threadIdx.x < kLimbs) limbs[threadIdx.x] = 0;
   __syncthreads();
   pdl_wait();
@@ -227,22 +226,22 @@ __global__ void __launch_bounds__(512) dq_sum_kernel(const float* __restrict__ a
     runner_flush(r, limbs);
   }
   __syncthreads();
-  if (threadIdx.x < kLimbs) {
-    const long long t = limbs[threadIdx.x];
-    // values of similar magnitude touch two or three limbs: skip the zero ones (all limbs share one cache line)
-    if (t != 0) atomicAdd(&ws->limb[threadIdx.x], (unsigned long long)t);  // wraps mod 2^64 = signed add
-  }
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) s_last = atomicAdd(&ws->count, 1u) == gridDim.x - 1;
-  __syncthreads();
-  if (s_last && threadIdx.x == 0) {  // every other CTA has added its share
-    __threadfence();
-    long long l[kLimbs];
+  if (threadIdx.x < 32) {  // warp 0 alone hands the CTA's limbs on and counts the CTA in
+    if (threadIdx.x < kLimbs) {
+      const long long t = limbs[threadIdx.x];
+      // values of similar magnitude touch two or three limbs: skip the zero ones (all limbs share one cache line)
+      if (t != 0) atomicAdd(&ws->limb[threadIdx.x], (unsigned long long)t);  // wraps mod 2^64 = signed add
+      __threadfence();  // the limb additions before the count below
+    }
+    __syncwarp();
+    if (threadIdx.x == 0 && atomicAdd(&ws->count, 1u) == gridDim.x - 1) {  // every other CTA has added its share
+      __threadfence();
+      long long l[kLimbs];
 #pragma unroll
-    for (int L = 0; L < kLimbs; ++L) l[L] = (long long)atomicExch(&ws->limb[L], 0ull);  // read and reset
-    *mean_out = finish_mean(l, nb);
-    ws->count = 0;
+      for (int L = 0; L < kLimbs; ++L) l[L] = (long long)atomicExch(&ws->limb[L], 0ull);  // read and reset
+      *mean_out = finish_mean(l, nb);
+      ws->count = 0;
+    }
   }
 }
 
