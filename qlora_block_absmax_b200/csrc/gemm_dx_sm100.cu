@@ -50,7 +50,7 @@ constexpr int kWHalf = kTileR * 32;            // 2 KB: one level-1 block of cod
 constexpr int kWBytes = 2 * kWHalf;            // 4 KB: the stage's two blocks per row
 constexpr int kSBytes = kTileR * 16;           // 1 KB: 16-byte scale chunk per row
 constexpr int kRingBytes = kXStages * kBBytes + kAStages * kABytes + kWStages * (kWBytes + kSBytes);
-static_assert(kXStages * kBBytes >= kSplitStageBytes, "split reduction staging fits in the operand ring");
+static_assert(kXStages * kBBytes >= split_stage_bytes(kTileM), "split reduction staging fits in the operand ring");
 constexpr int kTmemCols = 2 * kAccCols;        // two accumulators
 constexpr int kThreads = 15 * 32;
 constexpr int kProdWarp0 = 4;
@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   Work wk;
   wk.ntiles_m = (m_total + kTileM - 1) / kTileM;
+  wk.tm = kTileM;
   wk.splits = splits;
   wk.units = (cols / kTileN) * wk.ntiles_m * splits;
   wk.kps = rows / kTileR / splits;
@@ -286,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!wait_or_abort(&sm->acc_full[acc], (ucount >> 1) & 1, sm, err)) break;
       tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + acc * kAccCols;
-      epilogue_unit(wk, u, taddr, out_stage, sm, &sm->acc_empty[acc], o, gbase);
+      epilogue_unit<kTileM>(wk, u, taddr, out_stage, sm, &sm->acc_empty[acc], o, gbase);
     }
   }
 

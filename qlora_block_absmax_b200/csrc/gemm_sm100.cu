@@ -47,32 +47,40 @@ namespace {
 using namespace umma;
 
 constexpr int kTileK = 64;        // k per stage (128 bytes of bf16: one swizzle atom)
-constexpr int kXStages = 5;  // activation-tile ring (TMA from L2/HBM)
 // producer groups of four warps, one stage each in turn (3 or 4 groups -- more warps with fewer registers each --
 // measured 3 to 25 % slower at every shape)
 constexpr int kGroups = 2;
 constexpr int kAStages = 2 * kGroups;     // decoded weight-tile ring in TMEM (written by the producer warps)
 constexpr int kWStages = 6;  // packed-code + scale ring (TMA from HBM), deeper to hide its latency
-constexpr int kBBytes = kTileM * kTileK * 2;  // 32 KB: activation tile (operand B)
 constexpr int kWBytes = kTileN * kTileK / 2;  // 4 KB: packed codes of the weight tile
 constexpr int kSBytes = kTileN * 16;          // 2 KB: 16-byte scale chunk per weight row
-constexpr int kRingBytes = kXStages * kBBytes + kWStages * (kWBytes + kSBytes);  // A lives in TMEM
-static_assert(kXStages * kBBytes >= kSplitStageBytes, "split reduction staging fits in the operand ring");
-constexpr int kTmemCols = 512;               // accumulator (256 columns) + the A ring of 32-column stages
 constexpr int kProdWarp0 = 4;                 // producers: warps 4 .. 4 + 4 kGroups - 1
 constexpr int kTmaWarp = kProdWarp0 + 4 * kGroups;  // activation tiles
 constexpr int kMmaWarp = kTmaWarp + 1;
 constexpr int kTmaWWarp = kTmaWarp + 2;             // packed codes and scales
 constexpr int kThreads = (kTmaWWarp + 1) * 32;
-static_assert(kAccCols + kAStages * 32 <= 512, "TMEM: accumulator + A ring");
-constexpr size_t kSmemBytes = (size_t)kRingBytes + kEpiWarps * kStageOutBytes + 1024 /*align*/ +
-                              2048 /*barriers, lut*/;
+constexpr int kXStagesMax = 8;
+
+// Per activation-tile width TM (the UMMA N: 256, or 64 for up to 64 activation rows, where a 256-wide tile would
+// spend three quarters of every MMA on padding rows): the activation ring and the TMEM budget.
+template <int TM>
+struct TileCfg {
+  static constexpr int kXStages = TM == 256 ? 5 : 8;  // activation-tile ring (TMA from L2/HBM)
+  static constexpr int kBBytes = TM * kTileK * 2;     // activation tile (operand B): 32 KB at TM = 256
+  static constexpr int kRingBytes = kXStages * kBBytes + kWStages * (kWBytes + kSBytes);  // A lives in TMEM
+  static constexpr int kTmemCols = TM + kAStages * 32 <= 256 ? 256 : 512;  // accumulator + A ring, a power of 2
+  static constexpr size_t kSmemBytes = (size_t)kRingBytes + kEpiWarps * kStageOutBytes + 1024 /*align*/ +
+                                       2048 /*barriers, lut*/;
+  static_assert(kXStages * kBBytes >= split_stage_bytes(TM), "split reduction staging fits in the operand ring");
+  static_assert(TM + kAStages * 32 <= kTmemCols, "TMEM: accumulator + A ring");
+  static_assert(kXStages <= kXStagesMax, "barrier array");
+};
 
 struct Smem {  // placed after the 1024-aligned stage buffers
   uint64_t wfull[kWStages];   // packed codes + scale chunk landed (TMA)
   uint64_t wempty[kWStages];  // codes read by the producer warps
-  uint64_t xfull[kXStages];   // activation tile landed (TMA)
-  uint64_t xempty[kXStages];  // activation tile consumed by the MMAs (tcgen05.commit)
+  uint64_t xfull[kXStagesMax];   // activation tile landed (TMA)
+  uint64_t xempty[kXStagesMax];  // activation tile consumed by the MMAs (tcgen05.commit)
   uint64_t afull[kAStages];   // decoded weight tile written (producer warps)
   uint64_t aempty[kAStages];  // decoded tile consumed by the MMAs (tcgen05.commit)
   uint64_t acc_full[2];
@@ -91,13 +99,17 @@ __device__ unsigned long long g_trace[1024 * 16];
 #define NF4_STAMP(slot) ((void)0)
 #endif
 
-template <bool kDQ, bool kScaleTma, int kBook>
+template <bool kDQ, bool kScaleTma, int kBook, int TM>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(Scales s, int rows, int cols, int m_total, int splits, const __grid_constant__ CUtensorMap xmap,
                 const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
                 __nv_bfloat16* __restrict__ y, float* __restrict__ part, unsigned* __restrict__ tile_count,
                 unsigned* err, const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __restrict__ lora_up,
                 int lora_r) {
+  using Cfg = TileCfg<TM>;
+  constexpr int kXStages = Cfg::kXStages, kBBytes = Cfg::kBBytes, kRingBytes = Cfg::kRingBytes;
+  constexpr int kTmemCols = Cfg::kTmemCols;
+  constexpr int kAccColsT = TM;  // accumulator columns; the A ring follows
   extern __shared__ uint8_t smem_raw[];
   pdl_launch_dependents();
   const uint32_t raw = smem_u32(smem_raw);
@@ -112,7 +124,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   Work wk;
-  wk.ntiles_m = (m_total + kTileM - 1) / kTileM;
+  wk.ntiles_m = (m_total + TM - 1) / TM;
+  wk.tm = TM;
   wk.splits = splits;
   wk.units = (rows / kTileN) * wk.ntiles_m * splits;
   wk.kps = cols / kTileK / splits;
@@ -189,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             r[j + 3] = v.w;
           }
           if (!wait_or_abort(&sm->aempty[as], aph ^ 1, sm, err)) break;
-          const uint32_t ta = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(kAccCols + as * 32);
+          const uint32_t ta = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(kAccColsT + as * 32);
           tmem_st32(ta, r);
           tc_fence_before();
           __syncwarp();
@@ -227,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           r[4 * c + 3] = d[3];
         }
         if (!wait_or_abort(&sm->aempty[as], aph ^ 1, sm, err)) break;  // the MMAs left this slot
-        tmem_st32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(kAccCols + as * 32), r);
+        tmem_st32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(kAccColsT + as * 32), r);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm->afull[as]);
@@ -286,13 +299,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = instr_desc(kTileN, kTileM);
+      constexpr uint32_t idesc = instr_desc(kTileN, TM);
       uint32_t it = 0, ucount = 0;
       for (int u = blockIdx.x; u < wk.units && !aborted(sm); u += gridDim.x, ++ucount) {
         const int acc = 0;  // one accumulator: the A ring takes the other TMEM columns
         if (!wait_or_abort(&sm->acc_empty[acc], (ucount & 1) ^ 1, sm, err)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem + acc * kAccCols;
+        const uint32_t d_tmem = tmem + acc * kAccColsT;
         bool ok = true;
         const int nst = wk.kps + (lora_r > 0 && wk.split(u) == 0 ? 1 : 0);  // + the adapter stage
         for (int j = 0; j < nst; ++j, ++it) {
@@ -304,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           if (it == 0) NF4_STAMP(2);
-          const uint32_t a_tm = tmem + (uint32_t)(kAccCols + as * 32), b_addr = b_smem0 + xs * kBBytes;
+          const uint32_t a_tm = tmem + (uint32_t)(kAccColsT + as * 32), b_addr = b_smem0 + xs * kBBytes;
           const int nkk = j < wk.kps ? kTileK / 16 : lora_r / 8;  // the adapter stage reduces over 2r only
 #pragma unroll
           for (int kk = 0; kk < kTileK / 16; ++kk)  // 16 bf16 per MMA along k: 8 TMEM columns, 32 smem bytes
@@ -326,8 +339,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!wait_or_abort(&sm->acc_full[acc], ucount & 1, sm, err)) break;
       tc_fence_after();
       if (threadIdx.x == 0) NF4_STAMP(4);
-      const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + acc * kAccCols;
-      epilogue_unit(wk, u, taddr, out_stage, sm, &sm->acc_empty[acc], o, gbase);
+      const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + acc * kAccColsT;
+      epilogue_unit<TM>(wk, u, taddr, out_stage, sm, &sm->acc_empty[acc], o, gbase);
       if (threadIdx.x == 0) NF4_STAMP(6);
     }
   }
@@ -359,9 +372,17 @@ EncodeTiled get_encoder() {
   return fn;
 }
 
+// activation rows per tile: 64 while they cover m (the MMA's N then carries no padding rows beyond 64), else 256
+int gemm_tile_m(int64_t m) { return m <= 64 ? 64 : 256; }
+
+int64_t gemm_tiles(int64_t rows, int64_t m) {
+  const int tm = gemm_tile_m(m);
+  return (rows / kTileN) * ((m + tm - 1) / tm);
+}
+
 int gemm_splits(int64_t rows, int64_t cols, int64_t m, int num_sms) {
   if (m <= 8) return 1;  // served by the GEMV
-  return reduction_splits((rows / kTileN) * ((m + kTileM - 1) / kTileM), cols / kTileK, num_sms);
+  return reduction_splits(gemm_tiles(rows, m), cols / kTileK, num_sms);
 }
 
 }  // namespace
@@ -387,10 +408,10 @@ int reduction_splits(int64_t ntiles, int64_t stages, int num_sms) {
   return best;
 }
 
-size_t split_workspace_bytes(int64_t ntiles, int splits) {
+size_t split_workspace_bytes(int64_t ntiles, int splits, int tm) {
   if (splits == 1) return 0;
   const size_t counters = ((size_t)ntiles * 4 + 255) & ~(size_t)255;
-  return counters + (size_t)ntiles * splits * kTileN * kTileM * sizeof(float);
+  return counters + (size_t)ntiles * splits * kTileN * tm * sizeof(float);
 }
 
 int sm_count() {
@@ -403,32 +424,48 @@ int sm_count() {
 
 size_t gemm_workspace_bytes(int64_t rows, int64_t cols, int64_t m) {
   const int sp = gemm_splits(rows, cols, m, sm_count());
-  return split_workspace_bytes((rows / kTileN) * ((m + kTileM - 1) / kTileM), sp);
+  return split_workspace_bytes(gemm_tiles(rows, m), sp, gemm_tile_m(m));
 }
 
 namespace {
 
-template <bool kDQ, bool kScaleTma, int kBook>
+template <bool kDQ, bool kScaleTma, int kBook, int TM>
 cudaError_t launch_variant(const Scales& s, int rows, int cols, int m, int splits, const CUtensorMap& xmap,
                            const CUtensorMap& wmap, const CUtensorMap& smap, __nv_bfloat16* y, float* part,
                            unsigned* counters, unsigned* err, int grid, cudaStream_t stream, const CUtensorMap& tmap,
                            const __nv_bfloat16* lora_up, int lora_r) {
+  constexpr size_t smem = TileCfg<TM>::kSmemBytes;
   // the shared-memory opt-in is a per-device function attribute: set it once
   // per device (outside any stream capture that later calls may be part of)
   static std::atomic<uint64_t> attr_done{0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!(attr_done.load() & (1ull << dev))) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<kDQ, kScaleTma, kBook>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<kDQ, kScaleTma, kBook, TM>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr_done.fetch_or(1ull << dev);
   }
-  const cudaError_t e = launch_pdl(gemm_kernel<kDQ, kScaleTma, kBook>, dim3(grid), dim3(kThreads), kSmemBytes, stream, s,
+  const cudaError_t e = launch_pdl(gemm_kernel<kDQ, kScaleTma, kBook, TM>, dim3(grid), dim3(kThreads), smem, stream, s,
                                    rows, cols, m, splits, xmap, wmap, smap, y, part, counters, err, tmap, lora_up,
                                    lora_r);
   count_launches(1);
   return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+template <int TM>
+cudaError_t launch_book_scales(bool dq, bool scale_tma, int book, const Scales& s, int R, int C, int M, int splits,
+                               const CUtensorMap& xmap, const CUtensorMap& wmap, const CUtensorMap& smap,
+                               __nv_bfloat16* yb, float* part, unsigned* counters, unsigned* err, int grid,
+                               cudaStream_t stream, const CUtensorMap& tmap, const __nv_bfloat16* up, int lora_r) {
+#define NF4_GEMM_VARIANT(DQ, ST, BK)                                                                                 \
+  launch_variant<DQ, ST, BK, TM>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream, tmap, \
+                                 up, lora_r)
+  if (dq && scale_tma) return book ? NF4_GEMM_VARIANT(true, true, 1) : NF4_GEMM_VARIANT(true, true, 0);
+  if (dq) return book ? NF4_GEMM_VARIANT(true, false, 1) : NF4_GEMM_VARIANT(true, false, 0);
+  if (scale_tma) return book ? NF4_GEMM_VARIANT(false, true, 1) : NF4_GEMM_VARIANT(false, true, 0);
+  return book ? NF4_GEMM_VARIANT(false, false, 1) : NF4_GEMM_VARIANT(false, false, 0);
+#undef NF4_GEMM_VARIANT
 }
 
 }  // namespace
@@ -444,13 +481,14 @@ cudaError_t launch_tc(const uint8_t* packed, const Scales& s, int64_t rows, int6
   if (rows > INT32_MAX || cols > INT32_MAX || m > INT32_MAX) return cudaErrorInvalidValue;
   const bool dq = s.absmax == nullptr;
   const int64_t rb = cols / kBlock;  // level-1 blocks per weight row
+  const int tm = gemm_tile_m(m);
   CUtensorMap xmap, wmap, smap, tmap;
-  if (!make_map(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, cols, m, kTileK, kTileM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+  if (!make_map(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, cols, m, kTileK, tm, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, packed, cols / 2, rows, kTileK / 2, kTileN,
                 CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorNotSupported;
   if (lora_r > 0) {
-    if (!make_map(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, t, kTileK, m, kTileK, kTileM, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!make_map(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, t, kTileK, m, kTileK, tm, CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorNotSupported;
   } else {
     tmap = xmap;  // unused
@@ -465,7 +503,7 @@ cudaError_t launch_tc(const uint8_t* packed, const Scales& s, int64_t rows, int6
                    : make_map(&smap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, sbase, rb, rows, 4, kTileN,
                               CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!scale_tma) smap = wmap;  // unused by the kernel variant
-  const int64_t ntiles = (rows / kTileN) * ((m + kTileM - 1) / kTileM);
+  const int64_t ntiles = gemm_tiles(rows, m);
   const int64_t units = ntiles * splits;
   const int grid = (int)(units < num_sms ? units : num_sms);
   unsigned* counters = nullptr;
@@ -477,27 +515,16 @@ cudaError_t launch_tc(const uint8_t* packed, const Scales& s, int64_t rows, int6
   }
   const int R = (int)rows, C = (int)cols, M = (int)m;
   const auto* up = static_cast<const __nv_bfloat16*>(lora_up);
-  if (dq && scale_tma)
-    return s.book ? launch_variant<true, true, 1>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
-                                      tmap, up, lora_r) : launch_variant<true, true, 0>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
-                                      tmap, up, lora_r);
-  if (dq)
-    return s.book ? launch_variant<true, false, 1>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
-                                       tmap, up, lora_r) : launch_variant<true, false, 0>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
-                                       tmap, up, lora_r);
-  if (scale_tma)
-    return s.book ? launch_variant<false, true, 1>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
-                                       tmap, up, lora_r) : launch_variant<false, true, 0>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
-                                       tmap, up, lora_r);
-  return s.book ? launch_variant<false, false, 1>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
-                                      tmap, up, lora_r) : launch_variant<false, false, 0>(s, R, C, M, splits, xmap, wmap, smap, yb, part, counters, err, grid, stream,
-                                      tmap, up, lora_r);
+  return tm == 64 ? launch_book_scales<64>(dq, scale_tma, s.book, s, R, C, M, splits, xmap, wmap, smap, yb, part,
+                                           counters, err, grid, stream, tmap, up, lora_r)
+                  : launch_book_scales<256>(dq, scale_tma, s.book, s, R, C, M, splits, xmap, wmap, smap, yb, part,
+                                            counters, err, grid, stream, tmap, up, lora_r);
 }
 
 // the adapter path: its own split choice (no GEMV route for small m), the [m, 64] bf16 down-map output first
 // in the workspace, the split-K scratch after it
 int lora_splits(int64_t rows, int64_t cols, int64_t m, int num_sms) {
-  return reduction_splits((rows / kTileN) * ((m + kTileM - 1) / kTileM), cols / kTileK, num_sms);
+  return reduction_splits(gemm_tiles(rows, m), cols / kTileK, num_sms);
 }
 
 size_t lora_t_bytes(int64_t m) { return ((size_t)m * kTileK * 2 + 255) & ~(size_t)255; }
@@ -506,16 +533,16 @@ size_t lora_t_bytes(int64_t m) { return ((size_t)m * kTileK * 2 + 255) & ~(size_
 
 cudaError_t launch_gemm(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x, int64_t m,
                         void* y, void* workspace, unsigned* err, cudaStream_t stream, int num_sms) {
-  // up to 8 activation rows: the decode GEMV; from 9 rows the tensor-core kernel (its 256-row activation tile is
-  // padded with zero rows: measured 161 us -> ~41 us at 14336x4096, m = 64, against the 8-column-tile GEMV)
+  // up to 8 activation rows: the decode GEMV; from 9 rows the tensor-core kernel (64-row activation tiles up to 64
+  // rows, 256 above)
   if (m <= 8) return launch_gemv(packed, s, rows, cols, x, (int)m, y, err, stream, num_sms);
   return launch_tc(packed, s, rows, cols, x, m, y, gemm_splits(rows, cols, m, num_sms), workspace, err, stream,
                    num_sms, nullptr, nullptr, 0);
 }
 
 size_t gemm_lora_workspace_bytes(int64_t rows, int64_t cols, int64_t m) {
-  const int64_t ntiles = (rows / kTileN) * ((m + kTileM - 1) / kTileM);
-  return lora_t_bytes(m) + split_workspace_bytes(ntiles, lora_splits(rows, cols, m, sm_count()));
+  return lora_t_bytes(m) + split_workspace_bytes(gemm_tiles(rows, m), lora_splits(rows, cols, m, sm_count()),
+                                                 gemm_tile_m(m));
 }
 
 cudaError_t launch_gemm_lora(const uint8_t* packed, const Scales& s, int64_t rows, int64_t cols, const void* x,

@@ -4,7 +4,7 @@
 // persistent work split, the accumulator epilogue, and host-side tensor maps.
 //
 // Both kernels keep one accumulator tile of 128 output columns (UMMA M, TMEM
-// lanes) x 256 activation rows (UMMA N, TMEM columns) and reduce over stages of
+// lanes) x 256 activation rows (UMMA N, TMEM columns; the forward takes 64 at small M) and reduce over stages of
 // 64.  Both write a bf16 row-major output [m, ldy].
 #pragma once
 #include <cuda.h>
@@ -16,7 +16,7 @@ namespace nf4 {
 namespace umma {
 
 constexpr int kTileN = 128;  // output columns per tile (UMMA M, TMEM lanes)
-constexpr int kTileM = 256;  // activation rows per tile (UMMA N, fp32 TMEM columns)
+constexpr int kTileM = 256;  // activation rows per tile (UMMA N, fp32 TMEM columns); the forward GEMM also uses 64
 constexpr int kAccCols = kTileM;
 constexpr int kEpiWarps = 4;                  // warps 0..3 read TMEM lanes 32w..32w+31
 constexpr int kStageOutBytes = 32 * 32 * 2;   // per epilogue warp: 32 rows x 32 columns of bf16
@@ -153,10 +153,11 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Sm
 // ready for the next call.
 struct Work {
   int ntiles_m, units, splits, kps;
+  int tm;  // activation rows per tile
   __device__ int tile(int u) const { return u / splits; }
   __device__ int split(int u) const { return u % splits; }
   __device__ int n0(int u) const { return (tile(u) / ntiles_m) * kTileN; }  // first output column
-  __device__ int m0(int u) const { return (tile(u) % ntiles_m) * kTileM; }  // first activation row
+  __device__ int m0(int u) const { return (tile(u) % ntiles_m) * tm; }      // first activation row
 };
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory"); }
@@ -173,19 +174,28 @@ struct EpiOut {
 // columns = activation rows m0 .. m0+255) -> Y, run by warps 0..3.  Releases
 // the accumulator through `acc_empty` as soon as it has been read.
 // Shared memory the split reduction stages the other splits' partials in: 16 bytes per piece and epilogue
-// thread; pieces = own 32-row chunks (ceil(8 / splits)) x 2 halves x (splits - 1) other partials x 4, at most
-// 48 (32 with two splits, 48 with three or four): 96 KB with 128 epilogue threads.
+// thread; pieces = own 32-row chunks (ceil(TM / 32 / splits)) x 2 halves x (splits - 1) other partials x 4.
+// With 2 to 4 splits that is at most 48 pieces (96 KB with 128 epilogue threads) for TM = 256 and 24 (48 KB)
+// for TM = 64.
 static_assert(kMaxSplits <= 4, "split staging size");
-constexpr int kSplitStagePieces = 48;
-constexpr int kSplitStageBytes = kSplitStagePieces * kEpiWarps * 32 * 16;
+__host__ __device__ constexpr int split_stage_pieces(int tm) {
+  int best = 0;
+  for (int sp = 2; sp <= kMaxSplits; ++sp) {
+    const int p = ((tm / 32 + sp - 1) / sp) * 2 * (sp - 1) * 4;
+    best = p > best ? p : best;
+  }
+  return best;
+}
+__host__ __device__ constexpr int split_stage_bytes(int tm) { return split_stage_pieces(tm) * kEpiWarps * 32 * 16; }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
 
-// `stage_in`: kSplitStageBytes of shared memory that is idle once the unit's MMAs have finished (the operand
-// ring; with splits > 1 a CTA has a single unit, so nothing refills it)
-template <class Sm>
+// TM: activation rows of the tile (accumulator columns).  `stage_in`: split_stage_bytes(TM) of shared memory
+// that is idle once the unit's MMAs have finished (the operand ring; with splits > 1 a CTA has a single unit, so
+// nothing refills it)
+template <int TM, class Sm>
 __device__ __forceinline__ void epilogue_unit(const Work& wk, int u, uint32_t taddr, uint16_t* out_stage, Sm* sm,
                                               uint64_t* acc_empty, const EpiOut& o, uint8_t* stage_in) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -209,7 +219,7 @@ __device__ __forceinline__ void epilogue_unit(const Work& wk, int u, uint32_t ta
   };
   if (wk.splits == 1) {
 #pragma unroll 1
-    for (int c = 0; c < kTileM / 32; ++c) {
+    for (int c = 0; c < TM / 32; ++c) {
       uint32_t v[32];
       tmem_ld32(taddr + c * 32, v);
 #pragma unroll
@@ -225,9 +235,9 @@ __device__ __forceinline__ void epilogue_unit(const Work& wk, int u, uint32_t ta
   // 16-byte access of a warp covers 32 consecutive n, 512 contiguous bytes), except the 32-row chunks this
   // split reduces itself (c = split, split + splits, ...): those stay in TMEM until the reduction.
   const int my = wk.split(u);
-  float* mine = o.part + (size_t)u * (kTileN * kTileM);
+  float* mine = o.part + (size_t)u * (kTileN * TM);
 #pragma unroll 1
-  for (int c = 0; c < kTileM / 32; ++c) {
+  for (int c = 0; c < TM / 32; ++c) {
     if (c % wk.splits == my) continue;
     uint32_t v[32];
     tmem_ld32(taddr + c * 32, v);
@@ -260,14 +270,14 @@ __device__ __forceinline__ void epilogue_unit(const Work& wk, int u, uint32_t ta
   epi_bar();
   if (!aborted(sm)) {
     __threadfence();
-    const float* tp = o.part + (size_t)wk.tile(u) * wk.splits * (kTileN * kTileM);
+    const float* tp = o.part + (size_t)wk.tile(u) * wk.splits * (kTileN * TM);
     // Every other split's partial of this split's chunks, copied into shared memory with all copies in flight
     // at once (one round of L2 latency), piece p of this thread at stage_in + (p * 128 + nl) * 16.
     const uint32_t stage = smem_u32(stage_in);
     fence_proxy_async_smem();  // the ring was last written by TMA and read by the MMAs
     int pc = 0;
 #pragma unroll 1
-    for (int c = my; c < kTileM / 32; c += wk.splits)
+    for (int c = my; c < TM / 32; c += wk.splits)
 #pragma unroll
       for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -277,14 +287,14 @@ __device__ __forceinline__ void epilogue_unit(const Work& wk, int u, uint32_t ta
 #pragma unroll
             for (int j = 0; j < 4; ++j, ++pc)
               cp_async16(stage + (uint32_t)(pc * (kEpiWarps * 32) + nl) * 16u,
-                         tp + (size_t)sp * (kTileN * kTileM) + ((size_t)(c * 8 + h * 4 + j) * kTileN + nl) * 4);
+                         tp + (size_t)sp * (kTileN * TM) + ((size_t)(c * 8 + h * 4 + j) * kTileN + nl) * 4);
           }
         }
     asm volatile("cp.async.commit_group;\n cp.async.wait_group 0;" ::: "memory");
     const float4* staged = reinterpret_cast<const float4*>(stage_in);
     pc = 0;
 #pragma unroll 1
-    for (int c = my; c < kTileM / 32; c += wk.splits) {
+    for (int c = my; c < TM / 32; c += wk.splits) {
       uint32_t v[32];
       tmem_ld32(taddr + c * 32, v);  // this split's own partial of the chunk
 #pragma unroll
@@ -353,8 +363,8 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType type, size_t esize, const vo
 // split at least 8 stages.
 int reduction_splits(int64_t ntiles, int64_t stages, int num_sms);
 
-// bytes of the split-K workspace: one counter per tile, then the fp32 partials
-size_t split_workspace_bytes(int64_t ntiles, int splits);
+// bytes of the split-K workspace: one counter per tile, then the fp32 partials of tm-row tiles
+size_t split_workspace_bytes(int64_t ntiles, int splits, int tm = kTileM);
 
 int sm_count();
 
