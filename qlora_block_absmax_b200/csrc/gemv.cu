@@ -241,27 +241,32 @@ template <int NT, int kBook>
 cudaError_t launch_nt(const GemvGroup& grp, int64_t cols, const void* x, int batch, bool dq, cudaStream_t stream) {
   const unsigned grid = (unsigned)grp.tile_end[grp.count - 1];
   const auto* xb = static_cast<const __nv_bfloat16*>(x);
-  cudaError_t e;
-  if (NT == 1 && batch == 1) {  // decode at batch 1: the mixed decode with the 64 KB pair table
-    // the table needs the shared-memory opt-in: set it once per device and variant
-    static std::atomic<uint64_t> attr_done[2];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!(attr_done[dq].load() & (1ull << dev))) {
-      e = cudaFuncSetAttribute(dq ? (const void*)gemv_kernel<NT, true, true, kBook> : (const void*)gemv_kernel<NT, false, true, kBook>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, kPairTableBytes);
-      if (e != cudaSuccess) return e;
-      attr_done[dq].fetch_or(1ull << dev);
+  cudaError_t e = cudaSuccess;
+  bool table = false;
+  if constexpr (NT == 1) table = batch == 1;  // decode at batch 1: the mixed decode with the 64 KB pair table
+  if constexpr (NT == 1) {
+    if (table) {
+      // the table needs the shared-memory opt-in: set it once per device and variant
+      static std::atomic<uint64_t> attr_done[2];
+      int dev = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+      if (!(attr_done[dq].load() & (1ull << dev))) {
+        e = cudaFuncSetAttribute(
+            dq ? (const void*)gemv_kernel<NT, true, true, kBook> : (const void*)gemv_kernel<NT, false, true, kBook>,
+            cudaFuncAttributeMaxDynamicSharedMemorySize, kPairTableBytes);
+        if (e != cudaSuccess) return e;
+        attr_done[dq].fetch_or(1ull << dev);
+      }
+      e = dq ? launch_pdl(gemv_kernel<NT, true, true, kBook>, dim3(grid), dim3(kWarps * 32), kPairTableBytes, stream,
+                          grp, cols, xb, batch)
+             : launch_pdl(gemv_kernel<NT, false, true, kBook>, dim3(grid), dim3(kWarps * 32), kPairTableBytes, stream,
+                          grp, cols, xb, batch);
     }
-    e = dq ? launch_pdl(gemv_kernel<NT, true, true, kBook>, dim3(grid), dim3(kWarps * 32), kPairTableBytes, stream, grp,
-                        cols, xb, batch)
-           : launch_pdl(gemv_kernel<NT, false, true, kBook>, dim3(grid), dim3(kWarps * 32), kPairTableBytes, stream, grp,
-                        cols, xb, batch);
-  } else {
+  }
+  if (!table)
     e = dq ? launch_pdl(gemv_kernel<NT, true, false, kBook>, dim3(grid), dim3(kWarps * 32), 0, stream, grp, cols, xb, batch)
            : launch_pdl(gemv_kernel<NT, false, false, kBook>, dim3(grid), dim3(kWarps * 32), 0, stream, grp, cols, xb,
                         batch);
-  }
   count_launches(1);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
