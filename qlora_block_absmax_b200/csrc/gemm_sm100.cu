@@ -7,20 +7,20 @@
 // expansion happens tile by tile in shared memory, and the multiply is a
 // tcgen05 bf16 x bf16 -> fp32 MMA with the accumulator in tensor memory.
 //
-// Tile: 128 weight rows (UMMA M, operand A) x 256 activation rows (UMMA N,
-// operand B) x 64 k per pipeline stage (one level-1 block per weight row).
-// D[n, m] lives in TMEM (lane = weight row, column = activation row, 256
-// columns); the decoded weight tile goes straight into TMEM too (a 3-stage
-// ring of 32 columns: lane = weight row, column j = codes 2j, 2j+1 as bf16x2),
-// so the MMA reads only the activation tile from shared memory.  One
-// persistent CTA per SM walks the tiles; warp roles:
+// Tile: 128 weight rows (UMMA M, operand A) x TM activation rows (UMMA N,
+// operand B; TM = 256, or 64 while m <= 64) x 64 k per pipeline stage (one
+// level-1 block per weight row).  D[n, m] lives in TMEM (lane = weight row,
+// column = activation row, TM columns); the decoded weight tile goes straight
+// into TMEM too (a 2G-stage ring of 32 columns: lane = weight row, column j =
+// codes 2j, 2j+1 as bf16x2), so the MMA reads only the activation tile from
+// shared memory.  One persistent CTA per SM walks the tiles; warp roles:
 //   warps 0-3   epilogue: tcgen05.ld -> bf16 -> Y (warp w reads TMEM lanes 32w..)
 //   warps 4..4+4G-1  dequant producers, G groups of four taking stages in
 //               turn: thread p decodes weight row p of the stage (64 codes)
 //               with the byte-permute tables and stores it to its TMEM lane
 //               (tcgen05.st); a decode is a long dependent chain per thread,
 //               so the groups in flight are what keep the issue slots busy
-//   next warp   TMA producer: activation tile (256 x 64 bf16, 128B swizzle)
+//   next warp   TMA producer: activation tile (TM x 64 bf16, 128B swizzle)
 //   next warp   TMEM allocator and MMA issuer (one elected thread)
 //   last warp   TMA producer: packed codes and 16-byte scale chunks
 // With a low-rank adapter (QLoRA: "bitsandbytes quantization tutorial",
