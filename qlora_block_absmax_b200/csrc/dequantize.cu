@@ -18,6 +18,9 @@ namespace nf4 {
 namespace {
 
 __constant__ float c_code[2][16] = {NF4_CODE_INIT, FP4_CODE_INIT};  // by code book: NF4, FP4
+// bf16 output: warps per CTA.  Four (up to 16 CTAs per SM) measured 1 % faster than eight at 4096x4096 and 17 %
+// at 1024x1024: the last partial wave of CTAs is smaller.
+constexpr int kDeqWarps = 4;
 
 template <bool kDQ>
 __device__ __forceinline__ float block_scale(const Scales& s, const float* unit_lut, int64_t b) {
@@ -104,12 +107,13 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restri
 // warp's 32 consecutive blocks (4 KB of bf16) go through a swizzled shared
 // tile so the global stores are 512 contiguous bytes per instruction.
 template <bool kDQ, int kBook, int kB>
-__global__ void __launch_bounds__(256) dequantize_bf16_kernel(const uint8_t* __restrict__ packed, Scales s,
+__global__ void __launch_bounds__(kDeqWarps * 32) dequantize_bf16_kernel(const uint8_t* __restrict__ packed, Scales s,
                                                               int64_t n, __nv_bfloat16* __restrict__ out) {
   __shared__ float unit_lut[kDQ ? 256 : 1];
-  __shared__ __align__(16) uint4 stage[8][32 * 8];  // per warp: 32 blocks x 8 chunks of 16 bytes
+  __shared__ __align__(16) uint4 stage[kDeqWarps][32 * 8];  // per warp: 32 chunks x 8 pieces of 16 bytes
   pdl_launch_dependents();
-  if (kDQ) unit_lut[threadIdx.x & 255] = dq_unit(threadIdx.x & 255, s.dq_code);
+  if (kDQ)
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) unit_lut[i] = dq_unit(i, s.dq_code);
   __syncthreads();
   pdl_wait();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -181,13 +185,13 @@ cudaError_t launch_block(const uint8_t* packed, const Scales& s, int64_t n, void
   const bool dq = s.absmax == nullptr;
   cudaError_t e;
   if (out_bf16) {
-    int64_t g2 = ((n + kBlock - 1) / kBlock + 255) / 256;  // 8 warps x 32 chunks of 64 per CTA per pass
-    if (g2 > cap) g2 = cap;
+    int64_t g2 = ((n + kBlock - 1) / kBlock + 32 * kDeqWarps - 1) / (32 * kDeqWarps);  // 32 chunks of 64 per warp
+    if (g2 > 2 * cap) g2 = 2 * cap;
     if (g2 < 1) g2 = 1;
     auto* ob = static_cast<__nv_bfloat16*>(out);
-    e = dq ? launch_pdl(dequantize_bf16_kernel<true, kBook, kB>, dim3((unsigned)g2), dim3(256), 0, stream, packed, s, n,
+    e = dq ? launch_pdl(dequantize_bf16_kernel<true, kBook, kB>, dim3((unsigned)g2), dim3(kDeqWarps * 32), 0, stream, packed, s, n,
                         ob)
-           : launch_pdl(dequantize_bf16_kernel<false, kBook, kB>, dim3((unsigned)g2), dim3(256), 0, stream, packed, s,
+           : launch_pdl(dequantize_bf16_kernel<false, kBook, kB>, dim3((unsigned)g2), dim3(kDeqWarps * 32), 0, stream, packed, s,
                         n, ob);
   } else {
     constexpr int kL = kB / 16;
