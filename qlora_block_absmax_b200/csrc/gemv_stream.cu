@@ -50,7 +50,7 @@ namespace {
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
 constexpr int kStepCols = 256;                 // columns per warp step (4 level-1 blocks)
-constexpr int kGroupSteps = 2;                 // steps per round-robin group
+constexpr int kGroupSteps = 4;                 // steps per round-robin group
 constexpr int kSlots = 4;                      // partial-sum slots (tiles in flight per CTA)
 constexpr int kPairTableBytes = 256 * 32 * 8;  // fp32 code pairs, one copy per lane
 constexpr int kSlotFloats = kWarps * 16 * 8;   // one slot: [group in tile][row][batch column]
@@ -255,7 +255,7 @@ __device__ __forceinline__ void prefetch_tile(const Params<kMax>& p, int j, int 
 // tiles prefetched ahead of the one a CTA starts: about 128 KB of codes
 __device__ __forceinline__ int prefetch_distance(int cols) { return max(2, 131072 / (8 * cols)); }
 
-template <int kMax, int kP0, int kP1, int kBook, int kOpt>
+template <int kMax, int kP0, int kP1, int kBook>
 __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_constant__ Params<kMax> p,
                                                                   unsigned* err) {
   extern __shared__ __align__(16) uint8_t smem[];
@@ -308,10 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
   // prmt source for table addresses: byte 0 = 8 * lane, byte 1 = 0, bytes 2-3 = the table's 64 KB-aligned base
   const uint32_t lane_base = (uint32_t)(lane * 8) | (uint32_t)__cvta_generic_to_shared(table);
   const DecodeMul dm = decode_mul();
-  // options: bit 0 groups of 4 steps (else 2); bit 1 block scales rebuilt one step ahead; bit 2 release/acquire
-  // atomics for the partial hand-off instead of a block fence; bit 3 a step's activation loads issued up front
-  constexpr int kG = (kOpt & 1) ? 4 : 2;
-  constexpr bool kPre = (kOpt & 2) != 0, kRel = (kOpt & 4) != 0, kXHoist = (kOpt & 8) != 0;
+  constexpr int kG = kGroupSteps;  // steps per round-robin group
 
   // this warp's walk
   Walk wk;
@@ -359,7 +356,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
     // slot free: the reduction of tile cur_lj - kSlots is done (red_gen counts the slot's finished reductions)
     const int want = cur_lj / kSlots;
     auto gen_now = [&]() {
-      if (!kRel) return *(volatile int*)&red_gen[slot];
       int v;
       asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(&red_gen[slot])) : "memory");
       return v;
@@ -379,26 +375,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
     *reinterpret_cast<float2*>(r + (g + 8) * 8 + 2 * t) = make_float2(acc[2] + acc2[2], acc[3] + acc2[3]);
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[i] = acc2[i] = 0.0f;
-    if (!kRel) __threadfence_block();
     __syncwarp();
     const int tile = t_begin + cur_lj;
     while (tile >= p.tile_end[red_item]) ++red_item;
     const Item& it = p.item[red_item];
     const int parts = min(kWarps, tile_groups<kG>(it.cols));
     int last = 0;
-    if (lane == 0) {
-      if (kRel) {  // release this warp's partial (ordered before lane 0 by __syncwarp); acquire the others'
-        uint32_t old;
-        asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;"
-                     : "=r"(old) : "r"(smem_u32(&red_count[slot])) : "memory");
-        last = (int)old == parts - 1;
-      } else {
-        last = atomicAdd(&red_count[slot], 1) == parts - 1;
-      }
+    if (lane == 0) {  // release this warp's partial (ordered before lane 0 by __syncwarp); acquire the others'
+      uint32_t old;
+      asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;"
+                   : "=r"(old) : "r"(smem_u32(&red_count[slot])) : "memory");
+      last = (int)old == parts - 1;
     }
     last = __shfl_sync(0xffffffffu, last, 0);
     if (last) {  // the tile's last warp: partials in group order, then y
-      if (!kRel) __threadfence_block();
       __syncwarp();
       const int64_t rows = (int64_t)(p.tile_end[red_item] - tile_begin(p, red_item)) * 16;
       const int64_t row0 = (int64_t)(tile - tile_begin(p, red_item)) * 16;
@@ -412,12 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
       __syncwarp();
       if (lane == 0) {
         red_count[slot] = 0;
-        if (kRel) {
-          asm volatile("red.release.cta.shared::cta.add.u32 [%0], 1;" ::"r"(smem_u32(&red_gen[slot])) : "memory");
-        } else {
-          __threadfence_block();
-          atomicAdd(&red_gen[slot], 1);
-        }
+        asm volatile("red.release.cta.shared::cta.add.u32 [%0], 1;" ::"r"(smem_u32(&red_gen[slot])) : "memory");
       }
     }
   };
@@ -434,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
     }
   };
   auto prep = [&](Step& d) {
-    if (kPre && d.lj >= 0) rebuild(d, d.a0, d.a1);
+    if (d.lj >= 0) rebuild(d, d.a0, d.a1);
   };
 
   // decode + multiply one step into the accumulators
@@ -444,18 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
       cur_lj = d.lj;
     }
     cur_info = d.info;
-    float a0, a1;
-    if (kPre) {
-      a0 = d.a0;
-      a1 = d.a1;
-    } else {
-      rebuild(d, a0, a1);
-    }
-    uint4 xh[kXHoist ? 8 : 1];
-    if (kXHoist) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) xh[j] = __ldg(reinterpret_cast<const uint4*>(d.xp + 8 * j));
-    }
+    const float a0 = d.a0, a1 = d.a1;  // rebuilt one step ahead (prep)
     Table T0, T1;
     if (kP0 > 0) T0 = make_table<kBook>(a0);
     if (kP1 > 0) T1 = make_table<kBook>(a1);
@@ -466,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
       uint32_t e0[4], e1[4];
       if (j < kP0) decode_word(w0[j], T0, e0, dm); else table_decode(w0[j], a0, lane_base, e0);
       if (j < kP1) decode_word(w1[j], T1, e1, dm); else table_decode(w1[j], a1, lane_base, e1);
-      const uint4 xv = kXHoist ? xh[j] : __ldg(reinterpret_cast<const uint4*>(d.xp + 8 * j));
+      const uint4 xv = __ldg(reinterpret_cast<const uint4*>(d.xp + 8 * j));
       float(&c)[4] = (j & 1) ? acc2 : acc;
       mma_bf16(c, e0[0], e1[0], e0[1], e1[1], xv.x, xv.y);
       mma_bf16(c, e0[2], e1[2], e0[3], e1[3], xv.z, xv.w);
@@ -474,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
   };
 
   // two steps in flight: consume one while the next one's loads are outstanding (its scales, loaded a step
-  // earlier, are rebuilt right after the current step when kPre)
+  // earlier, are rebuilt right after the current step)
   prep(b0);
   for (;;) {
     if (b0.lj < 0) break;
@@ -491,19 +465,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
   flush();
 }
 
-template <int kMax, int kP0, int kP1, int kBook, int kOpt = 0>
+template <int kMax, int kP0, int kP1, int kBook>
 cudaError_t launch_variant(const Params<kMax>& p, int grid, unsigned* err, cudaStream_t stream) {
   constexpr size_t smem = kSmemBytes;
   static bool attr_done[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_done[dev]) {  // idempotent: a race only repeats the call
-    const cudaError_t e = cudaFuncSetAttribute(gemv_stream_kernel<kMax, kP0, kP1, kBook, kOpt>,
+    const cudaError_t e = cudaFuncSetAttribute(gemv_stream_kernel<kMax, kP0, kP1, kBook>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr_done[dev] = true;
   }
-  const cudaError_t e = launch_pdl(gemv_stream_kernel<kMax, kP0, kP1, kBook, kOpt>, dim3(grid), dim3(kThreads), smem, stream, p, err);
+  const cudaError_t e = launch_pdl(gemv_stream_kernel<kMax, kP0, kP1, kBook>, dim3(grid), dim3(kThreads), smem, stream, p, err);
   count_launches(1);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
@@ -517,7 +491,7 @@ cudaError_t launch_items(const GemvItem* items, int count, int batch, unsigned* 
     const GemvItem& s = items[i];
     if (s.cols > INT32_MAX) return cudaErrorInvalidValue;
     tiles += s.rows / 16;
-    work += s.rows / 16 * tile_groups<4>((int)s.cols);
+    work += s.rows / 16 * tile_groups<kGroupSteps>((int)s.cols);
     if (tiles > INT32_MAX) return cudaErrorInvalidValue;
     Item& d = p.item[i];
     d.packed = s.packed;
@@ -547,7 +521,7 @@ cudaError_t launch_items(const GemvItem* items, int count, int batch, unsigned* 
   for (int c = 1; c < grid; ++c) {
     const int64_t target = work * c / grid;
     for (;;) {
-      const int64_t n = items[item].rows / 16, per = tile_groups<4>((int)items[item].cols);
+      const int64_t n = items[item].rows / 16, per = tile_groups<kGroupSteps>((int)items[item].cols);
       if (item == count - 1 || target < wb + n * per) {
         const int64_t k = std::min(n, std::max<int64_t>(0, (target - wb + per / 2) / per));
         p.cta_tile[c] = std::max<int32_t>(p.cta_tile[c - 1], (int32_t)(t0 + k));
@@ -568,10 +542,10 @@ cudaError_t launch_items(const GemvItem* items, int count, int batch, unsigned* 
   // options 7: groups of 4 steps, scales rebuilt one step ahead, release/acquire hand-off of the partials (measured
   // 4-7% faster than none of them at 14336x4096, batch 1 and 8; hoisting a step's activation loads spilled)
   if (batch == 1)
-    return book ? launch_variant<kMax, 6, 0, 1, 7>(p, grid, err, stream)
-                : launch_variant<kMax, 6, 0, 0, 7>(p, grid, err, stream);
-  return book ? launch_variant<kMax, 8, 0, 1, 7>(p, grid, err, stream)
-              : launch_variant<kMax, 8, 0, 0, 7>(p, grid, err, stream);
+    return book ? launch_variant<kMax, 6, 0, 1>(p, grid, err, stream)
+                : launch_variant<kMax, 6, 0, 0>(p, grid, err, stream);
+  return book ? launch_variant<kMax, 8, 0, 1>(p, grid, err, stream)
+              : launch_variant<kMax, 8, 0, 0>(p, grid, err, stream);
 }
 
 }  // namespace
