@@ -72,19 +72,6 @@ __device__ __forceinline__ uint32_t code_fast_fp4(uint32_t entry, float q, float
   return (e & 15u) + (aq > thr ? 1u : 0u) + ((__float_as_uint(q) >> 31) << 3);
 }
 
-// `entry` is this lane's bucket word; every lane of the warp must call this
-// (the lookup is a shuffle).  q estimates w / a within 3 * 2^-24.  `gap`
-// tracks the smallest distance between an estimate and its entry.
-__device__ __forceinline__ uint32_t code_fast(uint32_t entry, float q, float& gap) {
-  // v = 2^23 + 16 + floor(16 S q) lies in [2^23, 2^23 + 32): the bucket is its low 5 mantissa bits,
-  // and a shuffle takes its source lane modulo 32
-  const float v = __fmaf_rd(q, 16.0f * NF4_Q32_SCALE, 0x1p23f + 16.0f);
-  const uint32_t e = __shfl_sync(0xffffffffu, entry, __float_as_int(v));
-  const float thr = __uint_as_float(e);
-  gap = fminf(gap, fabsf(q - thr));
-  return (e & 15u) + (q > thr ? 1u : 0u);
-}
-
 // Two elements of NF4 at once: q = w * r and the bucket value v = RD(16 S q + 2^23 + 16) as paired fp32
 // operations (each half rounded as its scalar form), two shuffles fetch the bucket entries, and d = thr - q (also
 // paired, exact in sign: the difference of two fp32 values is never rounded to zero) gives both the decision
