@@ -427,9 +427,11 @@ def run_ours(args):
     recs = [nf4.QuantizedWeight(packed=c0.packed.clone(), rows=ROWS, cols=COLS, absmax_q=c0.q.clone(),
                                 absmax_scale=c0.scale.clone(), absmax_mean=c0.mean.clone(), dq_code=nf4.NF4_DQ_E4M3)
             for _ in range(k_rec)]
-    deq_out = [torch.empty(ROWS, COLS, dtype=torch.bfloat16, device=dev) for _ in range(4)]
-    per_kernel_ms["dequantize"] = time_calls([lambda q=q, o=deq_out[i % 4]: nf4.dequantize(q, torch.bfloat16, out=o)
-                                              for i, q in enumerate(recs)])
+    # a fresh output per call as well (every write goes to lines not in L2, like every read)
+    deq_out = [torch.empty(ROWS, COLS, dtype=torch.bfloat16, device=dev) for _ in range(k_rec)]
+    per_kernel_ms["dequantize"] = time_calls([lambda q=q, o=o: nf4.dequantize(q, torch.bfloat16, out=o)
+                                              for q, o in zip(recs, deq_out)])
+    del deq_out
     ys = [torch.empty(GEMV_B, ROWS, dtype=torch.bfloat16, device=dev) for _ in range(k_rec)]
     per_kernel_ms["gemv"] = time_calls([lambda q=q, y=y: nf4.gemv(q, c0.x, out=y) for q, y in zip(recs, ys)])
     Xs = [cs[i % copies].X for i in range(3)]
@@ -446,7 +448,7 @@ def run_ours(args):
                                                                                workspace=c0.lws)
                                  for i, q in enumerate(recs)]),
     }
-    del recs, ys, Ys, dXs, deq_out
+    del recs, ys, Ys, dXs
 
     # ------------------------------------------------------------------ configs
     configs = {}

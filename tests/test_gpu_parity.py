@@ -341,21 +341,25 @@ def test_gemm_split_k(m):
 
 
 def test_gemm_deterministic_and_bench_shape():
-    """4096 x 4096 weight, M = 256 (split-K path): bit-identical across calls,
-    sampled outputs within tolerance"""
+    """4096 x 4096 weight, M = 256 (split-K path), the step's own product: bit-identical across calls and every one
+    of the 1,048,576 outputs within tolerance of the oracle"""
     rows, cols, m = 4096, 4096, 256
     qw, p_ref, a_ref = quantized_pair(rows, cols, 1002, True)
     x = synth.activations((m, cols), 1277)
     y1 = nf4.gemm(qw, dev_bf16(x))
     y2 = nf4.gemm(qw, dev_bf16(x))
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
-    r = synth.rng(9)
-    bs, ns = r.integers(0, m, 4096), r.integers(0, rows, 4096)
-    ref = oracle.matmul_sampled(p_ref, a_ref, rows, cols, x, bs, ns)
-    full_row = oracle.matmul(p_ref, a_ref, rows, cols, x[:1])
-    rms = np.sqrt(np.mean(full_row ** 2))
-    got = y1.float().cpu().numpy().astype(np.float64)[bs, ns]
-    assert np.all(np.abs(got - ref) <= REL_TOL * np.maximum(np.abs(ref), FLOOR * rms))
+    check_matmul(y1, oracle.matmul(p_ref, a_ref, rows, cols, x), "gemm 4096x4096 m256 in full")
+
+
+def test_gemm_dx_bench_shape_in_full():
+    """dX = dY . Wc for the 4096 x 4096 weight at M = 256 (split-K path), every one of the 1,048,576 outputs within
+    tolerance of the oracle"""
+    rows, cols, m = 4096, 4096, 256
+    qw, p_ref, a_ref = quantized_pair(rows, cols, 1003, True)
+    dy = synth.activations((m, rows), 1279)
+    dx = nf4.gemm_dx(qw, dev_bf16(dy))
+    check_matmul(dx, oracle.matmul_dx(p_ref, a_ref, rows, cols, dy), "dx 4096x4096 m256 in full")
 
 
 @pytest.mark.parametrize("rows,m", [(14336, 1024), (4096, 4096), (14336, 256)])
