@@ -11,9 +11,12 @@
 // operand B; TM = 256, or 64 while m <= 64) x 64 k per pipeline stage (one
 // level-1 block per weight row).  D[n, m] lives in TMEM (lane = weight row,
 // column = activation row, TM columns); the decoded weight tile goes straight
-// into TMEM too (a 2G-stage ring of 32 columns: lane = weight row, column j =
-// codes 2j, 2j+1 as bf16x2), so the MMA reads only the activation tile from
-// shared memory.  One persistent CTA per SM walks the tiles; warp roles:
+// into TMEM too (32 columns per stage of the operand ring: lane = weight row,
+// column j = codes 2j, 2j+1 as bf16x2), so the MMA reads only the activation
+// tile from shared memory.  The issuing thread is the pipeline's critical path
+// (each tcgen05 instruction and barrier test costs it tens of cycles), so a
+// stage's two tiles share one full and one empty barrier.  One persistent CTA
+// per SM walks the tiles; warp roles:
 //   warps 0-3   epilogue: tcgen05.ld -> bf16 -> Y (warp w reads TMEM lanes 32w..)
 //   warps 4..4+4G-1  dequant producers, G groups of four taking stages in
 //               turn: thread p decodes weight row p of the stage (64 codes)
@@ -50,7 +53,6 @@ constexpr int kTileK = 64;        // k per stage (128 bytes of bf16: one swizzle
 // producer groups of four warps, one stage each in turn (3 or 4 groups -- more warps with fewer registers each --
 // measured 3 to 25 % slower at every shape)
 constexpr int kGroups = 2;
-constexpr int kAStages = 2 * kGroups;     // decoded weight-tile ring in TMEM (written by the producer warps)
 constexpr int kWStages = 6;  // packed-code + scale ring (TMA from HBM), deeper to hide its latency
 constexpr int kWBytes = kTileN * kTileK / 2;  // 4 KB: packed codes of the weight tile
 constexpr int kSBytes = kTileN * 16;          // 2 KB: 16-byte scale chunk per weight row
@@ -59,30 +61,31 @@ constexpr int kTmaWarp = kProdWarp0 + 4 * kGroups;  // activation tiles
 constexpr int kMmaWarp = kTmaWarp + 1;
 constexpr int kTmaWWarp = kTmaWarp + 2;             // packed codes and scales
 constexpr int kThreads = (kTmaWWarp + 1) * 32;
-constexpr int kXStagesMax = 8;
+constexpr int kStagesMax = 8;
 
 // Per activation-tile width TM (the UMMA N: 256, or 64 for up to 64 activation rows, where a 256-wide tile would
-// spend three quarters of every MMA on padding rows): the activation ring and the TMEM budget.
+// spend three quarters of every MMA on padding rows): the operand ring and the TMEM budget.  Stage s of the ring
+// is an activation tile in shared memory (TMA) and a decoded weight tile in TMEM columns (producer warps) that
+// fill and empty together: one full barrier (the TMA's bytes + the four producer warps of the stage's group) and
+// one empty barrier (one tcgen05.commit), so the single MMA-issuing thread waits once and commits once per stage.
 template <int TM>
 struct TileCfg {
-  static constexpr int kXStages = TM == 256 ? 5 : 8;  // activation-tile ring (TMA from L2/HBM)
-  static constexpr int kBBytes = TM * kTileK * 2;     // activation tile (operand B): 32 KB at TM = 256
-  static constexpr int kRingBytes = kXStages * kBBytes + kWStages * (kWBytes + kSBytes);  // A lives in TMEM
-  static constexpr int kTmemCols = TM + kAStages * 32 <= 256 ? 256 : 512;  // accumulator + A ring, a power of 2
+  static constexpr int kStages = TM == 256 ? 5 : 8;  // operand ring depth
+  static constexpr int kBBytes = TM * kTileK * 2;    // activation tile (operand B): 32 KB at TM = 256
+  static constexpr int kRingBytes = kStages * kBBytes + kWStages * (kWBytes + kSBytes);  // A lives in TMEM
+  static constexpr int kTmemCols = TM + kStages * 32 <= 256 ? 256 : 512;  // accumulator + A ring, a power of 2
   static constexpr size_t kSmemBytes = (size_t)kRingBytes + kEpiWarps * kStageOutBytes + 1024 /*align*/ +
                                        2048 /*barriers, lut*/;
-  static_assert(kXStages * kBBytes >= split_stage_bytes(TM), "split reduction staging fits in the operand ring");
-  static_assert(TM + kAStages * 32 <= kTmemCols, "TMEM: accumulator + A ring");
-  static_assert(kXStages <= kXStagesMax, "barrier array");
+  static_assert(kStages * kBBytes >= split_stage_bytes(TM), "split reduction staging fits in the operand ring");
+  static_assert(TM + kStages * 32 <= kTmemCols, "TMEM: accumulator + A ring");
+  static_assert(kStages <= kStagesMax, "barrier array");
 };
 
 struct Smem {  // placed after the 1024-aligned stage buffers
   uint64_t wfull[kWStages];   // packed codes + scale chunk landed (TMA)
   uint64_t wempty[kWStages];  // codes read by the producer warps
-  uint64_t xfull[kXStagesMax];   // activation tile landed (TMA)
-  uint64_t xempty[kXStagesMax];  // activation tile consumed by the MMAs (tcgen05.commit)
-  uint64_t afull[kAStages];   // decoded weight tile written (producer warps)
-  uint64_t aempty[kAStages];  // decoded tile consumed by the MMAs (tcgen05.commit)
+  uint64_t full[kStagesMax];   // activation tile landed (TMA) and decoded weight tile written (producer warps)
+  uint64_t empty[kStagesMax];  // both consumed by the stage's MMAs (tcgen05.commit)
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint32_t tmem_base;
@@ -107,7 +110,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 unsigned* err, const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __restrict__ lora_up,
                 int lora_r) {
   using Cfg = TileCfg<TM>;
-  constexpr int kXStages = Cfg::kXStages, kBBytes = Cfg::kBBytes, kRingBytes = Cfg::kRingBytes;
+  constexpr int kStages = Cfg::kStages, kBBytes = Cfg::kBBytes, kRingBytes = Cfg::kRingBytes;
   constexpr int kTmemCols = Cfg::kTmemCols;
   constexpr int kAccColsT = TM;  // accumulator columns; the A ring follows
   extern __shared__ uint8_t smem_raw[];
@@ -116,7 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;  // 1024-aligned stage buffers (swizzle atoms)
   uint8_t* gbase = smem_raw + (base - raw);
   const uint32_t b_smem0 = base;
-  const uint32_t w_smem0 = b_smem0 + kXStages * kBBytes, s_smem0 = w_smem0 + kWStages * kWBytes;
+  const uint32_t w_smem0 = b_smem0 + kStages * kBBytes, s_smem0 = w_smem0 + kWStages * kWBytes;
   const uint8_t* w_gen0 = gbase + (w_smem0 - base);
   const uint8_t* s_gen0 = gbase + (s_smem0 - base);
   uint16_t* out_stage = reinterpret_cast<uint16_t*>(gbase + kRingBytes);  // epilogue transpose
@@ -135,13 +138,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm->wfull[i], 1);   // TMA arrive.expect_tx
       mbar_init(&sm->wempty[i], 4);  // the 4 producer warps of the stage's group
     }
-    for (int i = 0; i < kXStages; ++i) {
-      mbar_init(&sm->xfull[i], 1);   // TMA arrive.expect_tx
-      mbar_init(&sm->xempty[i], 1);  // tcgen05.commit
-    }
-    for (int i = 0; i < kAStages; ++i) {
-      mbar_init(&sm->afull[i], 4);   // the 4 producer warps of the stage's group
-      mbar_init(&sm->aempty[i], 1);  // tcgen05.commit
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&sm->full[i], 1 + 4);  // TMA arrive.expect_tx + the 4 producer warps of the stage's group
+      mbar_init(&sm->empty[i], 1);     // tcgen05.commit
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm->acc_full[i], 1);
@@ -184,8 +183,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool adapter = ks == ks0 + wk.kps;
         if (!adapter) ++wit;
         if ((int)(it % kGroups) != group) continue;
-        const int as = it % kAStages;
-        const uint32_t aph = (it / kAStages) & 1;
+        const int as = it % kStages;
+        const uint32_t aph = (it / kStages) & 1;
         if (adapter) {
           // adapter stage: this row of the up map B[n, 0..r) twice, [B | B] in the first r columns of the A slot
           // (zeros after), against [T_hi | T_lo] of the down map
@@ -201,12 +200,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             r[j + 2] = v.z;
             r[j + 3] = v.w;
           }
-          if (!wait_or_abort(&sm->aempty[as], aph ^ 1, sm, err)) break;
+          if (!wait_or_abort(&sm->empty[as], aph ^ 1, sm, err)) break;
           const uint32_t ta = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(kAccColsT + as * 32);
           tmem_st32(ta, r);
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&sm->afull[as]);
+          if (lane == 0) mbar_arrive(&sm->full[as]);
           continue;
         }
         const int ws = (wit - 1) % kWStages;
@@ -239,11 +238,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           r[4 * c + 2] = d[2];
           r[4 * c + 3] = d[3];
         }
-        if (!wait_or_abort(&sm->aempty[as], aph ^ 1, sm, err)) break;  // the MMAs left this slot
+        if (!wait_or_abort(&sm->empty[as], aph ^ 1, sm, err)) break;  // the MMAs left this slot
         tmem_st32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(kAccColsT + as * 32), r);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm->afull[as]);
+        if (lane == 0) mbar_arrive(&sm->full[as]);
       }
       if (aborted(sm)) break;
     }
@@ -257,21 +256,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ks1 = ks0 + wk.kps + (lora_r > 0 && wk.split(u) == 0 ? 1 : 0);
         const int m0 = wk.m0(u);
         for (int ks = ks0; ks < ks1; ++ks, ++it) {
-          const int xs = it % kXStages;
-          if (!wait_or_abort(&sm->xempty[xs], ((it / kXStages) & 1) ^ 1, sm, err)) break;
+          const int xs = it % kStages;
+          if (!wait_or_abort(&sm->empty[xs], ((it / kStages) & 1) ^ 1, sm, err)) break;
           if (it == 0) NF4_STAMP(1);
-          mbar_expect_tx(&sm->xfull[xs], kBBytes);
+          mbar_expect_tx(&sm->full[xs], kBBytes);
           if (ks == ks0 + wk.kps) {  // adapter stage: the down map's [hi | lo | 0] rows, 64 wide
             pdl_wait();              // the down-map grid has finished and its writes are visible
-            tma_load_2d(b_smem0 + xs * kBBytes, &tmap, 0, m0, &sm->xfull[xs]);
+            tma_load_2d(b_smem0 + xs * kBBytes, &tmap, 0, m0, &sm->full[xs]);
           } else {
-            tma_load_2d(b_smem0 + xs * kBBytes, &xmap, ks * kTileK, m0, &sm->xfull[xs]);
+            tma_load_2d(b_smem0 + xs * kBBytes, &xmap, ks * kTileK, m0, &sm->full[xs]);
           }
         }
       }
       const uint32_t issued = it;  // drain the copies still in flight
-      for (uint32_t j = (issued > kXStages ? issued - kXStages : 0); j < issued; ++j)
-        mbar_wait_bounded(&sm->xfull[j % kXStages], (j / kXStages) & 1, err);
+      // (a stage's phase also needs the producers' arrivals: after an abort one timed-out wait is enough, the
+      // copies have long landed by then)
+      for (uint32_t j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+        if (!mbar_wait_bounded(&sm->full[j % kStages], (j / kStages) & 1, err)) break;
     }
   } else if (warp == kTmaWWarp) {
     // ------------------------------------------------ TMA: packed codes and scale chunks
@@ -309,21 +310,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         const int nst = wk.kps + (lora_r > 0 && wk.split(u) == 0 ? 1 : 0);  // + the adapter stage
         for (int j = 0; j < nst; ++j, ++it) {
-          const int as = it % kAStages, xs = it % kXStages;
-          if (!wait_or_abort(&sm->afull[as], (it / kAStages) & 1, sm, err) ||
-              !wait_or_abort(&sm->xfull[xs], (it / kXStages) & 1, sm, err)) {
+          const int st = it % kStages;
+          if (!wait_or_abort(&sm->full[st], (it / kStages) & 1, sm, err)) {
             ok = false;
             break;
           }
           tc_fence_after();
           if (it == 0) NF4_STAMP(2);
-          const uint32_t a_tm = tmem + (uint32_t)(kAccColsT + as * 32), b_addr = b_smem0 + xs * kBBytes;
+          const uint32_t a_tm = tmem + (uint32_t)(kAccColsT + st * 32), b_addr = b_smem0 + st * kBBytes;
           const int nkk = j < wk.kps ? kTileK / 16 : lora_r / 8;  // the adapter stage reduces over 2r only
 #pragma unroll
           for (int kk = 0; kk < kTileK / 16; ++kk)  // 16 bf16 per MMA along k: 8 TMEM columns, 32 smem bytes
             if (kk < nkk) tc_mma_ts(d_tmem, a_tm + kk * 8, smem_desc_sw128(b_addr + kk * 32), idesc, (j | kk) != 0);
-          tc_commit(&sm->aempty[as]);  // slots free once these MMAs have read them
-          tc_commit(&sm->xempty[xs]);
+          tc_commit(&sm->empty[st]);  // both tiles of the stage free once these MMAs have read them
         }
         if (!ok) break;
         NF4_STAMP(3);

@@ -132,9 +132,11 @@ __device__ __forceinline__ bool aborted(Sm* sm) {
   return *(volatile int*)&sm->abort != 0;
 }
 
-// bounded wait; on failure mark the CTA aborted so every role leaves its loop
+// bounded wait; on failure mark the CTA aborted so every role leaves its loop.  A phase that has already
+// completed returns at once (the abort word is read only when the thread would otherwise wait).
 template <class Sm>
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Sm* sm, unsigned* err) {
+  if (mbar_try_wait(bar, parity)) return true;
   if (aborted(sm)) return false;
   if (mbar_wait_bounded(bar, parity, err)) return true;
   *(volatile int*)&sm->abort = 1;
