@@ -41,16 +41,17 @@ namespace {
 using namespace umma;
 
 constexpr int kTileR = 64;                     // weight rows (reduction) per stage
-constexpr int kXStages = 4;                    // dY tile ring
-constexpr int kAStages = 3;                    // decoded Wc^T tile ring
-constexpr int kWStages = 6;                    // packed-code + scale ring
+// operand ring: stage s holds a dY tile (TMA) and a decoded Wc^T tile (producer warps) that fill and empty
+// together, one full and one empty barrier per stage for the single MMA-issuing thread
+constexpr int kStages = 4;
+constexpr int kWStages = 4;                    // packed-code + scale ring (4 + 4 stages: 223 KB of shared memory)
 constexpr int kBBytes = kTileM * kTileR * 2;   // 32 KB: dY tile (operand B)
 constexpr int kABytes = kTileR * kTileN * 2;   // 16 KB: decoded tile (operand A)
 constexpr int kWHalf = kTileR * 32;            // 2 KB: one level-1 block of codes per row
 constexpr int kWBytes = 2 * kWHalf;            // 4 KB: the stage's two blocks per row
 constexpr int kSBytes = kTileR * 16;           // 1 KB: 16-byte scale chunk per row
-constexpr int kRingBytes = kXStages * kBBytes + kAStages * kABytes + kWStages * (kWBytes + kSBytes);
-static_assert(kXStages * kBBytes >= split_stage_bytes(kTileM), "split reduction staging fits in the operand ring");
+constexpr int kRingBytes = kStages * (kBBytes + kABytes) + kWStages * (kWBytes + kSBytes);
+static_assert(kStages * kBBytes >= split_stage_bytes(kTileM), "split reduction staging fits in the operand ring");
 constexpr int kTmemCols = 2 * kAccCols;        // two accumulators
 constexpr int kThreads = 15 * 32;
 constexpr int kProdWarp0 = 4;
@@ -70,10 +71,8 @@ static_assert(kTileR / 8 * kKGroup == kABytes && 2 * kMnAtom == kKGroup, "A tile
 struct Smem {
   uint64_t wfull[kWStages];
   uint64_t wempty[kWStages];
-  uint64_t xfull[kXStages];
-  uint64_t xempty[kXStages];
-  uint64_t afull[kAStages];   // decoded tile written (producer warps)
-  uint64_t aempty[kAStages];  // decoded tile consumed by the MMAs (tcgen05.commit)
+  uint64_t full[kStages];   // dY tile landed (TMA) and decoded tile written (producer warps)
+  uint64_t empty[kStages];  // both consumed by the stage's MMAs (tcgen05.commit)
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint32_t tmem_base;
@@ -93,8 +92,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;  // 1024-aligned stage buffers (swizzle atoms)
   uint8_t* gbase = smem_raw + (base - raw);
   const uint32_t b_smem0 = base;
-  const uint32_t a_smem0 = b_smem0 + kXStages * kBBytes;
-  const uint32_t w_smem0 = a_smem0 + kAStages * kABytes;
+  const uint32_t a_smem0 = b_smem0 + kStages * kBBytes;
+  const uint32_t w_smem0 = a_smem0 + kStages * kABytes;
   const uint32_t s_smem0 = w_smem0 + kWStages * kWBytes;
   uint8_t* a_gen0 = gbase + (a_smem0 - base);
   const uint8_t* w_gen0 = gbase + (w_smem0 - base);
@@ -115,13 +114,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm->wfull[i], 1);
       mbar_init(&sm->wempty[i], 4);
     }
-    for (int i = 0; i < kXStages; ++i) {
-      mbar_init(&sm->xfull[i], 1);
-      mbar_init(&sm->xempty[i], 1);
-    }
-    for (int i = 0; i < kAStages; ++i) {
-      mbar_init(&sm->afull[i], 4);
-      mbar_init(&sm->aempty[i], 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&sm->full[i], 1 + 4);  // TMA arrive.expect_tx + the 4 producer warps of the stage's group
+      mbar_init(&sm->empty[i], 1);     // tcgen05.commit
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm->acc_full[i], 1);
@@ -161,8 +156,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int ks0 = wk.split(u) * wk.kps;
       for (int ks = ks0; ks < ks0 + wk.kps; ++ks, ++it) {
         if ((int)(it & 1) != group) continue;
-        const int ws = it % kWStages, as = it % kAStages;
-        const uint32_t wph = (it / kWStages) & 1, aph = (it / kAStages) & 1;
+        const int ws = it % kWStages, as = it % kStages;
+        const uint32_t wph = (it / kWStages) & 1, aph = (it / kStages) & 1;
         if (!wait_or_abort(&sm->wfull[ws], wph, sm, err)) break;
         const uint4* wsrc = reinterpret_cast<const uint4*>(w_gen0 + ws * kWBytes + h * kWHalf + r * 32);
         const uint4 w0 = wsrc[0], w1 = wsrc[1];
@@ -191,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           q[4 * c + 2] = d[2];
           q[4 * c + 3] = d[3];
         }
-        if (!wait_or_abort(&sm->aempty[as], aph ^ 1, sm, err)) break;  // the MMAs left this slot
+        if (!wait_or_abort(&sm->empty[as], aph ^ 1, sm, err)) break;  // the MMAs left this slot
         uint8_t* arow = a_gen0 + as * kABytes + a_row;
 #pragma unroll
         for (int c = 0; c < 8; ++c)
@@ -199,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               make_uint4(q[4 * c], q[4 * c + 1], q[4 * c + 2], q[4 * c + 3]);
         fence_proxy_async_smem();  // generic-proxy writes, read by the tensor cores (async proxy)
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm->afull[as]);
+        if (lane == 0) mbar_arrive(&sm->full[as]);
       }
       if (aborted(sm)) break;
     }
@@ -212,15 +207,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ks0 = wk.split(u) * wk.kps;
         const int m0 = wk.m0(u);
         for (int ks = ks0; ks < ks0 + wk.kps; ++ks, ++it) {
-          const int xs = it % kXStages;
-          if (!wait_or_abort(&sm->xempty[xs], ((it / kXStages) & 1) ^ 1, sm, err)) break;
-          mbar_expect_tx(&sm->xfull[xs], kBBytes);
-          tma_load_2d(b_smem0 + xs * kBBytes, &ymap, ks * kTileR, m0, &sm->xfull[xs]);
+          const int xs = it % kStages;
+          if (!wait_or_abort(&sm->empty[xs], ((it / kStages) & 1) ^ 1, sm, err)) break;
+          mbar_expect_tx(&sm->full[xs], kBBytes);
+          tma_load_2d(b_smem0 + xs * kBBytes, &ymap, ks * kTileR, m0, &sm->full[xs]);
         }
       }
       const uint32_t issued = it;  // drain the copies still in flight
-      for (uint32_t j = (issued > kXStages ? issued - kXStages : 0); j < issued; ++j)
-        mbar_wait_bounded(&sm->xfull[j % kXStages], (j / kXStages) & 1, err);
+      // (a stage's phase also needs the producers' arrivals: after an abort one timed-out wait is enough, the
+      // copies have long landed by then)
+      for (uint32_t j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+        if (!mbar_wait_bounded(&sm->full[j % kStages], (j / kStages) & 1, err)) break;
     }
   } else if (warp == kTmaWWarp) {
     // ------------------------------------------------ TMA: packed codes and scale chunks
@@ -259,20 +256,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d_tmem = tmem + acc * kAccCols;
         bool ok = true;
         for (int j = 0; j < wk.kps; ++j, ++it) {
-          const int as = it % kAStages, xs = it % kXStages;
-          if (!wait_or_abort(&sm->afull[as], (it / kAStages) & 1, sm, err) ||
-              !wait_or_abort(&sm->xfull[xs], (it / kXStages) & 1, sm, err)) {
+          const int st = it % kStages;
+          if (!wait_or_abort(&sm->full[st], (it / kStages) & 1, sm, err)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = a_smem0 + as * kABytes, b_addr = b_smem0 + xs * kBBytes;
+          const uint32_t a_addr = a_smem0 + st * kABytes, b_addr = b_smem0 + st * kBBytes;
 #pragma unroll
           for (int kk = 0; kk < kTileR / 16; ++kk)  // 16 weight rows per MMA: two 8-row groups, 32 bytes of dY
             tc_mma_ss(d_tmem, smem_desc_mn_sw128(a_addr + kk * 2 * kKGroup, kMnAtom, kKGroup),
                       smem_desc_sw128(b_addr + kk * 32), idesc, (j | kk) != 0);
-          tc_commit(&sm->aempty[as]);
-          tc_commit(&sm->xempty[xs]);
+          tc_commit(&sm->empty[st]);  // both tiles of the stage free once these MMAs have read them
         }
         if (!ok) break;
         tc_commit(&sm->acc_full[acc]);
