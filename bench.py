@@ -739,8 +739,8 @@ def model_config(args, nf4, synth, dev, time_calls, peaks):
 # kernels; gemm_lora: the down map and the GEMM), from the captures summarised in profiles/ (ncu flushes the caches
 # before each replayed launch, so these are cold-read figures); an entry is removed whenever its kernel changes
 # after the capture
-TRAFFIC = {"quantize": 33579264, "double_quant": 2136576, "dequantize": 18662912, "gemv": 8682496, "gemm": None,
-           "gemm_dx": None, "gemm_lora": None, "gemv_grouped": 13010432}
+TRAFFIC = {"quantize": 33579264, "double_quant": 2136576, "dequantize": 8688896, "gemv": 8682496, "gemm": 10823424,
+           "gemm_dx": 10819328, "gemm_lora": 13227264, "gemv_grouped": 13010432}
 
 
 def oracle_table(args):
