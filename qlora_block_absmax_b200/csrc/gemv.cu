@@ -56,7 +56,10 @@ struct GemvGroup {
   int tile_end[kMaxGroup];
   int count;
 };
-constexpr int kPairTableBytes = 256 * 32 * 8;  // fp32 code pairs, one copy per bank
+// fp32 code pairs: entry v of copy c at 256 v + 8 c, 16 copies (the first 128 bytes of every 256-byte row; a
+// byte permute of the code with the lane's offset is the address).  A 64-bit shared load is served in two
+// half-warp phases, so lane l reading copy l % 16 keeps each phase free of bank conflicts.
+constexpr int kPairTableBytes = 256 * 32 * 8;
 
 __constant__ float c_code_gemv[2][16] = {NF4_CODE_INIT, FP4_CODE_INIT};  // by code book: NF4, FP4
 
@@ -107,7 +110,7 @@ __global__ void __launch_bounds__(kWarps * 32, NT >= 4 ? 1 : 2)
     gemv_kernel(GemvGroup grp, int64_t cols, const __nv_bfloat16* __restrict__ x, int batch) {
   __shared__ float unit_lut[kDQ ? 256 : 1];
   __shared__ float red[kWarps][16][8 * NT];
-  extern __shared__ __align__(16) uint8_t pair_table[];  // entry v of lane l at 256 v + 8 l
+  extern __shared__ __align__(16) uint8_t pair_table[];  // entry v of lane l at 256 v + 8 (l % 16)
   pdl_launch_dependents();
   // this CTA's weight of the group (every index below is a compile-time constant)
   const uint8_t* __restrict__ packed = grp.packed[0];
@@ -133,10 +136,11 @@ __global__ void __launch_bounds__(kWarps * 32, NT >= 4 ? 1 : 2)
     if (threadIdx.x < 16) code_s[threadIdx.x] = c_code_gemv[kBook][threadIdx.x];
     __syncthreads();
 #pragma unroll
-    for (int k = 0; k < kPairTableBytes / 16 / (kWarps * 32); ++k) {
-      const int idx = threadIdx.x + k * kWarps * 32;  // 16-byte pieces: two lanes' copies of one entry
-      const float hi = code_s[idx >> 8], lo = code_s[(idx >> 4) & 15];
-      *reinterpret_cast<float4*>(pair_table + idx * 16) = make_float4(hi, lo, hi, lo);
+    for (int k = 0; k < 256 * 8 / (kWarps * 32); ++k) {
+      const int idx = threadIdx.x + k * kWarps * 32;  // 16-byte pieces: copies 2i, 2i + 1 of one entry
+      const int v = idx >> 3, i = idx & 7;
+      const float hi = code_s[v >> 4], lo = code_s[v & 15];
+      *reinterpret_cast<float4*>(pair_table + v * 256 + i * 16) = make_float4(hi, lo, hi, lo);
     }
   }
   __syncthreads();
@@ -161,7 +165,7 @@ __global__ void __launch_bounds__(kWarps * 32, NT >= 4 ? 1 : 2)
   for (int nt = 0; nt < NT; ++nt) xrow[nt] = (8 * nt + g < batch) ? x + (int64_t)(8 * nt + g) * cols : nullptr;
 
   const DecodeMul dm = decode_mul();
-  const uint32_t lane8 = (uint32_t)(lane * 8);
+  const uint32_t lane8 = (uint32_t)((lane & 15) * 8);
   StepData cur, nxt;
   int64_t st = warp;
   if (st < nsteps) load_step<kDQ>(cur, packed, s, row0, cols, st * 4 + t, st * 4 + t < nblk);
