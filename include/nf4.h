@@ -155,6 +155,26 @@ NF4_API nf4_status nf4_double_quant(const float *absmax, int64_t nb, int32_t dq_
                             size_t workspace_bytes, nf4_stream_t stream);
 NF4_API size_t nf4_double_quant_workspace_bytes(int64_t nb);
 
+/* nf4_double_quant of up to NF4_DQ_MANY_MAX absmax arrays in two launches (a
+ * model's weights quantized one after another, as [bnb-tut] "4-bit Loading with
+ * NF4" loads every linear layer of an 8B model), each with its own mean: array
+ * i gets exactly the q, scale and mean that nf4_double_quant gives it.
+ *   absmax, nb, q_out, scale_out, mean_out   host arrays of `count` entries: the
+ *               device pointers and sizes of each array, as in nf4_double_quant
+ *   count       1 .. NF4_DQ_MANY_MAX
+ *   workspace   device scratch of nf4_double_quant_many_workspace_bytes(count)
+ *               bytes, 16-byte aligned; zero-filled before its first use, left
+ *               ready by every call that completes (as for nf4_double_quant)
+ * An array with nb == 0 is skipped (its mean_out stays unset).  Every array is
+ * checked before anything launches; the first error is returned and nothing
+ * runs.  Arrays and outputs must not overlap one another. */
+#define NF4_DQ_MANY_MAX 256
+NF4_API nf4_status nf4_double_quant_many(const float *const *absmax, const int64_t *nb, int32_t count,
+                                         int32_t dq_blocksize, int32_t dq_code, uint8_t *const *q_out,
+                                         float *const *scale_out, float *const *mean_out, void *workspace,
+                                         size_t workspace_bytes, nf4_stream_t stream);
+NF4_API size_t nf4_double_quant_many_workspace_bytes(int32_t count);
+
 /* nf4_double_quant without a caller-provided workspace, for callers that
  * cannot allocate device memory: code that runs under a fixed memory budget
  * set at start-up, or inside a host framework that owns the device allocator

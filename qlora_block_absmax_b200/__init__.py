@@ -24,6 +24,7 @@ from ._lib import NF4_BF16, NF4_DQ_E4M3, NF4_DQ_INT8, NF4_F32, NF4_QUANT_FP4, NF
 
 __all__ = ["QuantizedWeight", "quantize", "double_quant", "quantize_weight", "dequantize", "gemv", "gemm",
            "storage_bytes", "gemm_workspace_bytes", "gemm_dx", "gemm_dx_workspace_bytes", "gemm_lora", "gemv_grouped", "gemv_stream",
+           "double_quant_many",
            "gemm_lora_workspace_bytes", "code_table", "check_device_error", "kernel_launches", "NF4Error", "library_path"]
 
 BLOCKSIZE = 64
@@ -121,6 +122,35 @@ def double_quant(absmax: torch.Tensor, code: str = "e4m3", dq_blocksize: int = D
                               _ptr(workspace), workspace.numel(), _stream(stream))
     _lib.check(st, "nf4_double_quant")
     return q, scale, mean
+
+
+def double_quant_many(absmaxes, code: str = "e4m3", dq_blocksize: int = DQ_BLOCKSIZE, outs=None,
+                      workspace: Optional[torch.Tensor] = None, stream=None) -> list:
+    """double_quant of up to 256 fp32 absmax arrays (each with its own mean) in two launches.
+    Returns [(q, scale, mean)] per array, the same values double_quant gives each one."""
+    absmaxes = list(absmaxes)
+    if not absmaxes:
+        raise ValueError("double_quant_many takes at least one array")
+    lib = _lib.load()
+    for a in absmaxes:
+        _need_cuda(a, "absmax")
+    if outs is None:
+        outs = [(torch.empty(a.numel(), dtype=torch.uint8, device=a.device),
+                 torch.empty((a.numel() + dq_blocksize - 1) // dq_blocksize, dtype=torch.float32, device=a.device),
+                 torch.empty(1, dtype=torch.float32, device=a.device)) for a in absmaxes]
+    n = len(absmaxes)
+    ws_bytes = lib.nf4_double_quant_many_workspace_bytes(n)
+    if workspace is None:  # a fresh zeroed buffer (a caller's own buffer is zeroed once and reused)
+        workspace = torch.zeros(max(ws_bytes, 1), dtype=torch.uint8, device=absmaxes[0].device)
+    ap = (ctypes.c_void_p * n)(*[_ptr(a) for a in absmaxes])
+    nb = (ctypes.c_int64 * n)(*[a.numel() for a in absmaxes])
+    qp = (ctypes.c_void_p * n)(*[_ptr(o[0]) for o in outs])
+    sp = (ctypes.c_void_p * n)(*[_ptr(o[1]) for o in outs])
+    mp = (ctypes.c_void_p * n)(*[_ptr(o[2]) for o in outs])
+    st = lib.nf4_double_quant_many(ap, nb, n, dq_blocksize, _DQ_CODES[code], qp, sp, mp, _ptr(workspace),
+                                   workspace.numel(), _stream(stream))
+    _lib.check(st, "nf4_double_quant_many")
+    return outs
 
 
 def quantize_weight(w: torch.Tensor, use_double_quant: bool = True, code: str = "e4m3",

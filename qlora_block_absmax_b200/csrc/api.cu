@@ -173,6 +173,55 @@ nf4_status nf4_double_quant(const float* absmax, int64_t nb, int32_t dq_blocksiz
                                             d.error_word, reinterpret_cast<cudaStream_t>(stream), d.num_sms));
 }
 
+static_assert(NF4_DQ_MANY_MAX == nf4::kDqManyMax, "array limit");
+
+size_t nf4_double_quant_many_workspace_bytes(int32_t count) {
+  return count < 1 || count > NF4_DQ_MANY_MAX ? 0 : (size_t)count * nf4::kDqManyRecord;
+}
+
+nf4_status nf4_double_quant_many(const float* const* absmax, const int64_t* nb, int32_t count, int32_t dq_blocksize,
+                                 int32_t dq_code, uint8_t* const* q_out, float* const* scale_out,
+                                 float* const* mean_out, void* workspace, size_t workspace_bytes,
+                                 nf4_stream_t stream) {
+  if (count < 1 || count > NF4_DQ_MANY_MAX) return NF4_ERR_INVALID_ARG;
+  if (absmax == nullptr || nb == nullptr || q_out == nullptr || scale_out == nullptr || mean_out == nullptr)
+    return NF4_ERR_INVALID_ARG;
+  if (dq_code != NF4_DQ_E4M3 && dq_code != NF4_DQ_INT8) return NF4_ERR_INVALID_ARG;
+  if (dq_blocksize != nf4::kDqBlock) return NF4_ERR_UNSUPPORTED;
+  if (workspace == nullptr || workspace_bytes < nf4_double_quant_many_workspace_bytes(count))
+    return NF4_ERR_INVALID_ARG;
+  if (!aligned(workspace, 16)) return NF4_ERR_MISALIGNED;
+  // every array is checked before anything is launched; empty ones are left out (their mean_out stays unset)
+  static thread_local nf4::DqManyParams p;  // 14 KB: kept off the stack
+  p.count = 0;
+  p.total = 0;
+  p.groups = 0;
+  for (int32_t i = 0; i < count; ++i) {
+    if (nb[i] < 0 || nb[i] > NF4_DQ_MAX_NB) return NF4_ERR_INVALID_ARG;
+    if (nb[i] == 0) continue;
+    if (absmax[i] == nullptr || q_out[i] == nullptr || scale_out[i] == nullptr || mean_out[i] == nullptr)
+      return NF4_ERR_INVALID_ARG;
+    if (!aligned(absmax[i], 16) || !aligned(q_out[i], 16) || !aligned(scale_out[i], 4) || !aligned(mean_out[i], 4))
+      return NF4_ERR_MISALIGNED;
+    nf4::DqItem& it = p.item[p.count++];
+    it.a = absmax[i];
+    it.q = q_out[i];
+    it.scale = scale_out[i];
+    it.mean = mean_out[i];
+    it.nb = nb[i];
+    it.e0 = p.total;
+    it.g0 = p.groups;
+    p.total += nb[i];
+    p.groups += (nb[i] + nf4::kDqBlock - 1) / nf4::kDqBlock;
+  }
+  if (p.count == 0) return NF4_OK;
+  DeviceInfo d;
+  nf4_status st = device_info(&d);
+  if (st != NF4_OK) return st;
+  return from_cuda(nf4::launch_double_quant_many(p, dq_code, workspace, reinterpret_cast<cudaStream_t>(stream),
+                                                 d.num_sms));
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------

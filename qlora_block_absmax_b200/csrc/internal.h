@@ -52,6 +52,27 @@ cudaError_t launch_double_quant(const float* absmax, int64_t nb, int dq_code, ui
                                 int num_sms);
 constexpr size_t kDoubleQuantWorkspace = 256;
 
+// double quantization of several absmax arrays in two launches (one exact-sum record per tensor in the workspace)
+constexpr int kDqManyMax = 256;
+constexpr size_t kDqManyRecord = 128;  // workspace bytes per tensor
+struct DqItem {
+  const float* a;  // absmax [nb], 16-byte aligned
+  uint8_t* q;      // codes [nb]
+  float* scale;    // [ceil(nb / 256)]
+  float* mean;     // [1]
+  int64_t nb;      // >= 1
+  int64_t e0;      // first element of this array in the concatenation of all of them
+  int64_t g0;      // first 256-block likewise
+};
+struct DqManyParams {
+  DqItem item[kDqManyMax];
+  int32_t count;   // >= 1
+  int64_t total;   // sum of nb
+  int64_t groups;  // sum of ceil(nb / 256)
+};
+cudaError_t launch_double_quant_many(const DqManyParams& p, int dq_code, void* workspace, cudaStream_t stream,
+                                     int num_sms);
+
 // blocksize 32, 64, 128 or 256
 cudaError_t launch_dequantize(const uint8_t* packed, const Scales& s, int64_t n, int blocksize, void* out,
                               bool out_bf16, cudaStream_t stream, int num_sms);

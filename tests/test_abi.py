@@ -80,6 +80,28 @@ def test_host_validation_before_cuda(lib):
     assert lib.nf4_double_quant_noalloc(0x1000, too_many, 256, 0, 0x2000, 0x3000, 0x4000, s) == \
         E["NF4_ERR_INVALID_ARG"]
     assert lib.nf4_double_quant_workspace_bytes(1 << 20) >= 128
+    # the many-array call checks every array before it touches the device
+    P = ctypes.c_void_p
+    one = lambda *v: (P * len(v))(*v)  # noqa: E731
+    nb = lambda *v: (ctypes.c_int64 * len(v))(*v)  # noqa: E731
+    dqm = lib.nf4_double_quant_many
+    assert dqm(one(0x1000), nb(10), 0, 256, 0, one(0x2000), one(0x3000), one(0x4000), 0x5000, 4096, s) == \
+        E["NF4_ERR_INVALID_ARG"]
+    assert dqm(one(0x1000), nb(10), 257, 256, 0, one(0x2000), one(0x3000), one(0x4000), 0x5000, 1 << 20, s) == \
+        E["NF4_ERR_INVALID_ARG"]
+    assert dqm(one(0x1000), nb(10), 1, 128, 0, one(0x2000), one(0x3000), one(0x4000), 0x5000, 4096, s) == \
+        E["NF4_ERR_UNSUPPORTED"]
+    assert dqm(one(0x1000), nb(10), 1, 256, 7, one(0x2000), one(0x3000), one(0x4000), 0x5000, 4096, s) == \
+        E["NF4_ERR_INVALID_ARG"]
+    assert dqm(one(0x1000), nb(10), 1, 256, 0, one(0x2000), one(0x3000), one(0x4000), 0x5000, 16, s) == \
+        E["NF4_ERR_INVALID_ARG"]  # workspace smaller than one record
+    assert dqm(one(0x1000, 0x1004), nb(10, 10), 2, 256, 0, one(0x2000, 0x2100), one(0x3000, 0x3100),
+               one(0x4000, 0x4100), 0x5000, 4096, s) == E["NF4_ERR_MISALIGNED"]  # second array misaligned
+    assert dqm(one(0x1000), nb(-1), 1, 256, 0, one(0x2000), one(0x3000), one(0x4000), 0x5000, 4096, s) == \
+        E["NF4_ERR_INVALID_ARG"]
+    assert dqm(one(0x1000), nb(0), 1, 256, 0, one(0x2000), one(0x3000), one(0x4000), 0x5000, 4096, s) == E["NF4_OK"]
+    assert lib.nf4_double_quant_many_workspace_bytes(3) == 3 * 128
+    assert lib.nf4_double_quant_many_workspace_bytes(0) == 0 and lib.nf4_double_quant_many_workspace_bytes(257) == 0
     # weight descriptor checks
     w = weight(bs=48)
     assert lib.nf4_dequantize(ctypes.byref(w), 0x9000, 0, s) == E["NF4_ERR_UNSUPPORTED"]
