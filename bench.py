@@ -700,25 +700,27 @@ def model_config(args, nf4, synth, dev, time_calls, peaks):
     absmaxes = [b[1] for b in bufs]
     dq_outs = [b[2:5] for b in bufs]
 
+    flat = [s.reshape(-1) for s in srcs]
+    q_outs = [b[0:2] for b in bufs]
+
     def quantize_pass():
-        # every weight quantized in turn, then the double quant of all 224 absmax arrays in one call
-        for s, (packed, absmax, _, _, _) in zip(srcs, bufs):
-            nf4.quantize(s, out=(packed, absmax))
+        # all 224 weights quantized in one call, then the double quant of all 224 absmax arrays in one call
+        nf4.quantize_many(flat, outs=q_outs)
         nf4.double_quant_many(absmaxes, "e4m3", outs=dq_outs, workspace=dq_ws)
 
     reps = 3
     t_quant = time_calls([quantize_pass], n=reps) * 1e-3
-    launches = (len(shapes) + 2) * reps
+    launches = 3 * reps
     mw = model_work(1)
     out = {"what": "32 layers x (q 4096x4096, k/v 1024x4096, o 4096x4096, gate/up 14336x4096, down 4096x14336) "
                    "bf16 ~N(0,0.02) (device generator, seed 2000 + 7 layer + proj), 6,979,321,856 weights; "
-                   f"quantize of all 224 (one launch each), then E4M3 double quant of all 224 absmax arrays in one "
-                   f"nf4_double_quant_many call (2 launches; 226 per pass, {reps} passes timed); then "
+                   f"quantize of all 224 in one nf4_quantize_many call, then E4M3 double quant of all 224 absmax "
+                   f"arrays in one nf4_double_quant_many call (3 launches per pass, {reps} passes timed); then "
                    "one decode GEMV pass over all 224 weights as one nf4_gemv_stream launch, inputs for q/k/v, o, "
                    "gate/up and down of every layer ~N(0,1) (seeds 3300 + 10 b + j)",
            "quantize_pass": {"ms": round(t_quant * 1e3, 4), "gelem_s": round(mw["quantize_pass"]["elems"] / t_quant / 1e9, 1),
                              "roofline": roofline_entry(mw["quantize_pass"], t_quant, peaks, "hbm")}}
-    del srcs
+    del srcs, flat
     torch.cuda.empty_cache()
     for b in GEMV_BATCHES:
         acts = [synth.activations_device((b, c), 3300 + 10 * b + j, device=dev)

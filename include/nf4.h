@@ -129,6 +129,21 @@ NF4_API nf4_status nf4_quantize_typed(const void *src, int32_t src_dtype, int64_
                                       int32_t quant_type, uint8_t *packed_out, float *absmax_out,
                                       nf4_stream_t stream);
 
+/* nf4_quantize_typed of up to NF4_QUANT_MANY_MAX tensors of one source dtype,
+ * block size and code book in one launch (a model's linear layers quantized
+ * as it loads, [bnb-tut] "4-bit Loading with NF4"): tensor i gets exactly the
+ * packed codes and absmax that nf4_quantize_typed gives it.
+ *   src, n, packed_out, absmax_out   host arrays of `count` entries: each
+ *               tensor's device pointers and element count, as in nf4_quantize
+ *   count       1 .. NF4_QUANT_MANY_MAX
+ * A tensor with n == 0 is skipped.  Every tensor is checked before anything
+ * launches; the first error is returned and nothing runs.  Tensors and
+ * outputs must not overlap one another. */
+#define NF4_QUANT_MANY_MAX 256
+NF4_API nf4_status nf4_quantize_many(const void *const *src, const int64_t *n, int32_t count, int32_t src_dtype,
+                                     int32_t blocksize, int32_t quant_type, uint8_t *const *packed_out,
+                                     float *const *absmax_out, nf4_stream_t stream);
+
 /* Double quantization of the fp32 absmax array, [bnb-tut] "How NF4 Works"
  * (scale constants quantized from float32 to float8) and [bnb-tools] "Double
  * quantization".  mu = fp32(fp64(exact sum of absmax) / nb) (one per tensor);

@@ -24,7 +24,7 @@ from ._lib import NF4_BF16, NF4_DQ_E4M3, NF4_DQ_INT8, NF4_F32, NF4_QUANT_FP4, NF
 
 __all__ = ["QuantizedWeight", "quantize", "double_quant", "quantize_weight", "dequantize", "gemv", "gemm",
            "storage_bytes", "gemm_workspace_bytes", "gemm_dx", "gemm_dx_workspace_bytes", "gemm_lora", "gemv_grouped", "gemv_stream",
-           "double_quant_many",
+           "double_quant_many", "quantize_many",
            "gemm_lora_workspace_bytes", "code_table", "check_device_error", "kernel_launches", "NF4Error", "library_path"]
 
 BLOCKSIZE = 64
@@ -100,6 +100,32 @@ def quantize(w: torch.Tensor, blocksize: int = BLOCKSIZE, out=None, stream=None,
                                         _QUANT_TYPES[quant_type], _ptr(packed), _ptr(absmax), _stream(stream))
     _lib.check(st, "nf4_quantize_typed")
     return packed, absmax
+
+
+def quantize_many(ws, blocksize: int = BLOCKSIZE, outs=None, stream=None, quant_type: str = "nf4") -> list:
+    """quantize of up to 256 flattened tensors of one dtype (fp32 or bf16) in one launch.
+    Returns [(packed, absmax)] per tensor, the same values quantize gives each one."""
+    ws = list(ws)
+    if not ws:
+        raise ValueError("quantize_many takes at least one tensor")
+    dt = ws[0].dtype
+    for w in ws:
+        _need_cuda(w, "w")
+        if w.dtype != dt or dt not in (torch.float32, torch.bfloat16):
+            raise TypeError("quantize_many takes tensors of one dtype, float32 or bfloat16")
+    if outs is None:
+        outs = [(torch.empty((w.numel() + 1) // 2, dtype=torch.uint8, device=w.device),
+                 torch.empty((w.numel() + blocksize - 1) // blocksize, dtype=torch.float32, device=w.device))
+                for w in ws]
+    k = len(ws)
+    sp = (ctypes.c_void_p * k)(*[_ptr(w) for w in ws])
+    ns = (ctypes.c_int64 * k)(*[w.numel() for w in ws])
+    pp = (ctypes.c_void_p * k)(*[_ptr(o[0]) for o in outs])
+    ap = (ctypes.c_void_p * k)(*[_ptr(o[1]) for o in outs])
+    st = _lib.load().nf4_quantize_many(sp, ns, k, NF4_BF16 if dt == torch.bfloat16 else NF4_F32, blocksize,
+                                       _QUANT_TYPES[quant_type], pp, ap, _stream(stream))
+    _lib.check(st, "nf4_quantize_many")
+    return outs
 
 
 def double_quant(absmax: torch.Tensor, code: str = "e4m3", dq_blocksize: int = DQ_BLOCKSIZE, out=None,

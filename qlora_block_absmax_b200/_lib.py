@@ -43,6 +43,8 @@ SIGNATURES = {
     "nf4_double_quant": (ctypes.c_int, [P, I64, I32, I32, P, P, P, P, SZ, P]),
     "nf4_double_quant_workspace_bytes": (SZ, [I64]),
     "nf4_double_quant_noalloc": (ctypes.c_int, [P, I64, I32, I32, P, P, P, P]),
+    "nf4_quantize_many": (ctypes.c_int, [ctypes.POINTER(P), ctypes.POINTER(I64), I32, I32, I32, I32, ctypes.POINTER(P),
+                                         ctypes.POINTER(P), P]),
     "nf4_double_quant_many": (ctypes.c_int, [ctypes.POINTER(P), ctypes.POINTER(I64), I32, I32, I32, ctypes.POINTER(P),
                                              ctypes.POINTER(P), ctypes.POINTER(P), P, SZ, P]),
     "nf4_double_quant_many_workspace_bytes": (SZ, [I32]),

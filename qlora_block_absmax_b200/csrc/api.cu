@@ -153,6 +153,39 @@ nf4_status nf4_quantize_typed(const void* src, int32_t src_dtype, int64_t n, int
                                         reinterpret_cast<cudaStream_t>(stream), d.num_sms));
 }
 
+static_assert(NF4_QUANT_MANY_MAX == nf4::kQuantManyMax, "array limit");
+
+nf4_status nf4_quantize_many(const void* const* src, const int64_t* n, int32_t count, int32_t src_dtype,
+                             int32_t blocksize, int32_t quant_type, uint8_t* const* packed_out,
+                             float* const* absmax_out, nf4_stream_t stream) {
+  if (count < 1 || count > NF4_QUANT_MANY_MAX) return NF4_ERR_INVALID_ARG;
+  if (src == nullptr || n == nullptr || packed_out == nullptr || absmax_out == nullptr) return NF4_ERR_INVALID_ARG;
+  if (quant_type != NF4_QUANT_NF4 && quant_type != NF4_QUANT_FP4) return NF4_ERR_INVALID_ARG;
+  if (src_dtype != NF4_F32 && src_dtype != NF4_BF16) return NF4_ERR_INVALID_ARG;
+  if (!level1_blocksize(blocksize)) return NF4_ERR_UNSUPPORTED;
+  // every tensor is checked before anything is launched; empty ones are left out
+  static thread_local nf4::QuantManyParams p;  // 10 KB: kept off the stack
+  p.count = 0;
+  for (int32_t i = 0; i < count; ++i) {
+    if (n[i] < 0) return NF4_ERR_INVALID_ARG;
+    if (n[i] == 0) continue;
+    if (src[i] == nullptr || packed_out[i] == nullptr || absmax_out[i] == nullptr) return NF4_ERR_INVALID_ARG;
+    if (!aligned(src[i], 16) || !aligned(packed_out[i], 16) || !aligned(absmax_out[i], 4))
+      return NF4_ERR_MISALIGNED;
+    nf4::QuantItem& it = p.item[p.count++];
+    it.src = src[i];
+    it.packed = packed_out[i];
+    it.absmax = absmax_out[i];
+    it.n = n[i];
+  }
+  if (p.count == 0) return NF4_OK;
+  DeviceInfo d;
+  nf4_status st = device_info(&d);
+  if (st != NF4_OK) return st;
+  return from_cuda(nf4::launch_quantize_many(p, src_dtype == NF4_BF16, blocksize, quant_type,
+                                             reinterpret_cast<cudaStream_t>(stream), d.num_sms));
+}
+
 nf4_status nf4_double_quant(const float* absmax, int64_t nb, int32_t dq_blocksize, int32_t dq_code, uint8_t* q_out,
                             float* scale_out, float* mean_out, void* workspace, size_t workspace_bytes,
                             nf4_stream_t stream) {

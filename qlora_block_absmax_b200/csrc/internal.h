@@ -46,6 +46,23 @@ struct Scales {
 cudaError_t launch_quantize(const void* src, bool bf16, int64_t n, int blocksize, uint8_t* packed, float* absmax,
                             int book, cudaStream_t stream, int num_sms);
 
+// several tensors of one dtype, block size and code book in one launch (w0 and iters are filled by the launcher)
+constexpr int kQuantManyMax = 256;
+struct QuantItem {
+  const void* src;  // n elements, 16-byte aligned
+  uint8_t* packed;  // ceil(n / 2)
+  float* absmax;    // ceil(n / blocksize)
+  int64_t n;        // >= 1
+  int64_t w0;       // first warp iteration of this tensor in the launch's sequence
+};
+struct QuantManyParams {
+  QuantItem item[kQuantManyMax];
+  int32_t count;  // >= 1
+  int64_t iters;  // warp iterations of all tensors
+};
+cudaError_t launch_quantize_many(QuantManyParams& p, bool bf16, int blocksize, int book, cudaStream_t stream,
+                                 int num_sms);
+
 // workspace: zero before its first use, left ready by every completed call; `clear` zeroes it first
 cudaError_t launch_double_quant(const float* absmax, int64_t nb, int dq_code, uint8_t* q, float* scale,
                                 float* mean, void* workspace, bool clear, unsigned* err, cudaStream_t stream,

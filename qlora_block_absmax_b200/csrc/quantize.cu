@@ -114,6 +114,102 @@ __device__ __forceinline__ float load1(const void* src, int64_t i) {
   return static_cast<const float*>(src)[i];
 }
 
+// One warp iteration over the 32 / kL blocks from block wb of one tensor: lane (block wb + lane / kL, part
+// lane % kL) loads its 16 consecutive elements (fetch, one iteration ahead) and codes them (code_slice).
+template <bool kBF16>
+using Raw = uint4[kBF16 ? 2 : 4];
+
+template <bool kBF16, int kL>
+__device__ __forceinline__ void fetch(const void* __restrict__ src, int64_t nfull, int64_t wb, int lane,
+                                      Raw<kBF16>& raw) {
+  constexpr int kB = 16 * kL;
+  const int64_t b = wb + lane / kL;
+  if (b < nfull) {
+    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(src) +
+                                                    (b * kB + (lane & (kL - 1)) * 16) * (kBF16 ? 2 : 4));
+#pragma unroll
+    for (int i = 0; i < (kBF16 ? 2 : 4); ++i) raw[i] = __ldcs(p + i);
+  }
+}
+
+template <bool kBF16, bool kFp4, int kL>
+__device__ __forceinline__ void code_slice(uint32_t entry, int lane, int64_t wb, const void* __restrict__ src,
+                                           int64_t n, int64_t nfull, int64_t nblocks, uint8_t* __restrict__ packed,
+                                           float* __restrict__ absmax, const Raw<kBF16>& cur) {
+  constexpr int kB = 16 * kL;
+  const int sub = lane & (kL - 1);  // which 16 of the block
+  const int64_t b = wb + lane / kL;
+  const bool live = b < nblocks;
+  const int64_t first = b * kB + sub * 16;
+  float w[16];
+  if (live && b < nfull) {
+    if (kBF16) {
+      const uint32_t u[8] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w, cur[1].x, cur[1].y, cur[1].z, cur[1].w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        w[2 * i] = bf16_lo_to_f32(u[i]);
+        w[2 * i + 1] = bf16_hi_to_f32(u[i]);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 v = cur[(kBF16 ? 0 : i)];
+        w[4 * i] = __uint_as_float(v.x);
+        w[4 * i + 1] = __uint_as_float(v.y);
+        w[4 * i + 2] = __uint_as_float(v.z);
+        w[4 * i + 3] = __uint_as_float(v.w);
+      }
+    }
+  } else {  // short last block (or no block): missing elements read as 0
+#pragma unroll
+    for (int i = 0; i < 16; ++i) w[i] = (live && first + i < n) ? load1<kBF16>(src, first + i) : 0.0f;
+  }
+  // Step 2: block absmax (exact; max is order-free)
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(w[i]));
+#pragma unroll
+  for (int off = 1; off < kL; off <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+
+  // Step 3: nearest code of RN(w / a); an all-zero block takes the zero code (7)
+  const bool zero = !(a > 0.0f);
+  const bool exact = !zero && a < kTinyScale;      // 1/a could overflow: divide exactly
+  const float r = __frcp_rn(zero ? 1.0f : a);
+  uint32_t c[16];
+  float gap = 1.0f;
+  if (kFp4) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) c[i] = code_fast_fp4(entry, __fmul_rn(w[i], r), gap);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) code_fast_pair(entry, w[i], w[i + 1], r, gap, c[i], c[i + 1]);
+  }
+  if (exact || gap <= kNearThreshold) {  // rare: redo this lane's 16 elements with exact quotients
+#pragma unroll
+    for (int i = 0; i < 16; ++i) c[i] = (uint32_t)(kFp4 ? code_exact_fp4(w[i], a) : code_exact(w[i], a));
+  }
+  // Step 4: element 2j -> high nibble of byte j; an all-zero block is all zero codes (NF4 7, FP4 +0)
+  uint32_t lo = pack8(c, 0), hi = pack8(c, 8);
+  if (zero) lo = hi = kFp4 ? 0u : 0x77777777u;
+  if (!live) return;
+  if (b < nfull) {
+    *reinterpret_cast<uint2*>(packed + first / 2) = make_uint2(lo, hi);
+  } else {
+    // short block: write only bytes holding real elements; an odd tail keeps
+    // the zero code (NF4 7, FP4 +0) in its low nibble
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int64_t e = first + 2 * j;  // element in the high nibble
+      if (e < n) {
+        uint8_t v = (uint8_t)((j < 4 ? lo : hi) >> (8 * (j & 3)));
+        if (e + 1 >= n) v = (uint8_t)((v & 0xf0u) | (kFp4 ? 0x0u : 0x7u));
+        packed[first / 2 + j] = v;
+      }
+    }
+  }
+  if (sub == 0) absmax[b] = a;
+}
+
 template <bool kBF16, bool kFp4, int kL>
 __global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ src, int64_t n,
                                                        uint8_t* __restrict__ packed,
@@ -124,7 +220,6 @@ __global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ 
   // kL lanes own one block of kB = 16 kL elements, 16 consecutive elements each
   constexpr int kB = 16 * kL;
   constexpr int kPerWarp = 32 / kL;                          // blocks per warp and iteration
-  const int sub = lane & (kL - 1);                           // which 16 of the block
   const int64_t nfull = n / kB;
   const int64_t nblocks = (n + kB - 1) / kB;
   const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -132,94 +227,52 @@ __global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ 
 
   // raw 16-element slices, one iteration ahead: the next slice's loads are in
   // flight while this one is coded
-  using Raw = uint4[kBF16 ? 2 : 4];
-  auto fetch = [&](int64_t wb, Raw& raw) {
-    const int64_t b = wb + lane / kL;
-    if (b < nfull) {
-      const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(src) +
-                                                      (b * kB + sub * 16) * (kBF16 ? 2 : 4));
-#pragma unroll
-      for (int i = 0; i < (kBF16 ? 2 : 4); ++i) raw[i] = __ldcs(p + i);
-    }
-  };
-  Raw cur, nxt;
+  Raw<kBF16> cur, nxt;
   int64_t wb = warp_id * kPerWarp;
   pdl_wait();
-  if (wb < nblocks) fetch(wb, cur);
+  if (wb < nblocks) fetch<kBF16, kL>(src, nfull, wb, lane, cur);
   for (; wb < nblocks; wb += warps_total * kPerWarp) {  // uniform per warp
-    if (wb + warps_total * kPerWarp < nblocks) fetch(wb + warps_total * kPerWarp, nxt);
-    const int64_t b = wb + lane / kL;
-    const bool live = b < nblocks;
-    const int64_t first = b * kB + sub * 16;
-    float w[16];
-    if (live && b < nfull) {
-      if (kBF16) {
-        const uint32_t u[8] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w, cur[1].x, cur[1].y, cur[1].z, cur[1].w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          w[2 * i] = bf16_lo_to_f32(u[i]);
-          w[2 * i + 1] = bf16_hi_to_f32(u[i]);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint4 v = cur[(kBF16 ? 0 : i)];
-          w[4 * i] = __uint_as_float(v.x);
-          w[4 * i + 1] = __uint_as_float(v.y);
-          w[4 * i + 2] = __uint_as_float(v.z);
-          w[4 * i + 3] = __uint_as_float(v.w);
-        }
-      }
-    } else {  // short last block (or no block): missing elements read as 0
-#pragma unroll
-      for (int i = 0; i < 16; ++i) w[i] = (live && first + i < n) ? load1<kBF16>(src, first + i) : 0.0f;
-    }
-    // Step 2: block absmax (exact; max is order-free)
-    float a = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(w[i]));
-#pragma unroll
-    for (int off = 1; off < kL; off <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
-
-    // Step 3: nearest code of RN(w / a); an all-zero block takes the zero code (7)
-    const bool zero = !(a > 0.0f);
-    const bool exact = !zero && a < kTinyScale;      // 1/a could overflow: divide exactly
-    const float r = __frcp_rn(zero ? 1.0f : a);
-    uint32_t c[16];
-    float gap = 1.0f;
-    if (kFp4) {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) c[i] = code_fast_fp4(entry, __fmul_rn(w[i], r), gap);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 16; i += 2) code_fast_pair(entry, w[i], w[i + 1], r, gap, c[i], c[i + 1]);
-    }
-    if (exact || gap <= kNearThreshold) {  // rare: redo this lane's 16 elements with exact quotients
-#pragma unroll
-      for (int i = 0; i < 16; ++i) c[i] = (uint32_t)(kFp4 ? code_exact_fp4(w[i], a) : code_exact(w[i], a));
-    }
-    // Step 4: element 2j -> high nibble of byte j; an all-zero block is all zero codes (NF4 7, FP4 +0)
-    uint32_t lo = pack8(c, 0), hi = pack8(c, 8);
-    if (zero) lo = hi = kFp4 ? 0u : 0x77777777u;
+    if (wb + warps_total * kPerWarp < nblocks) fetch<kBF16, kL>(src, nfull, wb + warps_total * kPerWarp, lane, nxt);
+    code_slice<kBF16, kFp4, kL>(entry, lane, wb, src, n, nfull, nblocks, packed, absmax, cur);
 #pragma unroll
     for (int i = 0; i < (kBF16 ? 2 : 4); ++i) cur[i] = nxt[i];
-    if (!live) continue;
-    if (b < nfull) {
-      *reinterpret_cast<uint2*>(packed + first / 2) = make_uint2(lo, hi);
+  }
+}
+
+// Several tensors of one dtype and block size: their blocks, each tensor's rounded up to whole warp iterations,
+// form one sequence that the warps walk as above (a warp's tensor index only moves forward).
+template <bool kBF16, bool kFp4, int kL>
+__global__ void __launch_bounds__(256) quantize_many_kernel(const __grid_constant__ QuantManyParams p) {
+  pdl_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const uint32_t entry = kFp4 ? c_q16[lane & 15] : c_q32[lane];
+  constexpr int kB = 16 * kL;
+  constexpr int kPerWarp = 32 / kL;
+  const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
+  int64_t W = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);  // warp iteration in the sequence
+  pdl_wait();
+  if (W >= p.iters) return;
+  int t = 0;
+  while (t + 1 < p.count && p.item[t + 1].w0 <= W) ++t;
+  Raw<kBF16> cur, nxt;
+  fetch<kBF16, kL>(p.item[t].src, p.item[t].n / kB, (W - p.item[t].w0) * kPerWarp, lane, cur);
+  while (W < p.iters) {
+    const QuantItem& it = p.item[t];
+    const int64_t wb = (W - it.w0) * kPerWarp;
+    W += warps_total;
+    if (W < p.iters) {
+      int tn = t;
+      while (tn + 1 < p.count && p.item[tn + 1].w0 <= W) ++tn;
+      fetch<kBF16, kL>(p.item[tn].src, p.item[tn].n / kB, (W - p.item[tn].w0) * kPerWarp, lane, nxt);
+      code_slice<kBF16, kFp4, kL>(entry, lane, wb, it.src, it.n, it.n / kB, (it.n + kB - 1) / kB, it.packed,
+                                  it.absmax, cur);
+      t = tn;
     } else {
-      // short block: write only bytes holding real elements; an odd tail keeps
-      // the zero code (NF4 7, FP4 +0) in its low nibble
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int64_t e = first + 2 * j;  // element in the high nibble
-        if (e < n) {
-          uint8_t v = (uint8_t)((j < 4 ? lo : hi) >> (8 * (j & 3)));
-          if (e + 1 >= n) v = (uint8_t)((v & 0xf0u) | (kFp4 ? 0x0u : 0x7u));
-          packed[first / 2 + j] = v;
-        }
-      }
+      code_slice<kBF16, kFp4, kL>(entry, lane, wb, it.src, it.n, it.n / kB, (it.n + kB - 1) / kB, it.packed,
+                                  it.absmax, cur);
     }
-    if (sub == 0) absmax[b] = a;
+#pragma unroll
+    for (int i = 0; i < (kBF16 ? 2 : 4); ++i) cur[i] = nxt[i];
   }
 }
 
@@ -253,7 +306,49 @@ cudaError_t launch_blocks(const void* src, int64_t n, int blocksize, uint8_t* pa
   }
 }
 
+template <bool kBF16, bool kFp4, int kL>
+cudaError_t launch_many_one(QuantManyParams& p, cudaStream_t stream, int num_sms) {
+  constexpr int kPerWarp = 32 / kL;
+  int64_t iters = 0;
+  for (int i = 0; i < p.count; ++i) {
+    p.item[i].w0 = iters;
+    iters += (p.item[i].n + 16 * kL * kPerWarp - 1) / (16 * kL * kPerWarp);
+  }
+  p.iters = iters;
+  int64_t grid = (iters + 7) / 8;  // 8 warps per CTA
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_many_kernel<kBF16, kFp4, kL>, 256, 0) !=
+          cudaSuccess || occ < 1)
+    occ = 1;
+  const int64_t cap = (int64_t)num_sms * occ;
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  const cudaError_t e = launch_pdl(quantize_many_kernel<kBF16, kFp4, kL>, dim3((unsigned)grid), dim3(256), 0, stream, p);
+  count_launches(1);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+template <bool kBF16, bool kFp4>
+cudaError_t launch_many_blocks(QuantManyParams& p, int blocksize, cudaStream_t stream, int num_sms) {
+  switch (blocksize) {
+    case 32: return launch_many_one<kBF16, kFp4, 2>(p, stream, num_sms);
+    case 64: return launch_many_one<kBF16, kFp4, 4>(p, stream, num_sms);
+    case 128: return launch_many_one<kBF16, kFp4, 8>(p, stream, num_sms);
+    case 256: return launch_many_one<kBF16, kFp4, 16>(p, stream, num_sms);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_quantize_many(QuantManyParams& p, bool bf16, int blocksize, int book, cudaStream_t stream,
+                                 int num_sms) {
+  if (bf16)
+    return book ? launch_many_blocks<true, true>(p, blocksize, stream, num_sms)
+                : launch_many_blocks<true, false>(p, blocksize, stream, num_sms);
+  return book ? launch_many_blocks<false, true>(p, blocksize, stream, num_sms)
+              : launch_many_blocks<false, false>(p, blocksize, stream, num_sms);
+}
 
 cudaError_t launch_quantize(const void* src, bool bf16, int64_t n, int blocksize, uint8_t* packed, float* absmax,
                             int book, cudaStream_t stream, int num_sms) {

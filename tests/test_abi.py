@@ -101,6 +101,16 @@ def test_host_validation_before_cuda(lib):
         E["NF4_ERR_INVALID_ARG"]
     assert dqm(one(0x1000), nb(0), 1, 256, 0, one(0x2000), one(0x3000), one(0x4000), 0x5000, 4096, s) == E["NF4_OK"]
     assert lib.nf4_double_quant_many_workspace_bytes(3) == 3 * 128
+    qm = lib.nf4_quantize_many
+    assert qm(one(0x1000), nb(10), 0, 0, 64, 0, one(0x2000), one(0x3000), s) == E["NF4_ERR_INVALID_ARG"]
+    assert qm(one(0x1000), nb(10), 257, 0, 64, 0, one(0x2000), one(0x3000), s) == E["NF4_ERR_INVALID_ARG"]
+    assert qm(one(0x1000), nb(10), 1, 7, 64, 0, one(0x2000), one(0x3000), s) == E["NF4_ERR_INVALID_ARG"]
+    assert qm(one(0x1000), nb(10), 1, 0, 48, 0, one(0x2000), one(0x3000), s) == E["NF4_ERR_UNSUPPORTED"]
+    assert qm(one(0x1000), nb(10), 1, 0, 64, 9, one(0x2000), one(0x3000), s) == E["NF4_ERR_INVALID_ARG"]
+    assert qm(one(0x1000, 0x1008), nb(10, 10), 2, 0, 64, 0, one(0x2000, 0x2100), one(0x3000, 0x3100), s) == \
+        E["NF4_ERR_MISALIGNED"]  # second source misaligned
+    assert qm(one(0x1000), nb(-1), 1, 0, 64, 0, one(0x2000), one(0x3000), s) == E["NF4_ERR_INVALID_ARG"]
+    assert qm(one(0x1000), nb(0), 1, 0, 64, 0, one(0x2000), one(0x3000), s) == E["NF4_OK"]
     assert lib.nf4_double_quant_many_workspace_bytes(0) == 0 and lib.nf4_double_quant_many_workspace_bytes(257) == 0
     # weight descriptor checks
     w = weight(bs=48)
