@@ -12,7 +12,7 @@ over enough independent copies that every step's working set is cold in the
 126 MB L2.
 
 Beside the step, `configs` reports every workload of the reference configs, each
-leg timed from its own CUDA graph of K launches over inputs rotating through at
+leg timed from its own CUDA graph of max(K, 64) launches over inputs rotating through at
 least 3x the L2 (or larger than it), with its own roofline fraction:
   1  fp32 1024x1024 quantize and dequantize (fp32 out), no double quant
   2  bf16 4096x4096 quantize, double quant E4M3 and INT8
@@ -294,8 +294,9 @@ def run_ours(args):
         return g
 
     def time_calls(calls, n=None, launches_per_call=1):
-        """device ms per call: a warm replay, then a timed replay of a graph of n calls rotating over the sets"""
-        n = n or args.steps
+        """device ms per call: a warm replay, then a timed replay of a graph of n calls rotating over the sets
+        (64 at least, so that the graph launch's own fixed cost is a small part of each call's share)"""
+        n = n or max(args.steps, 64)
         for c in calls[:3]:
             c()
         g = graph_of(calls, n)
@@ -663,7 +664,7 @@ def run_ours(args):
         "gpu_launches": int(launches),
         "gpu_launches_configs": int(cfg_launches),
         "launch": ("the K timed steps captured in one CUDA graph, launches chained with programmatic dependent "
-                   "launch; every per-kernel and per-config figure from one graph of K launches of that call over "
+                   "launch; every per-kernel and per-config figure from one graph of max(K, 64) launches of that call over "
                    "rotating input sets; e2e leg launches eagerly, copies in, library calls and copies out on three "
                    "streams overlapping across steps"),
         "clocks": clocks,

@@ -2,10 +2,13 @@
 
     python -m qlora_block_absmax_b200.run OP [--rows R] [--cols C] [--batch B] [--m M] [--iters N] [--fp4]
 
-OP: quantize | double_quant | dequantize | gemv | gemv_grouped | gemv_stream | gemm | gemm_dx | gemm_lora
+OP: quantize | double_quant | dequantize | gemv | gemv_grouped | gemv_stream | gemm | gemm_dx | gemm_lora |
+    quantize_many | double_quant_many
 Weights: bf16 ~N(0, 0.02) from the device generator (seed 1010), NF4 (or FP4 with --fp4) with E4M3 double quant;
 activations bf16 ~N(0, 1) (seed 1013).  gemv_stream runs one decoder layer of the 8B shape (7 weights) in one
-launch; gemv_grouped runs q, k, v of that layer (4096, 1024, 1024 x 4096) on one x in one launch.  Useful to look
+launch; gemv_grouped runs q, k, v of that layer (4096, 1024, 1024 x 4096) on one x in one launch;
+quantize_many quantizes that layer's 7 weights in one launch and double_quant_many double-quantizes their absmax
+arrays in one call.  Useful to look
 at one kernel in isolation (for instance under a profiler); prints one line per call
 with the device time of the last iteration.
 """
@@ -22,7 +25,7 @@ from qlora_block_absmax_b200 import synth
 def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("op", choices=["quantize", "double_quant", "dequantize", "gemv", "gemv_grouped", "gemv_stream",
-                                   "gemm", "gemm_dx", "gemm_lora"])
+                                   "gemm", "gemm_dx", "gemm_lora", "quantize_many", "double_quant_many"])
     ap.add_argument("--rows", type=int, default=4096)
     ap.add_argument("--cols", type=int, default=4096)
     ap.add_argument("--batch", type=int, default=1)
@@ -54,6 +57,17 @@ def main() -> None:
         qkv = [nf4.quantize_weight(synth.normal_weights_device((r, 4096), synth.layer_seed(0, p), device=dev),
                                    quant_type=qt) for p, (_, r, _) in enumerate(synth.LLAMA8B_LAYER[:3])]
         call = lambda: nf4.gemv_grouped(qkv, x)  # noqa: E731
+    elif a.op in ("quantize_many", "double_quant_many"):
+        srcs = [synth.normal_weights_device((r, c), synth.layer_seed(0, p), device=dev).reshape(-1)
+                for p, (_, r, c) in enumerate(synth.LLAMA8B_LAYER)]
+        outs = nf4.quantize_many(srcs)
+        if a.op == "quantize_many":
+            call = lambda: nf4.quantize_many(srcs, outs=outs)  # noqa: E731
+        else:
+            absmaxes = [o[1] for o in outs]
+            ws = torch.zeros(nf4._lib.load().nf4_double_quant_many_workspace_bytes(len(srcs)), dtype=torch.uint8,
+                             device=dev)
+            call = lambda: nf4.double_quant_many(absmaxes, "e4m3", workspace=ws)  # noqa: E731
     elif a.op == "gemv_stream":
         ws, xs = [], []
         acts = [synth.activations_device((a.batch, c), 3300 + j, device=dev) for j, c in enumerate((4096, 14336))]
