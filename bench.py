@@ -12,7 +12,7 @@ over enough independent copies that every step's working set is cold in the
 126 MB L2.
 
 Beside the step, `configs` reports every workload of the reference configs, each
-leg timed from its own CUDA graph of max(K, 64) launches over inputs rotating through at
+leg timed from its own CUDA graph of K to 64 launches (about 2 ms of work) over inputs rotating through at
 least 3x the L2 (or larger than it), with its own roofline fraction:
   1  fp32 1024x1024 quantize and dequantize (fp32 out), no double quant
   2  bf16 4096x4096 quantize, double quant E4M3 and INT8
@@ -294,11 +294,19 @@ def run_ours(args):
         return g
 
     def time_calls(calls, n=None, launches_per_call=1):
-        """device ms per call: a warm replay, then a timed replay of a graph of n calls rotating over the sets
-        (64 at least, so that the graph launch's own fixed cost is a small part of each call's share)"""
-        n = n or max(args.steps, 64)
+        """device ms per call: a warm replay, then a timed replay of a graph of n calls rotating over the sets.
+        Short calls get up to 64 per graph (the graph launch's own fixed cost then is a small part of each call's
+        share) while a graph stays near 2 ms of work, so a long call is still timed as a burst."""
         for c in calls[:3]:
             c()
+        if n is None:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            calls[3 % len(calls)]()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            n = max(args.steps, min(64, int(2.0 / max(e0.elapsed_time(e1), 1e-3))))
         g = graph_of(calls, n)
         g.replay()
         barrier()
@@ -664,7 +672,7 @@ def run_ours(args):
         "gpu_launches": int(launches),
         "gpu_launches_configs": int(cfg_launches),
         "launch": ("the K timed steps captured in one CUDA graph, launches chained with programmatic dependent "
-                   "launch; every per-kernel and per-config figure from one graph of max(K, 64) launches of that call over "
+                   "launch; every per-kernel and per-config figure from one graph of K to 64 launches (about 2 ms) of that call over "
                    "rotating input sets; e2e leg launches eagerly, copies in, library calls and copies out on three "
                    "streams overlapping across steps"),
         "clocks": clocks,
@@ -746,8 +754,8 @@ def model_config(args, nf4, synth, dev, time_calls, peaks):
 # kernels; gemm_lora: the down map and the GEMM), from the captures summarised in profiles/ (ncu flushes the caches
 # before each replayed launch, so these are cold-read figures); an entry is removed whenever its kernel changes
 # after the capture
-TRAFFIC = {"quantize": 33579264, "double_quant": 2136576, "dequantize": 8688896, "gemv": 8682496, "gemm": 10823424,
-           "gemm_dx": 10819328, "gemm_lora": 13227264, "gemv_grouped": 13010432}
+TRAFFIC = {"quantize": 33576448, "double_quant": 2161664, "dequantize": 8688896, "gemv": 8681984, "gemm": 10823424,
+           "gemm_dx": 10819328, "gemm_lora": 13227264, "gemv_grouped": 13011200}
 
 
 def oracle_table(args):
